@@ -1,0 +1,127 @@
+"""The CPU oracle against its pins (no GPU)."""
+
+import numpy as np
+import pytest
+
+import oracle
+import pins
+from sparse_linear_layers_fwd_b200 import synth
+
+
+def test_gamma_constant():
+    pins.check_gamma_constant(oracle)
+
+
+def test_gamma_floor():
+    pins.check_gamma_floor(oracle)
+
+
+def test_gamma_subnormals():
+    pins.check_gamma_subnormal_scale(oracle)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_gamma_exact_mean_random(seed):
+    w = synth.latent_weights(64, 256, seed=seed)
+    pins.check_gamma_exact_mean(oracle, w)
+    pins.check_gamma_fsum(oracle, w)
+
+
+def test_gamma_wide_exponent_range():
+    rng = np.random.default_rng(3)
+    w = rng.integers(0, 0x7F7F, size=(16, 64)).astype(np.uint16)   # finite, any exponent
+    w |= (rng.integers(0, 2, size=w.shape).astype(np.uint16) << 15)
+    pins.check_gamma_exact_mean(oracle, w)
+    pins.check_gamma_fsum(oracle, w)
+
+
+def test_gamma_gaussian():
+    pins.check_gamma_gaussian(oracle)
+
+
+def test_mask_hand():
+    pins.check_mask_hand(oracle)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_mask_bruteforce(seed):
+    pins.check_mask_bruteforce(oracle, seed)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8), (6, 8), (8, 16), (8, 8)])
+def test_mask_invariants(nm):
+    w = synth.latent_weights(32, 512, seed=4)
+    pins.check_mask_invariants(oracle, w, *nm)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (8, 8)])
+def test_codes_exact(nm):
+    w = synth.latent_weights(64, 512, seed=5)
+    pins.check_codes_exact(oracle, w, *nm)
+
+
+def test_codes_zero_fraction():
+    pins.check_codes_zero_fraction(oracle)
+
+
+def test_codes_constant():
+    pins.check_codes_constant(oracle)
+
+
+def test_pack_hand():
+    pins.check_pack_hand(oracle)
+
+
+def test_pack_random():
+    pins.check_pack_random(oracle)
+
+
+def test_acts_layer_small():
+    pins.check_acts(oracle, synth.layer_small()["x"])
+
+
+def test_acts_heavy_tail():
+    pins.check_acts(oracle, synth.activations(8, 896, seed=1, heavy_tail_channels=14))
+
+
+def test_acts_zero_row():
+    pins.check_acts_zero_row(oracle)
+
+
+def test_acc_bruteforce():
+    pins.check_acc_bruteforce(oracle)
+
+
+def test_acc_extremes():
+    pins.check_acc_extremes(oracle)
+
+
+def test_dequant():
+    pins.check_dequant(oracle)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 8)])
+def test_layer_small_vs_float(nm):
+    d = synth.layer_small()
+    pins.check_layer_vs_float(oracle, d["w"], d["x"], *nm)
+
+
+def test_sampled_matches_full():
+    d = synth.layer_small()
+    cb, mb, g, mask, dense = oracle.quantize_weights(d["w"], 2, 4)
+    q, s = oracle.quantize_acts(d["x"])
+    y, acc = oracle.bitlinear(q, s, cb, mb, g, 256, 2, 4)
+    rng = np.random.default_rng(0)
+    ti = rng.integers(0, 16, 50)
+    ni = rng.integers(0, 256, 50)
+    ys, accs = oracle.bitlinear_at(q, s, dense, g, ti, ni)
+    assert np.array_equal(accs, acc[ti, ni]) and np.array_equal(ys, y[ti, ni])
+
+
+def test_layer_small_zero_fraction_reported():
+    """Synthetic N(0, 0.02) weights: ~31% ternary zeros before masking, not
+    the 42.3% of the trained model in Figure 1 of the Sparse-BitNet page."""
+    w = synth.latent_weights(256, 256, seed=0)
+    g = oracle.absmean_gamma(w)
+    c = oracle.ternary_codes(w, g, np.ones(w.shape, bool))
+    assert 0.29 < float(np.mean(c == 0)) < 0.33
