@@ -1,0 +1,184 @@
+/*
+ * sbn.h -- C ABI of libsbn: the Sparse-BitNet BitLinear forward on B200 (sm_100a).
+ *
+ * The BitLinear forward ("Microsoft BitNet 1.58: The Era of 1-Bit Large
+ * Language Models", section "The BitLinear Layer") quantizes activations to
+ * INT8 with an absmax scale, quantizes the latent weights to ternary
+ * {-1, 0, +1} with an absmean scale, contracts the two in integer arithmetic
+ * and dequantizes the result. Sparse-BitNet ("Sparse-BitNet: 1.58-bit LLMs
+ * are Naturally Friendly to Semi-Structured Sparsity", Abstract) adds a
+ * dynamic N:M magnitude mask on the latent weights, recomputed every forward.
+ *
+ * Three calls make the path:
+ *   sbn_quantize_weights : mask + absmean ternary + pack   (latent bf16 W -> packed)
+ *   sbn_quantize_acts    : per-token absmax INT8           (bf16 X -> Xq, s)
+ *   sbn_bitlinear        : packed W x Xq, int32 accumulate, dequantize to bf16
+ *
+ * Conventions shared by every call
+ *   - Sizes: T tokens, K in-features, N_out out-features; n:m keeps n of every
+ *     m consecutive weights along K.
+ *   - Layouts (row-major): X [T, K] bf16; W [N_out, K] bf16 (nn.Linear
+ *     convention); Xq [T, K] int8; x_scale [T] fp32; Y [T, N_out] bf16;
+ *     acc [T, N_out] int32.
+ *   - Every pointer argument named "device" is device memory of the current
+ *     CUDA device, owned by the caller, 16-byte aligned. The library never
+ *     allocates or frees memory and never synchronizes, except
+ *     sbn_get_device_error. All work is enqueued on `stream` (a cudaStream_t;
+ *     NULL means the legacy default stream) and is asynchronous.
+ *   - Argument errors are returned synchronously before anything is enqueued;
+ *     outputs are then untouched. A failed launch returns SBN_ERR_CUDA.
+ *     Device-side failures (a bounded wait that ran out) are recorded in a
+ *     device error word and reported by sbn_get_device_error.
+ *   - Non-finite inputs (inf, NaN) give unspecified outputs.
+ *
+ * Packed weight format (canonical; produced by sbn_quantize_weights and read
+ * by sbn_bitlinear):
+ *   codes [N_out, codes_row_bytes]: per row, the ternary values of the kept
+ *     positions in ascending k; value j sits in bits 2*(j%4)..2*(j%4)+1 of
+ *     byte j/4, encoded 0 -> 00, +1 -> 01, -1 -> 11 (four 2-bit values per
+ *     byte, as in the section "bitnet.cpp: Matrix-Free Inference" of the
+ *     octagono page); codes_row_bytes = ceil(K*n/m/4) rounded up to 16, the
+ *     padding bytes are zero.
+ *   meta [N_out, meta_row_bytes]: per row, bit k%8 of byte k/8 is 1 iff
+ *     position k is kept; meta_row_bytes = K/8 rounded up to 16; absent
+ *     (0 bytes, pointer may be NULL) when n == m.
+ *   gamma: one fp32 device scalar, the absmean scale.
+ *
+ * Supported patterns: m in {4, 8, 16} and 1 <= n <= m with 4*n divisible by
+ * m (1:4 2:4 3:4 4:4, 2:8 4:8 6:8 8:8, 4:16 8:16 12:16 16:16). Shapes: K a
+ * multiple of 128; T, N_out >= 1; T*K, N_out*K and T*N_out below 2^31.
+ */
+#ifndef SBN_H
+#define SBN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SBN_OK = 0,
+  SBN_ERR_NULL = 1,      /* a required pointer is NULL */
+  SBN_ERR_SHAPE = 2,     /* a size is out of the supported range */
+  SBN_ERR_PATTERN = 3,   /* unsupported n:m */
+  SBN_ERR_ALIGN = 4,     /* a pointer is not 16-byte aligned */
+  SBN_ERR_WORKSPACE = 5, /* the workspace is smaller than required */
+  SBN_ERR_CUDA = 6,      /* a CUDA runtime call or kernel launch failed */
+  SBN_ERR_TIMEOUT = 7,   /* a bounded device-side wait gave up */
+  SBN_ERR_DEVICE = 8     /* the current device is not sm_100 */
+} sbn_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sbn_status_string(sbn_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int sbn_version(void);
+
+/* Bytes of one packed code row, of the whole codes array, of one meta row and
+ * of the whole meta array for the given shape and pattern (0 for an
+ * unsupported pattern or shape). */
+size_t sbn_codes_row_bytes(int32_t k, int32_t n, int32_t m);
+size_t sbn_codes_bytes(int32_t n_out, int32_t k, int32_t n, int32_t m);
+size_t sbn_meta_row_bytes(int32_t k, int32_t n, int32_t m);
+size_t sbn_meta_bytes(int32_t n_out, int32_t k, int32_t n, int32_t m);
+
+/* Device workspace that sbn_quantize_weights needs (exact-sum bins and the
+ * derived threshold), in bytes. */
+size_t sbn_quantize_weights_workspace_bytes(int32_t n_out, int32_t k);
+
+/*
+ * sbn_quantize_weights -- dynamic N:M mask, absmean ternary codes, packing.
+ *
+ * Defining passages: the absmean quantizer ("BitNet b1.58: How Ternary
+ * Weights Cut LLM Memory by 82% Without Losing Accuracy", section "How
+ * ternary quantization works during training": divide W by its mean absolute
+ * value, round, clamp to [-1, 1]); the N:M magnitude mask (Sparse-BitNet page,
+ * Abstract, and Figure 6: the per-block threshold t = |w|_(N+1)).
+ *
+ *   w_bf16     device, [n_out, k] bf16, read only.
+ *   codes      device, sbn_codes_bytes(n_out, k, n, m) bytes, written.
+ *   meta       device, sbn_meta_bytes(...) bytes, written; NULL allowed iff n == m.
+ *   gamma      device, one float, written:
+ *              gamma = max(fl32(fl64(S) / (n_out*k)), 1e-5) where S is the exact
+ *              sum of |w| and fl64(S) its correctly rounded double.
+ *   workspace  device, at least sbn_quantize_weights_workspace_bytes() bytes,
+ *              scratch owned by the caller; its contents on entry do not matter
+ *              and are overwritten. Calls that share a workspace must not
+ *              overlap in time (same stream, or ordered by events).
+ *
+ * Mask: within every group of m consecutive positions of a row, the n
+ * positions of largest |w| are kept; equal magnitudes keep the lower index.
+ * Codes: clamp(rint(fl32(w / gamma)), -1, 1) (IEEE fp32 division, round half
+ * to even) at kept positions; pruned positions are simply absent.
+ * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN,
+ * SBN_ERR_WORKSPACE (returned before any work is enqueued); SBN_ERR_CUDA.
+ */
+sbn_status sbn_quantize_weights(const void* w_bf16, int32_t n_out, int32_t k,
+                                int32_t n, int32_t m, uint8_t* codes,
+                                uint8_t* meta, float* gamma, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
+ * sbn_quantize_acts -- per-token absmax INT8 activations.
+ *
+ * Defining passage: "The BitLinear Layer" (octagono page), second operation:
+ * activations are quantized from bf16 to INT8 with absmax scaling and the
+ * scale is kept for dequantization; the promptingindex page (same section as
+ * above) makes the scale per token.
+ *
+ *   x_bf16   device, [t, k] bf16, read only (k a multiple of 16).
+ *   xq       device, [t, k] int8, written:
+ *            q = clamp(rint(fl32(x * fl32(127 / s_t))), -127, 127).
+ *   x_scale  device, [t] fp32, written: s_t = max(max_k |x_tk|, 1e-5).
+ * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_ALIGN; SBN_ERR_CUDA.
+ */
+sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k,
+                             int8_t* xq, float* x_scale, void* stream);
+
+/*
+ * sbn_bitlinear -- INT8 x ternary contraction with int32 accumulation and
+ * dequantization to bf16.
+ *
+ * Defining passage: "The BitLinear Layer" (octagono page), fourth and fifth
+ * operations: the product runs on the quantized values only (additions,
+ * subtractions, zero-skips) and is rescaled by the preserved scales.
+ *
+ *   xq, x_scale   device, from sbn_quantize_acts ([t, k] int8, [t] fp32).
+ *   codes, meta,  device, from sbn_quantize_weights for the same n_out, k, n, m
+ *   gamma         (meta NULL allowed iff n == m).
+ *   y_bf16        device, [t, n_out] bf16, written:
+ *                 y = bf16_rne(acc * gamma * s_t / 127) evaluated in fp32, where
+ *                 acc[t, o] = sum over kept k of xq[t, k] * code[o, k] (exact int32).
+ * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN;
+ * SBN_ERR_CUDA.
+ */
+sbn_status sbn_bitlinear(const int8_t* xq, const float* x_scale, int32_t t,
+                         int32_t k, int32_t n_out, int32_t n, int32_t m,
+                         const uint8_t* codes, const uint8_t* meta,
+                         const float* gamma, void* y_bf16, void* stream);
+
+/*
+ * sbn_bitlinear_acc32 -- the same contraction, writing the exact int32
+ * accumulators acc [t, n_out] (device, row-major) instead of y. Meant for
+ * verification; same arguments and errors as sbn_bitlinear.
+ */
+sbn_status sbn_bitlinear_acc32(const int8_t* xq, int32_t t, int32_t k,
+                               int32_t n_out, int32_t n, int32_t m,
+                               const uint8_t* codes, const uint8_t* meta,
+                               int32_t* acc, void* stream);
+
+/*
+ * sbn_get_device_error -- synchronizes `stream`, then reads and clears the
+ * device error word of the current device. Returns SBN_OK, SBN_ERR_TIMEOUT
+ * (a bounded device wait gave up; the affected outputs are unspecified) or
+ * SBN_ERR_CUDA (the synchronization itself failed).
+ */
+sbn_status sbn_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBN_H */

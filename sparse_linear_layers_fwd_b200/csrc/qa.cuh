@@ -1,0 +1,92 @@
+// sbn_quantize_acts kernel: per-token absmax INT8 activations.
+//
+// "Microsoft BitNet 1.58: The Era of 1-Bit Large Language Models", section
+// "The BitLinear Layer", second operation (bf16 -> INT8 with absmax scaling,
+// scale preserved); per-token scale as on the promptingindex page, section
+// "How ternary quantization works during training".
+//
+// One CTA of 128 threads per token row. The row is held in registers
+// (MAXC 16-byte chunks per thread), so X is read from HBM exactly once:
+// max |x| (integer max of the 15 magnitude bits), one IEEE division for the
+// multiplier 127/s, then q = clamp(rint(x * mult), -127, 127).
+#pragma once
+
+#include "common.cuh"
+
+namespace sbn {
+
+constexpr int kQaThreads = 128;
+
+SBN_DEVFN uint32_t quant_pair(uint32_t wd, float mult) {
+  int q0 = __float2int_rn(__fmul_rn(__uint_as_float(wd << 16), mult));
+  int q1 = __float2int_rn(__fmul_rn(__uint_as_float(wd & 0xFFFF0000u), mult));
+  q0 = min(max(q0, -127), 127);
+  q1 = min(max(q1, -127), 127);
+  return ((uint32_t)q0 & 0xFFu) | (((uint32_t)q1 & 0xFFu) << 8);
+}
+
+SBN_DEVFN uint32_t mag_max8(const uint4& v) {
+  const uint32_t m0 = max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu);
+  const uint32_t m1 = max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu);
+  const uint32_t m2 = max(v.z & 0x7FFFu, (v.z >> 16) & 0x7FFFu);
+  const uint32_t m3 = max(v.w & 0x7FFFu, (v.w >> 16) & 0x7FFFu);
+  return max(max(m0, m1), max(m2, m3));
+}
+
+SBN_DEVFN uint2 quant8(const uint4& v, float mult) {
+  const uint32_t p0 = quant_pair(v.x, mult), p1 = quant_pair(v.y, mult);
+  const uint32_t p2 = quant_pair(v.z, mult), p3 = quant_pair(v.w, mult);
+  return make_uint2(p0 | (p1 << 16), p2 | (p3 << 16));
+}
+
+SBN_DEVFN float block_absmax_scale(uint32_t amax) {
+  __shared__ uint32_t s_red[kQaThreads / 32];
+  amax = __reduce_max_sync(0xffffffffu, amax);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  uint32_t m = s_red[0];
+#pragma unroll
+  for (int i = 1; i < kQaThreads / 32; ++i) m = max(m, s_red[i]);
+  return fmaxf(__uint_as_float(m << 16), 1e-5f);
+}
+
+// MAXC > 0: the row stays in registers. kc = K / 8 chunks of 16 bytes.
+template <int MAXC>
+__global__ void __launch_bounds__(kQaThreads)
+qa_kernel(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+  const size_t row = blockIdx.x;
+  const uint4* xr = x + row * kc;
+  uint4 v[MAXC];
+  uint32_t amax = 0u;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int idx = threadIdx.x + c * kQaThreads;
+    v[c] = (idx < kc) ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
+    amax = max(amax, mag_max8(v[c]));
+  }
+  const float s = block_absmax_scale(amax);
+  const float mult = __fdiv_rn(127.0f, s);
+  if (threadIdx.x == 0) scale[row] = s;
+  uint2* qr = xq + row * kc;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int idx = threadIdx.x + c * kQaThreads;
+    if (idx < kc) qr[idx] = quant8(v[c], mult);
+  }
+}
+
+// Rows too long for registers: two passes over the row (the second from L2).
+__global__ void __launch_bounds__(kQaThreads)
+qa_kernel_long(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+  const size_t row = blockIdx.x;
+  const uint4* xr = x + row * kc;
+  uint32_t amax = 0u;
+  for (int idx = threadIdx.x; idx < kc; idx += kQaThreads) amax = max(amax, mag_max8(__ldg(xr + idx)));
+  const float s = block_absmax_scale(amax);
+  const float mult = __fdiv_rn(127.0f, s);
+  if (threadIdx.x == 0) scale[row] = s;
+  uint2* qr = xq + row * kc;
+  for (int idx = threadIdx.x; idx < kc; idx += kQaThreads) qr[idx] = quant8(__ldg(xr + idx), mult);
+}
+
+}  // namespace sbn

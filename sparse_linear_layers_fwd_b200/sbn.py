@@ -1,0 +1,239 @@
+"""ctypes binding of libsbn (include/sbn.h): argument marshalling only.
+
+Every step of the BitLinear forward runs in libsbn's CUDA kernels; PyTorch
+only supplies device memory and the current stream. There is no CPU
+fallback: if ``libsbn.so`` is missing, loading it raises.
+
+    packed = quantize_weights(w_bf16, n=6, m=8)       # dynamic N:M mask + ternary + pack
+    xq, s = quantize_acts(x_bf16)                      # per-token absmax INT8
+    y = bitlinear(xq, s, packed)                       # INT8 x ternary -> bf16
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsbn.so")
+
+SBN_STATUS = {
+    0: "SBN_OK", 1: "SBN_ERR_NULL", 2: "SBN_ERR_SHAPE", 3: "SBN_ERR_PATTERN",
+    4: "SBN_ERR_ALIGN", 5: "SBN_ERR_WORKSPACE", 6: "SBN_ERR_CUDA",
+    7: "SBN_ERR_TIMEOUT", 8: "SBN_ERR_DEVICE",
+}
+
+_c_i32, _c_sz, _c_p = ctypes.c_int32, ctypes.c_size_t, ctypes.c_void_p
+
+# name -> (restype, argtypes), mirroring include/sbn.h
+PROTOTYPES = {
+    "sbn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "sbn_version": (ctypes.c_int, []),
+    "sbn_codes_row_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32]),
+    "sbn_codes_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32, _c_i32]),
+    "sbn_meta_row_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32]),
+    "sbn_meta_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32, _c_i32]),
+    "sbn_quantize_weights_workspace_bytes": (_c_sz, [_c_i32, _c_i32]),
+    "sbn_quantize_weights": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p,
+                                            _c_p, _c_p, _c_sz, _c_p]),
+    "sbn_quantize_acts": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p]),
+    "sbn_bitlinear": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
+                                     _c_p, _c_p, _c_p, _c_p]),
+    "sbn_bitlinear_acc32": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
+                                           _c_p, _c_p, _c_p]),
+    "sbn_get_device_error": (ctypes.c_int, [_c_p]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsbn.so (once). Raises ImportError if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m sparse_linear_layers_fwd_b200.build` (needs nvcc)")
+        cdll = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in PROTOTYPES.items():
+            fn = getattr(cdll, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = cdll
+    return _lib
+
+
+class SbnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().sbn_status_string(status).decode()
+        super().__init__(f"{where}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SbnError(status, where)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, what: str):
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+
+
+@dataclass
+class Pattern:
+    n: int
+    m: int
+
+
+@dataclass
+class PackedWeights:
+    """Packed ternary weights in the canonical format of include/sbn.h."""
+    codes: torch.Tensor            # uint8 [n_out, codes_row_bytes]
+    meta: Optional[torch.Tensor]   # uint8 [n_out, meta_row_bytes] or None (n == m)
+    gamma: torch.Tensor            # float32 [1]
+    n_out: int
+    k: int
+    n: int
+    m: int
+
+
+def codes_row_bytes(k: int, n: int, m: int) -> int:
+    return int(lib().sbn_codes_row_bytes(k, n, m))
+
+
+def meta_row_bytes(k: int, n: int, m: int) -> int:
+    return int(lib().sbn_meta_row_bytes(k, n, m))
+
+
+def workspace_bytes(n_out: int, k: int) -> int:
+    return int(lib().sbn_quantize_weights_workspace_bytes(n_out, k))
+
+
+def alloc_packed(n_out: int, k: int, n: int, m: int, device) -> PackedWeights:
+    cr, mr = codes_row_bytes(k, n, m), meta_row_bytes(k, n, m)
+    if cr == 0:
+        raise SbnError(3, "alloc_packed")
+    codes = torch.empty((n_out, cr), dtype=torch.uint8, device=device)
+    meta = torch.empty((n_out, mr), dtype=torch.uint8, device=device) if mr else None
+    gamma = torch.empty((1,), dtype=torch.float32, device=device)
+    return PackedWeights(codes, meta, gamma, n_out, k, n, m)
+
+
+def quantize_weights(w: torch.Tensor, n: int, m: int, out: Optional[PackedWeights] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None) -> PackedWeights:
+    """sbn_quantize_weights: N:M magnitude mask, absmean ternary codes, packing."""
+    _need(w, torch.bfloat16, "w")
+    n_out, k = w.shape
+    if out is None:
+        out = alloc_packed(n_out, k, n, m, w.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(n_out, k), dtype=torch.uint8, device=w.device)
+    st = lib().sbn_quantize_weights(_ptr(w), n_out, k, n, m, _ptr(out.codes), _ptr(out.meta),
+                                    _ptr(out.gamma), _ptr(workspace), workspace.numel(),
+                                    _stream_ptr(stream))
+    _check(st, "sbn_quantize_weights")
+    return out
+
+
+def quantize_acts(x: torch.Tensor, out_q: Optional[torch.Tensor] = None,
+                  out_s: Optional[torch.Tensor] = None, stream=None):
+    """sbn_quantize_acts: per-token absmax INT8. Returns (xq int8 [T,K], s fp32 [T])."""
+    _need(x, torch.bfloat16, "x")
+    t, k = x.shape
+    if out_q is None:
+        out_q = torch.empty((t, k), dtype=torch.int8, device=x.device)
+    if out_s is None:
+        out_s = torch.empty((t,), dtype=torch.float32, device=x.device)
+    st = lib().sbn_quantize_acts(_ptr(x), t, k, _ptr(out_q), _ptr(out_s), _stream_ptr(stream))
+    _check(st, "sbn_quantize_acts")
+    return out_q, out_s
+
+
+def bitlinear(xq: torch.Tensor, s: torch.Tensor, w: PackedWeights,
+              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """sbn_bitlinear: y[t, o] = bf16(acc * gamma * s_t / 127)."""
+    _need(xq, torch.int8, "xq")
+    _need(s, torch.float32, "s")
+    t, k = xq.shape
+    if k != w.k:
+        raise ValueError("K mismatch between activations and weights")
+    if out is None:
+        out = torch.empty((t, w.n_out), dtype=torch.bfloat16, device=xq.device)
+    st = lib().sbn_bitlinear(_ptr(xq), _ptr(s), t, k, w.n_out, w.n, w.m, _ptr(w.codes),
+                             _ptr(w.meta), _ptr(w.gamma), _ptr(out), _stream_ptr(stream))
+    _check(st, "sbn_bitlinear")
+    return out
+
+
+def bitlinear_acc32(xq: torch.Tensor, w: PackedWeights, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """sbn_bitlinear_acc32: the exact int32 accumulators [T, N_out]."""
+    _need(xq, torch.int8, "xq")
+    t, k = xq.shape
+    if out is None:
+        out = torch.empty((t, w.n_out), dtype=torch.int32, device=xq.device)
+    st = lib().sbn_bitlinear_acc32(_ptr(xq), t, k, w.n_out, w.n, w.m, _ptr(w.codes),
+                                   _ptr(w.meta), _ptr(out), _stream_ptr(stream))
+    _check(st, "sbn_bitlinear_acc32")
+    return out
+
+
+def get_device_error(stream=None) -> int:
+    """sbn_get_device_error: sync the stream, read and clear the device error word."""
+    return int(lib().sbn_get_device_error(_stream_ptr(stream)))
+
+
+class BitLinear(torch.nn.Module):
+    """BitLinear layer with a dynamic N:M mask on latent bf16 weights.
+
+    Every forward re-derives the packed ternary weights from the latent
+    weights (the mask is dynamic), quantizes the activations per token and
+    runs the integer contraction. No bias. Inference only (no autograd).
+    """
+
+    def __init__(self, in_features: int, out_features: int, n: int = 6, m: int = 8,
+                 device=None, weight: Optional[torch.Tensor] = None):
+        super().__init__()
+        if weight is None:
+            weight = torch.empty((out_features, in_features), dtype=torch.bfloat16, device=device)
+            torch.nn.init.normal_(weight, std=0.02)
+        self.weight = torch.nn.Parameter(weight, requires_grad=False)
+        self.n, self.m = n, m
+        self._ws = None
+        self._packed = None
+
+    def pack(self) -> PackedWeights:
+        w = self.weight.data
+        if self._packed is None or self._packed.codes.device != w.device:
+            self._packed = alloc_packed(w.shape[0], w.shape[1], self.n, self.m, w.device)
+            self._ws = torch.empty(workspace_bytes(*w.shape), dtype=torch.uint8, device=w.device)
+        return quantize_weights(w, self.n, self.m, out=self._packed, workspace=self._ws)
+
+    @torch.no_grad()
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        x2 = x.reshape(-1, x.shape[-1]).contiguous()
+        packed = self.pack()
+        xq, s = quantize_acts(x2)
+        y = bitlinear(xq, s, packed)
+        return y.reshape(*lead, packed.n_out)

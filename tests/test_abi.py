@@ -1,0 +1,125 @@
+"""The C ABI without a GPU: symbols, sizes and host-side validation."""
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+import torch
+
+import oracle
+
+HEADER = Path(__file__).resolve().parents[1] / "include" / "sbn.h"
+
+SUPPORTED = [(1, 4), (2, 4), (3, 4), (4, 4), (2, 8), (4, 8), (6, 8), (8, 8),
+             (4, 16), (8, 16), (12, 16), (16, 16)]
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sbn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for required in ["sbn_quantize_weights", "sbn_quantize_acts", "sbn_bitlinear"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(sbn_lib):
+    for name in declared_functions():
+        assert hasattr(sbn_lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    from sparse_linear_layers_fwd_b200 import sbn
+    assert set(declared_functions()) <= set(sbn.PROTOTYPES)
+
+
+def test_status_strings(sbn_lib):
+    for code in range(9):
+        assert sbn_lib.sbn_status_string(code).startswith(b"SBN_")
+    assert sbn_lib.sbn_version() >= 100
+
+
+@pytest.mark.parametrize("nm", SUPPORTED)
+@pytest.mark.parametrize("k", [128, 896, 2560, 11008])
+def test_row_bytes_match_oracle(sbn_lib, nm, k):
+    n, m = nm
+    assert sbn_lib.sbn_codes_row_bytes(k, n, m) == oracle.codes_row_bytes(k, n, m)
+    assert sbn_lib.sbn_meta_row_bytes(k, n, m) == oracle.meta_row_bytes(k, n, m)
+    assert sbn_lib.sbn_codes_bytes(7, k, n, m) == 7 * oracle.codes_row_bytes(k, n, m)
+
+
+@pytest.mark.parametrize("nm", [(3, 8), (5, 8), (7, 8), (0, 4), (5, 4), (2, 6), (1, 16), (8, 32)])
+def test_unsupported_patterns_report_zero_bytes(sbn_lib, nm):
+    assert sbn_lib.sbn_codes_row_bytes(256, *nm) == 0
+
+
+A = 0x10000          # a fake, 16-byte aligned device address (never dereferenced)
+MIS = 0x10008        # misaligned by 8
+
+
+def qw(lib, w=A, n_out=64, k=256, n=2, m=4, codes=A, meta=A, gamma=A, ws=A, wsb=4096):
+    return lib.sbn_quantize_weights(w, n_out, k, n, m, codes, meta, gamma, ws, wsb, None)
+
+
+def test_quantize_weights_validation(sbn_lib):
+    lib = sbn_lib
+    assert qw(lib, w=None) == 1
+    assert qw(lib, codes=None) == 1
+    assert qw(lib, meta=None) == 1               # meta required when n < m
+    assert qw(lib, gamma=None) == 1
+    assert qw(lib, ws=None) == 1
+    assert qw(lib, n=3, m=8) == 3
+    assert qw(lib, n=0, m=4) == 3
+    assert qw(lib, k=200) == 2                    # K not a multiple of 128
+    assert qw(lib, n_out=0) == 2
+    assert qw(lib, n_out=1 << 20, k=1 << 12) == 2  # N_out*K >= 2^31
+    assert qw(lib, w=MIS) == 4
+    assert qw(lib, codes=MIS) == 4
+    assert qw(lib, wsb=100) == 5
+
+
+def test_quantize_acts_validation(sbn_lib):
+    lib = sbn_lib
+    assert lib.sbn_quantize_acts(None, 4, 256, A, A, None) == 1
+    assert lib.sbn_quantize_acts(A, 0, 256, A, A, None) == 2
+    assert lib.sbn_quantize_acts(A, 4, 24, A, A, None) == 2
+    assert lib.sbn_quantize_acts(MIS, 4, 256, A, A, None) == 4
+
+
+def test_bitlinear_validation(sbn_lib):
+    lib = sbn_lib
+    ok = dict(xq=A, s=A, t=4, k=256, n_out=64, n=2, m=4, codes=A, meta=A, g=A, y=A)
+
+    def bl(**kw):
+        a = dict(ok, **kw)
+        return lib.sbn_bitlinear(a["xq"], a["s"], a["t"], a["k"], a["n_out"], a["n"], a["m"],
+                                 a["codes"], a["meta"], a["g"], a["y"], None)
+    assert bl(xq=None) == 1
+    assert bl(y=None) == 1
+    assert bl(meta=None) == 1
+    assert bl(meta=None, n=4, m=4) != 1          # dense needs no meta
+    assert bl(n=5, m=8) == 3
+    assert bl(t=0) == 2
+    assert bl(k=100) == 2
+    assert bl(xq=MIS) == 4
+    assert lib.sbn_bitlinear_acc32(A, 4, 256, 64, 2, 4, A, A, None, None) == 1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")
+def test_valid_arguments_without_gpu_fail_cleanly(sbn_lib):
+    # every argument is valid, so the call reaches the device check and stops there
+    assert qw(sbn_lib) in (6, 8)
+    assert sbn_lib.sbn_get_device_error(None) in (6, 8)
+
+
+def test_product_path_does_not_import_oracle():
+    pkg = Path(__file__).resolve().parents[1] / "sparse_linear_layers_fwd_b200"
+    for f in pkg.rglob("*.py"):
+        text = f.read_text()
+        assert "import oracle" not in text and "from oracle" not in text, f
+    for f in list(pkg.rglob("*.cu")) + list(pkg.rglob("*.cuh")):
+        assert "oracle" not in f.read_text(), f

@@ -1,0 +1,212 @@
+"""CUDA path against the oracle, element by element (needs a B200).
+
+Bar: bit-exact gamma, masks (meta), packed codes, INT8 activations, scales
+and int32 accumulators; bf16 outputs within 1e-2 relative.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from gpu_util import (assert_weights_exact, assert_y_close, full_parity, run_layer,
+                      run_quantize_weights, packed_to_numpy, to_dev_bf16, bf16_tensor_bits)
+from sparse_linear_layers_fwd_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+SUPPORTED = [(1, 4), (2, 4), (3, 4), (4, 4), (2, 8), (4, 8), (6, 8), (8, 8),
+             (4, 16), (8, 16), (12, 16), (16, 16)]
+SHAPES = [(1, 128, 1), (5, 384, 7), (17, 1024, 130), (33, 256, 64), (100, 512, 257)]
+
+
+@pytest.fixture(autouse=True)
+def _lib(sbn_lib, cuda_ok):
+    return sbn_lib
+
+
+def test_layer_small_full_parity():
+    d = synth.layer_small()
+    full_parity(d["w"], d["x"], d["n"], d["m"])
+
+
+@pytest.mark.parametrize("nm", SUPPORTED)
+@pytest.mark.parametrize("shape", SHAPES)
+def test_patterns_and_ragged_shapes(nm, shape):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=1, tag=f"p{nm}{shape}")
+    x = synth.activations(t, k, seed=1, tag=f"p{nm}{shape}", outlier_channels=2)
+    full_parity(w, x, *nm)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (8, 8)])
+def test_all_zero_weights(nm):
+    w = np.zeros((40, 256), np.uint16)
+    w[::3] = 0x8000                                      # negative zeros too
+    x = synth.activations(3, 256, seed=2)
+    g = full_parity(w, x, *nm)
+    assert g["gamma"] == np.float32(1e-5)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16)])
+def test_constant_weights_tie_everywhere(nm):
+    w = np.full((24, 384), 0x3C23, np.uint16)            # 0.00995..., all equal magnitude
+    w[1::2] ^= 0x8000                                    # alternate signs, same magnitude
+    x = synth.activations(9, 384, seed=3)
+    full_parity(w, x, *nm)
+
+
+def test_exact_half_ties_in_codes():
+    # half the weights 0.25, half 0.75 in magnitude: gamma = 0.5 exactly and
+    # 0.25/gamma = 0.5 rounds (half to even) to 0
+    row = np.array([0.25, -0.75, 0.75, -0.25] * 64, dtype=np.float32)
+    w = np.tile((row.view(np.uint32) >> 16).astype(np.uint16), (16, 1))
+    x = synth.activations(4, 256, seed=4)
+    g = full_parity(w, x, 8, 8)
+    assert g["gamma"] == np.float32(0.5)
+
+
+def test_zero_and_tiny_activation_rows():
+    w = synth.latent_weights(64, 512, seed=5)
+    x = synth.activations(6, 512, seed=5)
+    x[0] = 0
+    x[1] = 0x8000
+    x[2] = 0x0001                                        # smallest subnormal everywhere
+    x[3, 7] = 0x7F7F                                     # largest finite bf16 in one channel
+    full_parity(w, x, 2, 4)
+
+
+def test_wide_exponent_weights():
+    rng = np.random.default_rng(6)
+    w = rng.integers(0, 0x7F00, size=(32, 512)).astype(np.uint16)   # every exponent, no inf
+    w |= (rng.integers(0, 2, size=w.shape).astype(np.uint16) << 15)
+    x = synth.activations(8, 512, seed=6)
+    g = run_layer(w, x, 6, 8, want_acc=False)
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, 6, 8)
+    assert_weights_exact(g, cb, mb, gamma)
+
+
+def test_subnormal_and_large_weights_gamma():
+    rng = np.random.default_rng(7)
+    w = synth.latent_weights(16, 256, seed=7)
+    w[0, :64] = rng.integers(1, 0x80, size=64).astype(np.uint16)      # subnormals
+    w[1, :8] = 0x7A00                                                 # ~1.7e35
+    w[2, :8] = 0x2000                                                 # ~1e-19
+    g = run_layer(w, synth.activations(2, 256, seed=7), 2, 4, want_acc=False)
+    cb, mb, gamma, _, _ = oracle.quantize_weights(w, 2, 4)
+    assert_weights_exact(g, cb, mb, gamma)
+
+
+def test_repeated_calls_reuse_workspace():
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    w1 = synth.latent_weights(256, 1024, seed=8, tag="a")
+    w2 = synth.latent_weights(256, 1024, seed=8, tag="b")
+    ws = torch.full((sbn.workspace_bytes(256, 1024),), 0xAB, dtype=torch.uint8, device="cuda")
+    out = sbn.alloc_packed(256, 1024, 6, 8, "cuda")
+    for w in [w1, w2, w1]:
+        sbn.quantize_weights(to_dev_bf16(w), 6, 8, out=out, workspace=ws)
+        c, mt, g = packed_to_numpy(out)
+        rc, rm, rg, _, _ = oracle.quantize_weights(w, 6, 8)
+        assert g == rg and np.array_equal(c, rc) and np.array_equal(mt, rm)
+
+
+# ---------------------------------------------------------------------------
+# the workloads at full size
+# ---------------------------------------------------------------------------
+
+@pytest.fixture(scope="module")
+def decode_ref():
+    w = synth.decode_weights()
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, 6, 8)
+    return w, cb, mb, gamma, dense
+
+
+@pytest.mark.parametrize("t", synth.DECODE_TOKENS)
+def test_decode_full_parity(decode_ref, t):
+    w, cb, mb, gamma, dense = decode_ref
+    x = synth.decode_acts(t)
+    g = run_layer(w, x, 6, 8)
+    assert_weights_exact(g, cb, mb, gamma)
+    q, s = oracle.quantize_acts(x)
+    assert np.array_equal(g["xq"], q) and np.array_equal(g["s"], s)
+    acc = oracle.bitlinear_acc(q, dense)
+    assert np.array_equal(g["acc"], acc)
+    assert_y_close(g["y"], oracle.dequant_bf16(acc, s, gamma))
+
+
+def _sampled_check(g, q, s, dense, gamma, t, n_out, seed, nsamp=4096):
+    rng = np.random.default_rng(seed)
+    ti = rng.integers(0, t, nsamp)
+    ni = rng.integers(0, n_out, nsamp)
+    # plus one full output row and one full output column
+    tr, nc = int(rng.integers(0, t)), int(rng.integers(0, n_out))
+    ti = np.concatenate([ti, np.full(n_out, tr), np.arange(t)])
+    ni = np.concatenate([ni, np.arange(n_out), np.full(t, nc)])
+    y_ref, acc_ref = oracle.bitlinear_at(q, s, dense, gamma, ti, ni)
+    assert np.array_equal(g["acc"][ti, ni], acc_ref)
+    assert_y_close(g["y"][ti, ni], y_ref)
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_prefill_sampled(which):
+    d = synth.prefill(which)
+    w, x, n, m = d["w"], d["x"], d["n"], d["m"]
+    g = run_layer(w, x, n, m)
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, n, m)
+    assert_weights_exact(g, cb, mb, gamma)
+    q, s = oracle.quantize_acts(x)
+    assert np.array_equal(g["xq"], q) and np.array_equal(g["s"], s)
+    _sampled_check(g, q, s, dense, gamma, x.shape[0], w.shape[0], seed=11)
+
+
+@pytest.mark.parametrize("proj", [p for p, _, _ in synth.QWEN05B_PROJ])
+def test_qwen_layer0_full(proj):
+    d = synth.qwen05b_layer(0, proj)
+    full_parity(d["w"], d["x"], d["n"], d["m"])
+
+
+@pytest.mark.parametrize("layer", [7, 23])
+def test_qwen_other_layers_sampled(layer):
+    for proj in ["q", "down"]:
+        d = synth.qwen05b_layer(layer, proj)
+        g = run_layer(d["w"], d["x"], 6, 8)
+        cb, mb, gamma, mask, dense = oracle.quantize_weights(d["w"], 6, 8)
+        assert_weights_exact(g, cb, mb, gamma)
+        q, s = oracle.quantize_acts(d["x"])
+        assert np.array_equal(g["xq"], q)
+        _sampled_check(g, q, s, dense, gamma, d["x"].shape[0], d["w"].shape[0], seed=layer)
+
+
+@pytest.mark.parametrize("nm", synth.FFN3B_PATTERNS)
+@pytest.mark.parametrize("proj", ["gate", "down"])
+def test_ffn3b_patterns(nm, proj):
+    for t in synth.FFN3B_TOKENS:
+        d = synth.ffn3b(proj, t, *nm)
+        g = run_layer(d["w"], d["x"], *nm)
+        if t == synth.FFN3B_TOKENS[0]:
+            cb, mb, gamma, mask, dense = oracle.quantize_weights(d["w"], *nm)
+            assert_weights_exact(g, cb, mb, gamma)
+        q, s = oracle.quantize_acts(d["x"])
+        assert np.array_equal(g["xq"], q) and np.array_equal(g["s"], s)
+        if t <= 64:
+            acc = oracle.bitlinear_acc(q, dense)
+            assert np.array_equal(g["acc"], acc)
+            assert_y_close(g["y"], oracle.dequant_bf16(acc, s, gamma))
+        else:
+            _sampled_check(g, q, s, dense, gamma, t, d["w"].shape[0], seed=t)
+
+
+def test_bitlinear_module_matches_calls():
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    d = synth.layer_small()
+    w = to_dev_bf16(d["w"])
+    layer = sbn.BitLinear(256, 256, n=2, m=4, weight=w.clone())
+    x = to_dev_bf16(d["x"]).reshape(2, 8, 256)
+    y = layer(x)
+    torch.cuda.synchronize()
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(d["w"], 2, 4)
+    q, s = oracle.quantize_acts(d["x"])
+    ref = oracle.dequant_bf16(oracle.bitlinear_acc(q, dense), s, gamma)
+    assert y.shape == (2, 8, 256)
+    assert_y_close(bf16_tensor_bits(y.reshape(16, 256)), ref)
