@@ -121,6 +121,32 @@ sbn_status sbn_quantize_weights(const void* w_bf16, int32_t n_out, int32_t k,
                                 size_t workspace_bytes, void* stream);
 
 /*
+ * sbn_quantize_weights_noalloc -- sbn_quantize_weights without a caller
+ * workspace. (Library addition; the pages describe nothing like it.)
+ *
+ * For callers that cannot allocate device memory: a plugin or kernel library
+ * that is handed only its input and output buffers, a real-time loop where
+ * the device-wide synchronization of cudaMalloc/cudaFree is not acceptable,
+ * or a process whose memory pool has already reserved all device memory.
+ * The scratch lives in a fixed array of SBN_NOALLOC_SCRATCH_BYTES (64 KiB)
+ * inside the library, reserved on every GPU that loads it until the process
+ * exits. This call performs no allocation of any kind.
+ *
+ *   Arguments, outputs and results are those of sbn_quantize_weights, minus
+ *   the workspace. Shapes whose workspace would exceed the fixed array are
+ *   rejected with SBN_ERR_WORKSPACE before anything is enqueued.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   All calls on a device share the one array: two calls that may run at the
+ *   same time on the GPU (different streams without ordering) race and give
+ *   wrong results. Calls on one stream are safe.
+ */
+#define SBN_NOALLOC_SCRATCH_BYTES (64 * 1024)
+sbn_status sbn_quantize_weights_noalloc(const void* w_bf16, int32_t n_out, int32_t k,
+                                        int32_t n, int32_t m, uint8_t* codes,
+                                        uint8_t* meta, float* gamma, void* stream);
+
+/*
  * sbn_quantize_acts -- per-token absmax INT8 activations.
  *
  * Defining passage: "The BitLinear Layer" (octagono page), second operation:

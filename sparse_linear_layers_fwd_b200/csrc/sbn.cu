@@ -110,7 +110,15 @@ sbn_status validate_bitlinear(const int8_t* xq, int32_t t, int32_t k, int32_t n_
   return SBN_OK;
 }
 
+// Fixed scratch of sbn_quantize_weights_noalloc (see include/sbn.h).
+constexpr size_t kNoAllocScratchBytes = SBN_NOALLOC_SCRATCH_BYTES;
+static_assert(kQwWorkspaceBytes <= kNoAllocScratchBytes, "workspace exceeds the fixed scratch");
+void* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+
 }  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 }  // namespace sbn
 
 using namespace sbn;
@@ -246,6 +254,54 @@ sbn_status sbn_bitlinear_acc32(const int8_t* xq, int32_t t, int32_t k, int32_t n
   if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
   return run_bitlinear<true>(xq, nullptr, t, k, n_out, n, m, codes, meta, nullptr, nullptr, acc,
                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Allocation-free variant of sbn_quantize_weights. Its scratch is a fixed
+// array in this file; the host side only ever uses the device address that
+// cudaGetSymbolAddress returns for it (looked up once per device, with that
+// device current). The bins are cleared on every call, on the caller's stream.
+sbn_status sbn_quantize_weights_noalloc(const void* w_bf16, int32_t n_out, int32_t k, int32_t n,
+                                        int32_t m, uint8_t* codes, uint8_t* meta, float* gamma,
+                                        void* stream) {
+  if (!w_bf16 || !codes || !gamma || (n != m && !meta)) return SBN_ERR_NULL;
+  sbn_status st = validate_weights_shape(n_out, k, n, m);
+  if (st != SBN_OK) return st;
+  if (!aligned16(w_bf16) || !aligned16(codes) || (meta && !aligned16(meta)) ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3u))
+    return SBN_ERR_ALIGN;
+  if (sbn_quantize_weights_workspace_bytes(n_out, k) > kNoAllocScratchBytes) return SBN_ERR_WORKSPACE;
+  int dev = 0, sms = 0;
+  if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* scratch = reinterpret_cast<char*>(g_noalloc_ptr[dev]);
+  unsigned long long* bins = reinterpret_cast<unsigned long long*>(scratch);
+  uint32_t* tau = reinterpret_cast<uint32_t*>(scratch + kQwTauOffset);
+  if (cudaMemsetAsync(bins, 0, kQwBins * sizeof(unsigned long long), s) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  const long long n_elems = (long long)n_out * k;
+  const long long nchunks = n_elems / 8;
+  const int blocks = (int)std::max<long long>(1, std::min<long long>((nchunks + 255) / 256, (long long)sms * 8));
+  qw_bins_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(w_bf16), nchunks, bins);
+  qw_finalize_kernel<<<1, 32, 0, s>>>(bins, n_elems, gamma, tau);
+  const uint16_t* w = reinterpret_cast<const uint16_t*>(w_bf16);
+  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
+  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
+  switch (m) {
+    case 4: launch_pack<4>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
+    case 8: launch_pack<8>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
+    default: launch_pack<16>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
+  }
+  return launch_status();
 }
 
 sbn_status sbn_get_device_error(void* stream) {

@@ -40,6 +40,8 @@ PROTOTYPES = {
     "sbn_quantize_weights_workspace_bytes": (_c_sz, [_c_i32, _c_i32]),
     "sbn_quantize_weights": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p,
                                             _c_p, _c_p, _c_sz, _c_p]),
+    "sbn_quantize_weights_noalloc": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
+                                                    _c_p, _c_p, _c_p]),
     "sbn_quantize_acts": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p]),
     "sbn_bitlinear": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
                                      _c_p, _c_p, _c_p, _c_p]),
@@ -152,6 +154,18 @@ def quantize_weights(w: torch.Tensor, n: int, m: int, out: Optional[PackedWeight
                                     _ptr(out.gamma), _ptr(workspace), workspace.numel(),
                                     _stream_ptr(stream))
     _check(st, "sbn_quantize_weights")
+    return out
+
+
+def quantize_weights_noalloc(w: torch.Tensor, n: int, m: int, out: PackedWeights,
+                             stream=None) -> PackedWeights:
+    """sbn_quantize_weights_noalloc: like quantize_weights, with the library's
+    fixed internal scratch instead of a caller workspace (no allocation)."""
+    _need(w, torch.bfloat16, "w")
+    n_out, k = w.shape
+    st = lib().sbn_quantize_weights_noalloc(_ptr(w), n_out, k, n, m, _ptr(out.codes),
+                                            _ptr(out.meta), _ptr(out.gamma), _stream_ptr(stream))
+    _check(st, "sbn_quantize_weights_noalloc")
     return out
 
 
