@@ -13,6 +13,9 @@ namespace sbn {
 // Error word: one per device, set by bounded waits that give up.
 // ---------------------------------------------------------------------------
 enum : unsigned { kDevErrNone = 0u, kDevErrTimeout = 1u };
+// The library is one translation unit (sbn.cu includes every kernel header),
+// so the word is defined here, once.
+__device__ unsigned int g_dev_error;
 
 // Packed-format geometry. A "unit" is 16 consecutive positions along K; for
 // every supported pattern a unit's kept codes fill a whole number of bytes

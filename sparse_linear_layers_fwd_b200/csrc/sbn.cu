@@ -15,11 +15,13 @@
 #include "common.cuh"
 #include "qa.cuh"
 #include "qw.cuh"
-#include "bl_simt.cuh"
+#include "qw_fused.cuh"
+#include "bl_decode.cuh"
+#include "bl_tc.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace sbn {
-
-__device__ unsigned int g_dev_error;
 
 namespace {
 
@@ -76,28 +78,176 @@ void launch_pack(const uint16_t* w, int n_out, int k, int n, const uint32_t* tau
   qw_pack_kernel<M><<<blocks, 256, 0, st>>>(w, n_out, k, n, tau, codes, cstride, meta, mstride);
 }
 
+// One cooperative launch of qw_fused_kernel: one CTA per SM, so that all
+// CTAs are resident for the grid barrier. The bins and the arrival counter
+// of the workspace are cleared first, on the same stream.
+template <int M>
+sbn_status launch_qw_fused(const uint16_t* w, int n_out, int k, int n, uint8_t* codes, int cstride,
+                           uint8_t* meta, int mstride, float* gamma, unsigned char* ws, int sms,
+                           cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)sms);
+  cfg.blockDim = dim3(512);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, qw_fused_kernel<M>, w, n_out, k, n, codes, cstride, meta, mstride,
+                         gamma, ws) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  return SBN_OK;
+}
+
+sbn_status launch_quantize_weights(const uint16_t* w, int n_out, int k, int n, int m, uint8_t* codes,
+                                   uint8_t* meta, float* gamma, unsigned char* ws, int sms,
+                                   cudaStream_t st) {
+  // Each CTA's exact sum counts units of 2^-37 of values below 8 in a u64:
+  // at most 2^24 elements per CTA (always true for N_out*K < 2^31 on 128+ SMs).
+  if ((long long)n_out * k > ((long long)sms << 24)) return SBN_ERR_SHAPE;
+  if (cudaMemsetAsync(ws, 0, kQwArriveOffset + 16, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
+  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
+  switch (m) {
+    case 4: return launch_qw_fused<4>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
+    case 8: return launch_qw_fused<8>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
+    default: return launch_qw_fused<16>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
+  }
+}
+
+template <int MM, int CB, int NT, bool DENSE, bool ACC>
+sbn_status launch_decode(const DecodeParams& p, int sms, cudaStream_t st) {
+  static bool attr_set = false;  // per instantiation (benign race: same value)
+  const size_t smem = decode_smem_bytes(p.rt, NT, CB, DENSE);
+  auto kern = bl_decode_kernel<MM, CB, NT, DENSE, ACC>;
+  if (!attr_set) {
+    // allow the largest footprint this instantiation can be launched with
+    const size_t smem_max = decode_smem_bytes(kDecMaxRT, NT, CB, DENSE);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) != cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set = true;
+  }
+  (void)sms;
+  const int rows = 16 * p.rt;
+  kern<<<(p.N + rows - 1) / rows, 32 * kDecKS * p.rt, smem, st>>>(p);
+  return launch_status();
+}
+
+template <int NT, bool ACC>
+sbn_status dispatch_decode(const DecodeParams& p, int n, int m, int sms, cudaStream_t st) {
+  const int cb = 4 * n / m;
+  if (n == m) return launch_decode<8, 4, NT, true, ACC>(p, sms, st);
+  switch (m * 8 + cb) {
+    case 4 * 8 + 1: return launch_decode<4, 1, NT, false, ACC>(p, sms, st);
+    case 4 * 8 + 2: return launch_decode<4, 2, NT, false, ACC>(p, sms, st);
+    case 4 * 8 + 3: return launch_decode<4, 3, NT, false, ACC>(p, sms, st);
+    case 8 * 8 + 1: return launch_decode<8, 1, NT, false, ACC>(p, sms, st);
+    case 8 * 8 + 2: return launch_decode<8, 2, NT, false, ACC>(p, sms, st);
+    case 8 * 8 + 3: return launch_decode<8, 3, NT, false, ACC>(p, sms, st);
+    case 16 * 8 + 1: return launch_decode<16, 1, NT, false, ACC>(p, sms, st);
+    case 16 * 8 + 2: return launch_decode<16, 2, NT, false, ACC>(p, sms, st);
+    case 16 * 8 + 3: return launch_decode<16, 3, NT, false, ACC>(p, sms, st);
+  }
+  return SBN_ERR_PATTERN;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+template <int MM, int CB, bool DENSE, bool ACC>
+sbn_status launch_tc(const CUtensorMap& tm, const TcParams& p, cudaStream_t st) {
+  static bool attr_set = false;
+  auto kern = bl_tc_kernel<MM, CB, DENSE, ACC>;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set = true;
+  }
+  dim3 grid((p.N + kTcBM - 1) / kTcBM, (p.T + kTcBN - 1) / kTcBN);
+  kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(tm, p);
+  return launch_status();
+}
+
+template <bool ACC>
+sbn_status dispatch_tc(const CUtensorMap& tm, const TcParams& p, int n, int m, cudaStream_t st) {
+  const int cb = 4 * n / m;
+  if (n == m) return launch_tc<8, 4, true, ACC>(tm, p, st);
+  switch (m * 8 + cb) {
+    case 4 * 8 + 1: return launch_tc<4, 1, false, ACC>(tm, p, st);
+    case 4 * 8 + 2: return launch_tc<4, 2, false, ACC>(tm, p, st);
+    case 4 * 8 + 3: return launch_tc<4, 3, false, ACC>(tm, p, st);
+    case 8 * 8 + 1: return launch_tc<8, 1, false, ACC>(tm, p, st);
+    case 8 * 8 + 2: return launch_tc<8, 2, false, ACC>(tm, p, st);
+    case 8 * 8 + 3: return launch_tc<8, 3, false, ACC>(tm, p, st);
+    case 16 * 8 + 1: return launch_tc<16, 1, false, ACC>(tm, p, st);
+    case 16 * 8 + 2: return launch_tc<16, 2, false, ACC>(tm, p, st);
+    case 16 * 8 + 3: return launch_tc<16, 3, false, ACC>(tm, p, st);
+  }
+  return SBN_ERR_PATTERN;
+}
+
+// TMA map of the INT8 activations [T, K]: boxes of 256 tokens x 128 bytes,
+// 128-byte swizzle (the layout the MMA descriptors describe).
+sbn_status make_act_tensor_map(CUtensorMap* tm, const int8_t* xq, int t, int k) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return SBN_ERR_CUDA;
+  cuuint64_t gdim[2] = {(cuuint64_t)k, (cuuint64_t)t};
+  cuuint64_t gstride[1] = {(cuuint64_t)k};
+  cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBN};
+  cuuint32_t estride[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(xq), gdim, gstride, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SBN_OK : SBN_ERR_CUDA;
+}
+
 template <bool ACC_OUT>
 sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k, int32_t n_out,
                          int32_t n, int32_t m, const uint8_t* codes, const uint8_t* meta,
-                         const float* gamma, uint16_t* y, int32_t* acc, cudaStream_t st) {
+                         const float* gamma, uint16_t* y, int32_t* acc, int sms, cudaStream_t st) {
   const int cstride = (int)sbn_codes_row_bytes(k, n, m);
   const int mstride = (int)sbn_meta_row_bytes(k, n, m);
-  dim3 grid((n_out + kSimtO - 1) / kSimtO, (t + kSimtT - 1) / kSimtT);
-  switch (m) {
-    case 4:
-      bl_simt_kernel<4, ACC_OUT><<<grid, 256, 0, st>>>(xq, xs, t, k, n_out, n, codes, cstride, meta,
-                                                       mstride, gamma, y, acc);
-      break;
-    case 8:
-      bl_simt_kernel<8, ACC_OUT><<<grid, 256, 0, st>>>(xq, xs, t, k, n_out, n, codes, cstride, meta,
-                                                       mstride, gamma, y, acc);
-      break;
-    default:
-      bl_simt_kernel<16, ACC_OUT><<<grid, 256, 0, st>>>(xq, xs, t, k, n_out, n, codes, cstride,
-                                                        meta, mstride, gamma, y, acc);
-      break;
+  if (t <= 16) {
+    DecodeParams p;
+    p.xq = xq; p.xs = xs; p.codes = codes; p.meta = meta; p.gamma = gamma; p.y = y; p.acc_out = acc;
+    p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
+    const int tiles = (n_out + 15) / 16;
+    p.rt = std::min(kDecMaxRT, std::max(1, (tiles + sms - 1) / sms));
+    return t <= 8 ? dispatch_decode<8, ACC_OUT>(p, n, m, sms, st)
+                  : dispatch_decode<16, ACC_OUT>(p, n, m, sms, st);
   }
-  return launch_status();
+  CUtensorMap tm;
+  const sbn_status st_map = make_act_tensor_map(&tm, xq, t, k);
+  if (st_map != SBN_OK) return st_map;
+  TcParams p;
+  p.codes = codes; p.meta = meta; p.xs = xs; p.gamma = gamma; p.y = y; p.acc_out = acc;
+  p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
+  return dispatch_tc<ACC_OUT>(tm, p, n, m, st);
 }
 
 sbn_status validate_bitlinear(const int8_t* xq, int32_t t, int32_t k, int32_t n_out, int32_t n,
@@ -183,26 +333,8 @@ sbn_status sbn_quantize_weights(const void* w_bf16, int32_t n_out, int32_t k, in
   if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-  unsigned long long* bins = reinterpret_cast<unsigned long long*>(workspace);
-  uint32_t* tau = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(workspace) + kQwTauOffset);
-  if (cudaMemsetAsync(bins, 0, kQwBins * sizeof(unsigned long long), s) != cudaSuccess) {
-    cudaGetLastError();
-    return SBN_ERR_CUDA;
-  }
-  const long long n_elems = (long long)n_out * k;
-  const long long nchunks = n_elems / 8;
-  const int blocks = (int)std::max<long long>(1, std::min<long long>((nchunks + 255) / 256, (long long)sms * 8));
-  qw_bins_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(w_bf16), nchunks, bins);
-  qw_finalize_kernel<<<1, 32, 0, s>>>(bins, n_elems, gamma, tau);
-  const uint16_t* w = reinterpret_cast<const uint16_t*>(w_bf16);
-  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
-  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
-  switch (m) {
-    case 4: launch_pack<4>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
-    case 8: launch_pack<8>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
-    default: launch_pack<16>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
-  }
-  return launch_status();
+  return launch_quantize_weights(reinterpret_cast<const uint16_t*>(w_bf16), n_out, k, n, m, codes,
+                                 meta, gamma, reinterpret_cast<unsigned char*>(workspace), sms, s);
 }
 
 sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k, int8_t* xq, float* x_scale,
@@ -239,7 +371,7 @@ sbn_status sbn_bitlinear(const int8_t* xq, const float* x_scale, int32_t t, int3
   int dev = 0, sms = 0;
   if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
   return run_bitlinear<false>(xq, x_scale, t, k, n_out, n, m, codes, meta, gamma,
-                              reinterpret_cast<uint16_t*>(y_bf16), nullptr,
+                              reinterpret_cast<uint16_t*>(y_bf16), nullptr, sms,
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -253,7 +385,7 @@ sbn_status sbn_bitlinear_acc32(const int8_t* xq, int32_t t, int32_t k, int32_t n
   int dev = 0, sms = 0;
   if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
   return run_bitlinear<true>(xq, nullptr, t, k, n_out, n, m, codes, meta, nullptr, nullptr, acc,
-                             reinterpret_cast<cudaStream_t>(stream));
+                             sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // Allocation-free variant of sbn_quantize_weights. Its scratch is a fixed
@@ -280,28 +412,9 @@ sbn_status sbn_quantize_weights_noalloc(const void* w_bf16, int32_t n_out, int32
     }
     g_noalloc_ptr[dev] = p;
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  char* scratch = reinterpret_cast<char*>(g_noalloc_ptr[dev]);
-  unsigned long long* bins = reinterpret_cast<unsigned long long*>(scratch);
-  uint32_t* tau = reinterpret_cast<uint32_t*>(scratch + kQwTauOffset);
-  if (cudaMemsetAsync(bins, 0, kQwBins * sizeof(unsigned long long), s) != cudaSuccess) {
-    cudaGetLastError();
-    return SBN_ERR_CUDA;
-  }
-  const long long n_elems = (long long)n_out * k;
-  const long long nchunks = n_elems / 8;
-  const int blocks = (int)std::max<long long>(1, std::min<long long>((nchunks + 255) / 256, (long long)sms * 8));
-  qw_bins_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(w_bf16), nchunks, bins);
-  qw_finalize_kernel<<<1, 32, 0, s>>>(bins, n_elems, gamma, tau);
-  const uint16_t* w = reinterpret_cast<const uint16_t*>(w_bf16);
-  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
-  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
-  switch (m) {
-    case 4: launch_pack<4>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
-    case 8: launch_pack<8>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
-    default: launch_pack<16>(w, n_out, k, n, tau, codes, cstride, meta, mstride, sms, s); break;
-  }
-  return launch_status();
+  return launch_quantize_weights(reinterpret_cast<const uint16_t*>(w_bf16), n_out, k, n, m, codes,
+                                 meta, gamma, reinterpret_cast<unsigned char*>(g_noalloc_ptr[dev]), sms,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_get_device_error(void* stream) {
