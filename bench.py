@@ -81,10 +81,12 @@ def bl_ops(t, k, n_out, n, m):
 
 WORKLOADS = {
     # name: list of layers (n_out, k, n, m, [token counts]) in one step
-    "decode": dict(desc="decode GEMV sweep: K=2560, N_out=6912, 6:8, T in {1,4,16}",
-                   layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
-    "prefill": dict(desc="prefill GEMM: T=4096, (K,N_out)=(2560,6912) and (6912,2560), 2:4",
-                    layers=[(6912, 2560, 2, 4, [4096]), (2560, 6912, 2, 4, [4096])]),
+    "decode": dict(desc="decode GEMV sweep: K=2560, N_out=6912, 6:8, T in {1,4,16}; value = "
+                        "algorithmic bytes of the step / step time",
+                   unit="GB/s", layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
+    "prefill": dict(desc="prefill GEMM: T=4096, (K,N_out)=(2560,6912) and (6912,2560), 2:4; value = "
+                         "algorithmic ops (2 per kept multiply-add) of the step / step time",
+                    unit="TOPS", layers=[(6912, 2560, 2, 4, [4096]), (2560, 6912, 2, 4, [4096])]),
 }
 
 
@@ -237,6 +239,17 @@ def oracle_sample_bytes(layers, rows_frac):
     return tot
 
 
+def oracle_sample_metric(workload, layers, rows_frac):
+    """The sample's amount of work in the workload's unit (GB or T-ops)."""
+    if WORKLOADS[workload]["unit"] == "TOPS":
+        tot = 0
+        for (n_out, k, n, m, ts) in layers:
+            r = max(1, int(n_out * rows_frac))
+            tot += sum(bl_ops(t, k, r, n, m) for t in ts)
+        return tot / 1e12
+    return oracle_sample_bytes(layers, rows_frac) / 1e9
+
+
 def make_layers_data(workload, rank=0):
     from sparse_linear_layers_fwd_b200 import synth
     out = []
@@ -380,8 +393,11 @@ def run_ours(args, rank, world, local_rank):
         ms = float(tt.item())
 
     sb = step_bytes(layers)
-    value_gbs = sb * args.steps * world / (ms * 1e-3) / 1e9
     ms_per_step = ms / args.steps
+    if WORKLOADS[args.workload]["unit"] == "TOPS":
+        value = step_ops(layers) * args.steps * world / (ms * 1e-3) / 1e12
+    else:
+        value = sb * args.steps * world / (ms * 1e-3) / 1e9
 
     # dominant call by total time in a step
     totals = {}
@@ -390,23 +406,41 @@ def run_ours(args, rank, world, local_rank):
         totals[name] += statistics.mean(v)
     dom = max(totals, key=totals.get)
     dom_ms = totals[dom]
-    if dom == "quantize_weights":
-        dom_bytes = sum(qw_bytes(n_out, k, n, m) for (n_out, k, n, m, ts) in layers)
-    elif dom == "quantize_acts":
-        dom_bytes = sum(qa_bytes(t, k) for (n_out, k, n, m, ts) in layers for t in ts)
-    else:
-        dom_bytes = sum(bl_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
     peaks = load_peaks()
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     n_dom_launches = len([c for c in call_names if c[0] == dom])
     traffic = ncu_traffic(dom, args.workload)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic, "kernel": dom,
-                "bytes_per_launch": dom_bytes // n_dom_launches,
-                "launch_us": round(dom_ms * 1e3 / n_dom_launches, 3),
-                "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)"
-                if peaks["source"] == "measured" else "fallback 6650 GB/s"}
+    tensor_bound = dom == "bitlinear" and min(t for (_, _, _, _, ts) in layers for t in ts) > 16
+    if tensor_bound:
+        # contraction on the tensor cores: algorithmic ops (2 per kept
+        # multiply-add) against the INT8 peak = measured bf16 peak x 2 (the
+        # nominal int8 : bf16 ratio of 4.5 : 2.25 POPS)
+        dom_ops = sum(bl_ops(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
+        achieved = dom_ops / (dom_ms * 1e-3) / 1e12
+        peak = 2.0 * peaks["bf16_tflops"]
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                    "unit": "TOPS", "frac": round(achieved / peak, 4), "traffic": traffic,
+                    "kernel": dom, "ops_per_launch": dom_ops // n_dom_launches,
+                    "launch_us": round(dom_ms * 1e3 / n_dom_launches, 3),
+                    "peak_source": f"2 x {peaks['source']} bf16_tflops {peaks['bf16_tflops']} "
+                                   f"(MEASURED_PEAKS.json; int8 = 2 x bf16 nominal)",
+                    "dense_equivalent_frac": round(
+                        sum(2 * t * k * n_out for (n_out, k, n, m, ts) in layers for t in ts)
+                        / (dom_ms * 1e-3) / 1e12 / peak, 4)}
+    else:
+        if dom == "quantize_weights":
+            dom_bytes = sum(qw_bytes(n_out, k, n, m) for (n_out, k, n, m, ts) in layers)
+        elif dom == "quantize_acts":
+            dom_bytes = sum(qa_bytes(t, k) for (n_out, k, n, m, ts) in layers for t in ts)
+        else:
+            dom_bytes = sum(bl_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
+        achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "traffic": traffic, "kernel": dom,
+                    "bytes_per_launch": dom_bytes // n_dom_launches,
+                    "launch_us": round(dom_ms * 1e3 / n_dom_launches, 3),
+                    "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)"
+                    if peaks["source"] == "measured" else "fallback 6650 GB/s"}
     breakdown = {}
     for (name, li, t), v in per_call.items():
         key = f"{name}[L{li}]" + (f"[T={t}]" if t else "")
@@ -423,6 +457,7 @@ def run_ours(args, rank, world, local_rank):
         if name == "bitlinear":
             ops = bl_ops(t, k, n_out, n, m)
             e["TOPS"] = round(ops / (us * 1e-6) / 1e12, 3)
+            e["dense_eq_TOPS"] = round(2 * t * k * n_out / (us * 1e-6) / 1e12, 3)
             e["tokens_per_s"] = round(t / (us * 1e-6), 1)
         breakdown[key] = e
 
@@ -433,15 +468,15 @@ def run_ours(args, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         frac, dt = run_oracle_timed(layers, data, target_s=args.cpu_seconds)
-        sbytes = oracle_sample_bytes(layers, frac)
-        cpu = {"value": round(sbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores_used(),
+        cpu = {"value": round(oracle_sample_metric(args.workload, layers, frac) / dt, 6),
+               "unit": WORKLOADS[args.workload]["unit"], "cores": cores_used(),
                "kind": "oracle",
                "sample": f"{frac:.3f} of the output features of every layer, full K and all "
                          f"token sets; one pass, {dt:.1f} s"}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value_gbs, 1), "unit": "GB/s",
+            "metric": METRIC, "value": round(value, 2), "unit": WORKLOADS[args.workload]["unit"],
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, bf16 io",
@@ -511,7 +546,11 @@ def run_e2e(args, data, layers, dev, stream, world):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
     sb = step_bytes(layers)
-    return {"value": round(sb * steps * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    if WORKLOADS[args.workload]["unit"] == "TOPS":
+        ev = step_ops(layers) * steps * world / (ms * 1e-3) / 1e12
+    else:
+        ev = sb * steps * world / (ms * 1e-3) / 1e9
+    return {"value": round(ev, 3), "unit": WORKLOADS[args.workload]["unit"],
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4)}
 
@@ -537,21 +576,21 @@ def run_reference(args, rank, world):
         for d, r in zip(data, rows):
             oracle_step([d], r)
     dt = time.perf_counter() - t0
-    sbytes = oracle_sample_bytes(layers, frac)
-    value = sbytes * args.steps / dt / 1e9
+    value = oracle_sample_metric(args.workload, layers, frac) * args.steps / dt
+    unit = WORKLOADS[args.workload]["unit"]
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, bf16 io",
         "data": "synthetic (seeded: W ~ N(0,0.02) bf16, X ~ N(0,1) bf16)",
         "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]["desc"],
                    "bytes_per_step": step_bytes(layers), "tokens_per_step": step_tokens(layers)},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores_used(),
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores_used(),
                          "kind": "oracle",
                          "sample": f"each step: {frac:.3f} of the output features of every "
                                    f"layer, full K, all token sets"},
-        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

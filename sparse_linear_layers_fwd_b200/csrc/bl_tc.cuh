@@ -4,23 +4,28 @@
 // "The BitLinear Layer", fourth and fifth operations; the Sparse-BitNet page
 // (Abstract, Table 3) runs the sparse BitLinear on tensor cores for prefill.
 //
-// One CTA computes a 128 (output features) x 256 (tokens) tile of
-// acc = Xq * W^T with `tcgen05.mma.cta_group::1.kind::i8` (int8 x int8 ->
-// int32), the accumulator in tensor memory:
-//   A (weights, 128 x 128 per K block) -- four producer warps read the packed
-//     codes + keep bits of their row from global memory, expand them to int8
-//     (expand.cuh) and store them in shared memory in the K-major
-//     128-byte-swizzled layout the MMA reads;
-//   B (activations, 256 x 128 per K block) -- one TMA load per stage, same
-//     swizzled layout;
-//   a ring of kTcStages stages: `full` barriers (128 producer arrivals + the
-//     TMA transaction bytes) and `empty` barriers (tcgen05.commit of the MMAs
-//     that read the stage);
-//   the MMA thread issues 4 MMAs (K = 32 each) per stage;
-//   the epilogue (the producer warps, which own TMEM lanes 0-127) reads the
-//     accumulator with tcgen05.ld and writes y = acc * gamma * s_t / 127.
-// Every mbarrier wait is bounded; a wait that gives up records
-// SBN_ERR_TIMEOUT in the device error word and the CTA winds down.
+// A persistent CTA per SM walks over 128 (output features) x 256 (tokens)
+// tiles of acc = Xq * W^T with `tcgen05.mma.cta_group::1.kind::i8` (int8 x
+// int8 -> int32), accumulating in tensor memory:
+//   warp 0      TMA loads of the activation tiles (256 x 128 bytes per K
+//               block, 128-byte swizzle);
+//   warp 1      TMEM allocation and the MMA thread: 4 MMAs (K = 32 each) per
+//               K block, tcgen05.commit to free a stage and, after the last
+//               K block of a tile, to hand the accumulator to the epilogue;
+//   warps 4-11  producers: two threads per weight row read the packed codes +
+//               keep bits of their row (prefetched two K blocks ahead),
+//               expand them to int8 (expand.cuh) and store them in the K-major
+//               128-byte-swizzled layout the MMA reads;
+//   warps 12-15 epilogue: tcgen05.ld of the accumulator (each warp owns one
+//               quadrant of the 128 TMEM lanes), y = acc * gamma * s_t / 127.
+// Two accumulators (2 x 256 TMEM columns) let the epilogue of one tile run
+// under the main loop of the next. Stage ring: `full` (256 producer arrivals
+// + the TMA bytes) and `empty` (MMA commit) barriers; accumulator ring:
+// `acc_full` (MMA commit) and `acc_empty` (one arrival per epilogue warp).
+// Barriers are waited on and arrived at once per warp (lane 0, then
+// __syncwarp), not per thread. Every mbarrier wait is bounded in time; a wait
+// that gives up records SBN_ERR_TIMEOUT in the device error word and the CTA
+// winds down.
 #pragma once
 
 #include <cuda.h>
@@ -37,17 +42,20 @@ constexpr int kTcStages = 4;
 constexpr int kTcABytes = kTcBM * kTcBK;
 constexpr int kTcBBytes = kTcBN * kTcBK;
 constexpr int kTcStageBytes = kTcABytes + kTcBBytes;
-constexpr int kTcThreads = 256;
-constexpr uint32_t kTcTmemCols = 256;
+constexpr int kTcThreads = 512;
+constexpr int kTcProducers = 256;     // two threads per weight row
+constexpr int kTcEpilogue = 128;
+constexpr uint32_t kTcTmemCols = 512; // two 256-column accumulators
 // instruction descriptor: s32 accumulate, signed 8-bit A and B, both K-major,
 // N = 256 (bits 17-22 hold N >> 3), M = 128 (bits 24-28 hold M >> 4)
 constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcBN >> 3) << 17) |
                               ((uint32_t)(kTcBM >> 4) << 24);
-constexpr long long kTcSpinLimit = 1ll << 22;  // try_wait rounds before giving up (~seconds)
+constexpr unsigned long long kTcWaitNs = 250000000ull;  // a wait gives up after 0.25 s
 
 // dynamic shared memory: stages (1024-aligned), then barriers and tables
+constexpr int kTcSelCopies = 8;       // selector table copies (fewer bank conflicts)
 constexpr size_t kTcSmemBytes = 1024 /*alignment slack*/ + (size_t)kTcStages * kTcStageBytes +
-                                 (2 * kTcStages + 2) * 8 + 16 + kTcBN * 4 + 256 * 4;
+                                 (2 * kTcStages + 4) * 8 + 16 + 256 * 4 * kTcSelCopies;
 
 struct TcParams {
   const uint8_t* codes;
@@ -73,17 +81,25 @@ SBN_DEVFN void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
-// Bounded wait for the phase of the given parity; false if it gave up.
+// Wait for the phase of the given parity, bounded in time (kTcWaitNs); false
+// (and SBN_ERR_TIMEOUT in the device error word) if it gave up. Polls with the
+// non-blocking test_wait so the thread sees the phase change at once.
 SBN_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
-  for (long long i = 0; i < kTcSpinLimit; ++i) {
+  unsigned long long t0 = 0;
+  for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+        "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(done)
         : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
+    if ((i & 63u) == 0u) {
+      const unsigned long long t = global_ns();
+      if (i == 0u) t0 = t;
+      else if (t - t0 > kTcWaitNs) break;
+    }
   }
   atomicOr(&g_dev_error, kDevErrTimeout);
   return false;
@@ -151,21 +167,25 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kTcStages * kTcStageBytes);
   uint64_t* empty = full + kTcStages;
-  uint64_t* accf = empty + kTcStages;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(accf + 2);
-  float* s_scale = reinterpret_cast<float*>(s_tmem + 4);
-  uint32_t* s_sel = reinterpret_cast<uint32_t*>(s_scale + kTcBN);
+  uint64_t* acc_full = empty + kTcStages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint32_t* s_sel = s_tmem + 4;             // [256][kTcSelCopies]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row0 = blockIdx.x * kTcBM, tok0 = blockIdx.y * kTcBN;
   const int nkb = p.K / kTcBK;
+  const int row_tiles = (p.N + kTcBM - 1) / kTcBM;
+  const int n_tiles = row_tiles * ((p.T + kTcBN - 1) / kTcBN);
 
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], kTcBM + 1);
+      mbar_init(&full[s], kTcProducers / 32 + 1);   // one arrival per producer warp + TMA
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kTcEpilogue / 32);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (warp == 1) {
@@ -174,13 +194,8 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  if (!DENSE) fill_selector_table(s_sel);
-  if (!ACC && (warp == 2 || warp == 3)) {
-    const float g = __ldg(p.gamma);
-    for (int j = tid - 64; j < kTcBN; j += 64) {
-      const int tok = tok0 + j;
-      s_scale[j] = tok < p.T ? __fdiv_rn(__fmul_rn(g, __ldg(p.xs + tok)), 127.0f) : 0.f;
-    }
+  if (!DENSE) {
+    for (int i = tid; i < 256 * kTcSelCopies; i += blockDim.x) s_sel[i] = expand_selector((uint32_t)(i / kTcSelCopies));
   }
   tc_fence_before();
   __syncthreads();
@@ -190,125 +205,184 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   if (warp == 0) {
     // ---- TMA producer of the activation tiles ----
     if (lane == 0) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kTcStages;
-        const uint32_t ph = (kb / kTcStages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u)) break;
-        uint8_t* bdst = smem + (size_t)s * kTcStageBytes + kTcABytes;
-        mbar_arrive_expect_tx(&full[s], kTcBBytes);
-        tma_load_2d(bdst, &tmap_x, kb * kTcBK, tok0, &full[s]);
+      int it = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int tok0 = (tile / row_tiles) * kTcBN;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kTcStages;
+          const uint32_t ph = (it / kTcStages) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], kTcBBytes);
+          tma_load_2d(smem + (size_t)s * kTcStageBytes + kTcABytes, &tmap_x, kb * kTcBK, tok0, &full[s]);
+        }
+        if (!ok) break;
       }
     }
   } else if (warp == 1) {
     // ---- MMA issuer ----
     if (lane == 0) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kTcStages;
-        const uint32_t ph = (kb / kTcStages) & 1u;
-        if (!mbar_wait(&full[s], ph)) break;
+      int it = 0, j = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++j) {
+        const int b = j & 1;
+        if (!mbar_wait(&acc_empty[b], ((j >> 1) & 1u) ^ 1u)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + (size_t)s * kTcStageBytes);
-        const uint32_t b_addr = a_addr + kTcABytes;
-        const uint64_t adesc = sw128_kmajor_desc(a_addr);
-        const uint64_t bdesc = sw128_kmajor_desc(b_addr);
+        const uint32_t d_tmem = tmem + (uint32_t)(b * kTcBN);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kTcStages;
+          const uint32_t ph = (it / kTcStages) & 1u;
+          if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+          const uint32_t a_addr = smem_u32(smem + (size_t)s * kTcStageBytes);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + kTcABytes);
 #pragma unroll
-        for (int k = 0; k < kTcBK / 32; ++k) {
-          // advance K by 32 bytes = 2 units of 16 bytes inside the swizzled row
-          tc_mma_i8(tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), (kb > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < kTcBK / 32; ++k) {
+            // K advances 32 bytes = 2 units of 16 bytes inside the swizzled row
+            tc_mma_i8(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
         }
-        tc_commit(&empty[s]);
+        tc_commit(&acc_full[b]);  // arrives once every MMA of this tile has completed
       }
-      tc_commit(accf);  // arrives once every MMA issued above has completed
     }
-  } else if (warp >= 4) {
-    // ---- A producers: expand the packed weights of row i of the tile ----
-    const int i = tid - 128;
-    const int row = row0 + i;
-    const bool row_ok = row < p.N;
-    const uint8_t* crow = p.codes + (size_t)(row_ok ? row : 0) * p.cstride;
-    const uint8_t* mrow = DENSE ? nullptr : p.meta + (size_t)(row_ok ? row : 0) * p.mstride;
+  } else if (warp >= 4 && warp < 12) {
+    // ---- producers: thread (i, h) expands units 4h..4h+3 of row i ----
+    const int pi = tid - 128;
+    const int i = pi & (kTcBM - 1), h = pi >> 7;
+    constexpr int kPre = 2;
+    constexpr int NW = CB;   // 32-bit words of codes for 4 units (4 * CB bytes)
+    uint32_t cwq[kPre + 1][NW];
+    uint2 mvq[kPre + 1];
+    const uint32_t* sel = s_sel + (lane & (kTcSelCopies - 1));
+    int it = 0;
     bool ok = true;
-    for (int kb = 0; kb < nkb && ok; ++kb) {
-      const int s = kb % kTcStages;
-      const uint32_t ph = (kb / kTcStages) & 1u;
-      // codes of this K block: 8 units x CB bytes; keep bits: 16 bytes
-      uint32_t cw[2 * CB];
-      uint4 mv = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-      if (row_ok) {
-        const uint2* cp = reinterpret_cast<const uint2*>(crow + (size_t)kb * 8 * CB);
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      const int row = (tile % row_tiles) * kTcBM + i;
+      const bool row_ok = row < p.N;
+      const uint8_t* crow = p.codes + (size_t)(row_ok ? row : 0) * p.cstride + h * 4 * CB;
+      const uint8_t* mrow = DENSE ? nullptr : p.meta + (size_t)(row_ok ? row : 0) * p.mstride + h * 8;
+      auto load_block = [&](int kb, uint32_t (&cw)[NW], uint2& mv) {
+        mv = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        if (row_ok && kb < nkb) {
+          const uint32_t* cp = reinterpret_cast<const uint32_t*>(crow + (size_t)kb * 8 * CB);
 #pragma unroll
-        for (int q = 0; q < CB; ++q) {
-          const uint2 v = __ldg(cp + q);
-          cw[2 * q] = v.x;
-          cw[2 * q + 1] = v.y;
-        }
-        if (!DENSE) mv = __ldg(reinterpret_cast<const uint4*>(mrow + (size_t)kb * 16));
-      } else {
-#pragma unroll
-        for (int q = 0; q < 2 * CB; ++q) cw[q] = 0u;
-      }
-      const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
-      if (!mbar_wait(&empty[s], ph ^ 1u)) {
-        ok = false;
-        break;
-      }
-      uint8_t* arow = smem + (size_t)s * kTcStageBytes + (size_t)i * 128;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t m16 = (mw[u >> 1] >> (16 * (u & 1))) & 0xFFFFu;
-        const uint32_t ucodes = code_bits<2 * CB>(cw, u * 8 * CB);  // this unit's 8*CB code bits
-        uint32_t out[4];
-        if (DENSE) {
-          codes8_to_s8(ucodes & 0xFFFFu, out[0], out[1]);
-          codes8_to_s8(ucodes >> 16, out[2], out[3]);
+          for (int q = 0; q < NW; ++q) cw[q] = __ldg(cp + q);
+          if (!DENSE) mv = __ldg(reinterpret_cast<const uint2*>(mrow + (size_t)kb * 16));
         } else {
-          const uint32_t m0 = m16 & 0xFFu, m1 = m16 >> 8;
-          const int p0 = (MM == 16) ? __popc(m0) : 2 * CB;
-          const uint32_t v0 = ucodes & ((1u << (2 * p0)) - 1u);
-          const uint32_t rest = ucodes >> (2 * p0);   // 2 * p0 <= 16
-          const int p1 = (MM == 16) ? __popc(m1) : 2 * CB;
-          const uint32_t v1 = rest & ((1u << (2 * p1)) - 1u);
-          expand8(m0, v0, s_sel, out[0], out[1]);
-          expand8(m1, v1, s_sel, out[2], out[3]);
+#pragma unroll
+          for (int q = 0; q < NW; ++q) cw[q] = 0u;
         }
-        *reinterpret_cast<uint4*>(arow + ((u ^ (i & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+      };
+#pragma unroll
+      for (int jj = 0; jj < kPre; ++jj) load_block(jj, cwq[jj], mvq[jj]);
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % kTcStages;
+        const uint32_t ph = (it / kTcStages) & 1u;
+        load_block(kb + kPre, cwq[kPre], mvq[kPre]);
+        uint32_t cw[NW];
+#pragma unroll
+        for (int q = 0; q < NW; ++q) cw[q] = cwq[0][q];
+        const uint2 mv = mvq[0];
+#pragma unroll
+        for (int jj = 0; jj < kPre; ++jj) {
+#pragma unroll
+          for (int q = 0; q < NW; ++q) cwq[jj][q] = cwq[jj + 1][q];
+          mvq[jj] = mvq[jj + 1];
+        }
+        // lane 0 waits for the stage, the warp follows
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&empty[s], ph ^ 1u) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        uint8_t* arow = smem + (size_t)s * kTcStageBytes + (size_t)i * 128;
+        const uint32_t mw[2] = {mv.x, mv.y};
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          const int u = 4 * h + uu;
+          const uint32_t m16 = (mw[uu >> 1] >> (16 * (uu & 1))) & 0xFFFFu;
+          const uint32_t ucodes = code_bits<NW>(cw, uu * 8 * CB);  // this unit's 8*CB code bits
+          uint32_t out[4];
+          if (DENSE) {
+            codes8_to_s8(ucodes & 0xFFFFu, out[0], out[1]);
+            codes8_to_s8(ucodes >> 16, out[2], out[3]);
+          } else {
+            const uint32_t m0 = m16 & 0xFFu, m1 = m16 >> 8;
+            const int p0 = (MM == 16) ? __popc(m0) : 2 * CB;
+            const uint32_t v0 = ucodes & ((1u << (2 * p0)) - 1u);
+            const uint32_t rest = ucodes >> (2 * p0);   // 2 * p0 <= 16
+            const int p1 = (MM == 16) ? __popc(m1) : 2 * CB;
+            const uint32_t v1 = rest & ((1u << (2 * p1)) - 1u);
+            uint32_t q0, q1;
+            codes8_to_s8(v0, q0, q1);
+            const uint32_t s0 = sel[m0 * kTcSelCopies];
+            out[0] = __byte_perm(q0, q1, s0 & 0xFFFFu);
+            out[1] = __byte_perm(q0, q1, s0 >> 16);
+            codes8_to_s8(v1, q0, q1);
+            const uint32_t s1 = sel[m1 * kTcSelCopies];
+            out[2] = __byte_perm(q0, q1, s1 & 0xFFFFu);
+            out[3] = __byte_perm(q0, q1, s1 >> 16);
+          }
+          *reinterpret_cast<uint4*>(arow + ((u ^ (i & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[s]);
       }
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      mbar_arrive(&full[s]);
     }
-
+  } else if (warp >= 12) {
     // ---- epilogue: TMEM -> registers -> y (or acc) ----
-    if (ok && mbar_wait(accf, 0u)) {
+    const int q = warp & 3;
+    const int row_in_tile = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const float g = ACC ? 0.f : __ldg(p.gamma);
+    int j = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
+      const int b = j & 1;
+      const int row = (tile % row_tiles) * kTcBM + row_in_tile;
+      const int tok0 = (tile / row_tiles) * kTcBN;
+      int got = 1;
+      if (lane == 0) got = mbar_wait(&acc_full[b], (j >> 1) & 1u) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
       tc_fence_after();
-      const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 #pragma unroll 1
       for (int c = 0; c < kTcBN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(32 * c), r);
-        if (row_ok) {
+        tmem_ld32(tmem + lane_base + (uint32_t)(b * kTcBN + 32 * c), r);
+        // lane jj holds the scale gamma * s_t / 127 of token tok0 + 32c + jj
+        const int my_tok = tok0 + 32 * c + lane;
+        const float my_sc = (ACC || my_tok >= p.T) ? 0.f : __fdiv_rn(__fmul_rn(g, __ldg(p.xs + my_tok)), 127.0f);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tok = tok0 + 32 * c + j;
-            if (tok < p.T) {
-              if (ACC) {
-                p.acc_out[(size_t)tok * p.N + row] = (int32_t)r[j];
-              } else {
-                const float yv = __fmul_rn((float)(int32_t)r[j], s_scale[32 * c + j]);
-                p.y[(size_t)tok * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
-              }
+        for (int jj = 0; jj < 32; ++jj) {
+          const int tok = tok0 + 32 * c + jj;
+          const float sc = __shfl_sync(0xffffffffu, my_sc, jj);
+          if (row < p.N && tok < p.T) {
+            if (ACC) {
+              p.acc_out[(size_t)tok * p.N + row] = (int32_t)r[jj];
+            } else {
+              const float yv = __fmul_rn((float)(int32_t)r[jj], sc);
+              p.y[(size_t)tok * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
             }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    // no MMA may still be writing the accumulator when it is freed (this
-    // matters only on the abort path; otherwise the phase is long complete)
-    if (lane == 0) mbar_wait(accf, 0u);
+    // no MMA may still be writing an accumulator when TMEM is freed (this
+    // matters only on the abort path): wait for the last commits
+    if (lane == 0) {
+      const int my_tiles = n_tiles > (int)blockIdx.x ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+      for (int jj = my_tiles - 2; jj < my_tiles; ++jj)
+        if (jj >= 0) mbar_wait(&acc_full[jj & 1], (jj >> 1) & 1u);
+    }
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTcTmemCols)

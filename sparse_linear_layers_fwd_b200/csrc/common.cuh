@@ -17,6 +17,13 @@ enum : unsigned { kDevErrNone = 0u, kDevErrTimeout = 1u };
 // so the word is defined here, once.
 __device__ unsigned int g_dev_error;
 
+// Nanoseconds of the GPU's global timer (for waits bounded in time).
+SBN_DEVFN unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Packed-format geometry. A "unit" is 16 consecutive positions along K; for
 // every supported pattern a unit's kept codes fill a whole number of bytes
 // (4*n/m) and its keep bits fill two bytes.

@@ -6,24 +6,25 @@
 // Naturally Friendly to Semi-Structured Sparsity", Abstract and Figure 6.
 //
 // gamma depends on the whole tensor while the codes depend on gamma, so the
-// kernel has two phases around one grid-wide barrier:
-//   phase 1  every CTA streams its rows of W from HBM once, adds every |w|
-//            exactly into per-exponent bins and computes the keep mask of
-//            every group (independent of gamma), written to meta;
+// kernel has two phases around a grid-wide barrier:
+//   phase 1  every CTA streams its rows of W from HBM once, sums |w| in fp64
+//            and computes the keep mask of every group (independent of
+//            gamma), written to meta;
 //   barrier  an arrival counter in the workspace; the spin is bounded and
 //            gives up with SBN_ERR_TIMEOUT in the device error word;
-//   phase 2  every CTA turns the bins into gamma and the code threshold tau
-//            (qw.cuh, one warp), re-reads its rows (now L2-resident) with the
-//            mask, and writes the kept codes.
-// The launch is cooperative, so all CTAs are resident and the barrier ends.
-//
-// Exact sum in phase 1: a bf16 magnitude with biased exponent e in
-// [97, 129] lies in [2^-30, 8) and is a multiple of 2^-37. A thread adds such
-// values into an fp64 accumulator; after at most 2048 of them the partial sum
-// is below 2^14 and still a multiple of 2^-37, i.e. an integer times 2^-37
-// below 2^51, so every fp64 addition was exact. The accumulator is then
-// moved (exactly) into a u64 count of 2^-37 units and restarted. All other
-// nonzero magnitudes go to shared per-exponent bins.
+//   gamma    every CTA reads the fp64 total S'. Its rounding error has a
+//            rigorous bound (positive terms: |S' - S| <= (additions on the
+//            longest path) * 2^-53 * S', plus 2^-126 per zero or subnormal
+//            |w|, which the fp64 construction below maps near 2^-127). If the
+//            whole interval of possible exact means rounds to one fp32 value,
+//            that value is gamma = max(fl32(fl64(S) / (N_out*K)), 1e-5). Else
+//            (an exact mean within ~2^-40 of an fp32 rounding midpoint, rare)
+//            every CTA re-reads its rows and adds every |w| exactly into
+//            integer bins, a second barrier follows, and gamma comes from the
+//            exact bins (qw.cuh);
+//   phase 2  every CTA derives the code threshold tau, re-reads its rows
+//            (now L2-resident) with the mask and writes the kept codes.
+// The launch is cooperative, so all CTAs are resident and the barriers end.
 #pragma once
 
 #include "common.cuh"
@@ -33,10 +34,9 @@ namespace sbn {
 
 // Workspace offsets beyond the bins and tau of qw.cuh.
 constexpr size_t kQwArriveOffset = kQwTauOffset + 16;   // u32 arrival counter
-constexpr long long kQwSpinLimit = 1ll << 24;            // ~1-2 s of polling
-constexpr uint32_t kQwF64Lo = 97u << 7;                  // smallest magnitude bits in the fp64 window
-constexpr uint32_t kQwF64Hi = 130u << 7;                 // first magnitude bits above it
-constexpr int kQwFlush = 2048;                           // fp64 window values per flush (at most)
+constexpr size_t kQwSumOffset = kQwArriveOffset + 16;   // f64 total of |w|
+constexpr size_t kQwClearBytes = kQwSumOffset + 16;     // cleared before every launch
+constexpr unsigned long long kQwWaitNs = 1000000000ull;  // the grid barrier gives up after 1 s
 
 SBN_DEVFN uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
@@ -44,20 +44,34 @@ SBN_DEVFN uint32_t ld_acquire_u32(const uint32_t* p) {
   return v;
 }
 
-// fp64 value of a normal bf16 magnitude (bits m, exponent field >= 1).
-SBN_DEVFN double bf16_mag_to_f64(uint32_t m) {
-  return __hiloint2double((int)((m << 13) + (896u << 20)), 0);
-}
+// High word of the fp64 value of a bf16 magnitude given as bits 16-30 of a
+// 32-bit word shifted down by 3 (exponent rebias 127 -> 1023); exact for
+// normal magnitudes, near 2^-127 for zero and subnormals.
+constexpr uint32_t kF64Rebias = 896u << 20;
 
-// Exact accumulation of one magnitude: fp64 window or shared bins.
-SBN_DEVFN void qw_accumulate(uint32_t mag, double& dacc, unsigned long long* sbins) {
-  if (mag - kQwF64Lo < kQwF64Hi - kQwF64Lo) {
-    dacc += bf16_mag_to_f64(mag);
-  } else if (mag) {
-    const uint32_t e = mag >> 7;
-    const uint32_t s = (mag & 0x7Fu) | (e ? 0x80u : 0u);
-    atomicAdd(&sbins[e ? e : 1u], (unsigned long long)s);
+// Bounded grid barrier: thread 0 of every CTA arrives and waits until the
+// counter reaches target. Returns false (and records a timeout) on give-up.
+SBN_DEVFN bool grid_barrier(uint32_t* arrive, uint32_t target, int* s_abort) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    atomicAdd(arrive, 1u);
+    const unsigned long long t0 = global_ns();
+    int abort = 0;
+    while (ld_acquire_u32(arrive) < target) {
+      if (global_ns() - t0 > kQwWaitNs) {
+        atomicOr(&g_dev_error, kDevErrTimeout);
+        abort = 1;
+        break;
+      }
+      __nanosleep(64);
+    }
+    *s_abort = abort;
   }
+  __syncthreads();
+  const bool ok = !*s_abort;
+  __threadfence();
+  return ok;
 }
 
 // Keep bits of 8 positions for m = 8 with exactly two pruned (6:8): the two
@@ -195,14 +209,16 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   constexpr int kWarps = 16;
   constexpr int kAhead = 4;  // units in flight per lane in phase 1
   __shared__ unsigned long long sbins[kQwBins];
+  __shared__ double swarp_d[kWarps];
   __shared__ unsigned long long swarp[kWarps];
   __shared__ __align__(16) uint8_t s_codes[kWarps][kSeg * 4];
   __shared__ uint32_t s_rm[256];
   __shared__ uint32_t s_tau;
-  __shared__ int s_abort;
+  __shared__ int s_abort, s_exact;
 
   unsigned long long* gbins = reinterpret_cast<unsigned long long*>(ws);
   uint32_t* arrive = reinterpret_cast<uint32_t*>(ws + kQwArriveOffset);
+  double* gsum = reinterpret_cast<double*>(ws + kQwSumOffset);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = k >> 4;
@@ -211,14 +227,10 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   const int r_begin = min(n_out, (int)blockIdx.x * rows_per_cta);
   const int r_end = min(n_out, r_begin + rows_per_cta);
 
-  for (int i = threadIdx.x; i < kQwBins; i += blockDim.x) sbins[i] = 0ull;
   if (M == 8 && n == 6) fill_remove_table(s_rm);
-  __syncthreads();
 
-  // ---- phase 1: exact sum and keep masks ------------------------------------
-  double dacc = 0.0;
-  int dcount = 0;                  // window values since the last flush
-  unsigned long long uacc = 0ull;  // flushed sum in units of 2^-37
+  // ---- phase 1: fp64 sum and keep masks -------------------------------------
+  double d0 = 0.0, d1 = 0.0;
   for (int row = r_begin + warp; row < r_end; row += kWarps) {
     const uint4* wrow = reinterpret_cast<const uint4*>(w + (size_t)row * k);
     for (int u0 = lane; u0 < units; u0 += 32 * kAhead) {
@@ -236,78 +248,103 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
         const int u = u0 + 32 * j;
         if (u >= units) break;
         const uint32_t wd[8] = {va[j].x, va[j].y, va[j].z, va[j].w, vb[j].x, vb[j].y, vb[j].z, vb[j].w};
-        uint32_t h[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          h[2 * i] = wd[i] & 0xFFFFu;
-          h[2 * i + 1] = wd[i] >> 16;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) qw_accumulate(h[i] & 0x7FFFu, dacc, sbins);
-        dcount += 16;
-        if (dcount > kQwFlush - 16) {
-          uacc += (unsigned long long)__double2ull_rz(dacc * 137438953472.0);  // * 2^37, exact
-          dacc = 0.0;
-          dcount = 0;
+          d0 += __hiloint2double((int)(((wd[i] & 0x7FFFu) << 13) + kF64Rebias), 0);
+          d1 += __hiloint2double((int)(((wd[i] >> 3) & 0x0FFFE000u) + kF64Rebias), 0);
         }
         if (has_meta) {
+          uint32_t h[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            h[2 * i] = wd[i] & 0xFFFFu;
+            h[2 * i + 1] = wd[i] >> 16;
+          }
           const uint32_t keep = unit_keep_bits<M>(h, n);
           *reinterpret_cast<uint16_t*>(meta + (size_t)row * meta_stride + 2 * u) = (uint16_t)keep;
         }
       }
     }
   }
-  uacc += (unsigned long long)__double2ull_rz(dacc * 137438953472.0);
+  double dsum = d0 + d1;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) uacc += __shfl_xor_sync(0xffffffffu, uacc, o);
-  if (lane == 0) swarp[warp] = uacc;
+  for (int o = 16; o; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+  if (lane == 0) swarp_d[warp] = dsum;
   __syncthreads();
   if (threadIdx.x == 0) {
-    unsigned long long a = 0ull;
-    for (int i = 0; i < kWarps; ++i) a += swarp[i];
-    // a counts units of 2^-37 = 2^(97-134): file it under exponents 97, 118
-    // and 139 in 21-bit pieces so every bin stays small
-    const unsigned long long mask21 = (1ull << 21) - 1ull;
-    const unsigned long long a0 = a & mask21, a1 = (a >> 21) & mask21, a2 = a >> 42;
-    if (a0) atomicAdd(&gbins[97], a0);
-    if (a1) atomicAdd(&gbins[118], a1);
-    if (a2) atomicAdd(&gbins[139], a2);
+    double a = 0.0;
+    for (int i = 0; i < kWarps; ++i) a += swarp_d[i];
+    atomicAdd(gsum, a);
   }
-  for (int i = threadIdx.x; i < kQwBins; i += blockDim.x)
-    if (sbins[i]) atomicAdd(&gbins[i], sbins[i]);
+  if (!grid_barrier(arrive, gridDim.x, &s_abort)) return;
 
-  // ---- grid barrier (bounded) -----------------------------------------------
-  __threadfence();
-  __syncthreads();
+  // ---- gamma: certified from the fp64 total, else exact ---------------------
   if (threadIdx.x == 0) {
-    atomicAdd(arrive, 1u);
-    long long spins = 0;
-    int abort = 0;
-    while (ld_acquire_u32(arrive) < gridDim.x) {
-      if (++spins > kQwSpinLimit) {
-        atomicOr(&g_dev_error, kDevErrTimeout);
-        abort = 1;
-        break;
+    const double S = __ldcg(gsum);
+    const double nk = (double)n_out * (double)k;
+    // additions on the longest path: per-thread accumulator, 2 -> 1, warp
+    // tree, CTA sum, one global atomic per CTA
+    const int per_thread = ((rows_per_cta + kWarps - 1) / kWarps) * ((units + 31) / 32) * 8;
+    const double adds = (double)per_thread + 1.0 + 5.0 + kWarps + (double)gridDim.x;
+    const double err = S * adds * 0x1p-53 * 1.01 + nk * 0x1p-126 * 1.01;
+    const double lo = (S - err) / nk * (1.0 - 0x1p-50);
+    const double hi = (S + err) / nk * (1.0 + 0x1p-50);
+    const float glo = fmaxf(__double2float_rn(lo), 1e-5f);
+    const float ghi = fmaxf(__double2float_rn(hi), 1e-5f);
+    s_exact = (glo == ghi) ? 0 : 1;
+    if (!s_exact) {
+      s_tau = code_threshold(glo);
+      if (blockIdx.x == 0) *gamma_out = glo;
+    }
+  }
+  __syncthreads();
+  if (s_exact) {
+    // rare: exact integer bins over the same rows (from L2), second barrier
+    for (int i = threadIdx.x; i < kQwBins; i += blockDim.x) sbins[i] = 0ull;
+    __syncthreads();
+    unsigned long long acc = 0ull;
+    for (int row = r_begin + warp; row < r_end; row += kWarps) {
+      const uint4* wrow = reinterpret_cast<const uint4*>(w + (size_t)row * k);
+      for (int u = lane; u < units; u += 32) {
+        const uint4 a = __ldg(wrow + 2 * u);
+        const uint4 b = __ldg(wrow + 2 * u + 1);
+        const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          exact_accumulate(wd[i] & 0x7FFFu, acc, sbins);
+          exact_accumulate((wd[i] >> 16) & 0x7FFFu, acc, sbins);
+        }
       }
-      __nanosleep(64);
     }
-    s_abort = abort;
-  }
-  __syncthreads();
-  if (s_abort) return;
-  __threadfence();
-
-  // ---- gamma and the code threshold (every CTA, one warp) -------------------
-  if (warp == 0) {
-    float g;
-    uint32_t tau;
-    gamma_and_tau_from_bins(gbins, (long long)n_out * k, &g, &tau);
-    if (lane == 0) {
-      s_tau = tau;
-      if (blockIdx.x == 0) *gamma_out = g;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) swarp[warp] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned long long a = 0ull;
+      for (int i = 0; i < kWarps; ++i) a += swarp[i];
+      // a counts units of 2^(kWinLo-134): file it under exponents kWinLo,
+      // kWinLo+21 and kWinLo+42 in 21-bit pieces so every bin stays small
+      const unsigned long long mask21 = (1ull << 21) - 1ull;
+      const unsigned long long a0 = a & mask21, a1 = (a >> 21) & mask21, a2 = a >> 42;
+      if (a0) atomicAdd(&gbins[kWinLo], a0);
+      if (a1) atomicAdd(&gbins[kWinLo + 21], a1);
+      if (a2) atomicAdd(&gbins[kWinLo + 42], a2);
     }
+    for (int i = threadIdx.x; i < kQwBins; i += blockDim.x)
+      if (sbins[i]) atomicAdd(&gbins[i], sbins[i]);
+    if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort)) return;
+    if (warp == 0) {
+      float g;
+      uint32_t tau;
+      gamma_and_tau_from_bins(gbins, (long long)n_out * k, &g, &tau);
+      if (lane == 0) {
+        s_tau = tau;
+        if (blockIdx.x == 0) *gamma_out = g;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
   const uint32_t tau = s_tau;
 
   // ---- phase 2: codes of the kept positions ---------------------------------

@@ -71,12 +71,6 @@ sbn_status validate_weights_shape(int32_t n_out, int32_t k, int32_t n, int32_t m
   return SBN_OK;
 }
 
-template <int M>
-void launch_pack(const uint16_t* w, int n_out, int k, int n, const uint32_t* tau, uint8_t* codes,
-                 int cstride, uint8_t* meta, int mstride, int sms, cudaStream_t st) {
-  const int blocks = (int)std::min<long long>((n_out + 7) / 8, (long long)sms * 4);
-  qw_pack_kernel<M><<<blocks, 256, 0, st>>>(w, n_out, k, n, tau, codes, cstride, meta, mstride);
-}
 
 // One cooperative launch of qw_fused_kernel: one CTA per SM, so that all
 // CTAs are resident for the grid barrier. The bins and the arrival counter
@@ -109,7 +103,7 @@ sbn_status launch_quantize_weights(const uint16_t* w, int n_out, int k, int n, i
   // Each CTA's exact sum counts units of 2^-37 of values below 8 in a u64:
   // at most 2^24 elements per CTA (always true for N_out*K < 2^31 on 128+ SMs).
   if ((long long)n_out * k > ((long long)sms << 24)) return SBN_ERR_SHAPE;
-  if (cudaMemsetAsync(ws, 0, kQwArriveOffset + 16, st) != cudaSuccess) {
+  if (cudaMemsetAsync(ws, 0, kQwClearBytes, st) != cudaSuccess) {
     cudaGetLastError();
     return SBN_ERR_CUDA;
   }
@@ -177,7 +171,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 template <int MM, int CB, bool DENSE, bool ACC>
-sbn_status launch_tc(const CUtensorMap& tm, const TcParams& p, cudaStream_t st) {
+sbn_status launch_tc(const CUtensorMap& tm, const TcParams& p, int sms, cudaStream_t st) {
   static bool attr_set = false;
   auto kern = bl_tc_kernel<MM, CB, DENSE, ACC>;
   if (!attr_set) {
@@ -188,25 +182,25 @@ sbn_status launch_tc(const CUtensorMap& tm, const TcParams& p, cudaStream_t st) 
     }
     attr_set = true;
   }
-  dim3 grid((p.N + kTcBM - 1) / kTcBM, (p.T + kTcBN - 1) / kTcBN);
-  kern<<<grid, kTcThreads, kTcSmemBytes, st>>>(tm, p);
+  const int tiles = ((p.N + kTcBM - 1) / kTcBM) * ((p.T + kTcBN - 1) / kTcBN);
+  kern<<<std::min(tiles, sms), kTcThreads, kTcSmemBytes, st>>>(tm, p);
   return launch_status();
 }
 
 template <bool ACC>
-sbn_status dispatch_tc(const CUtensorMap& tm, const TcParams& p, int n, int m, cudaStream_t st) {
+sbn_status dispatch_tc(const CUtensorMap& tm, const TcParams& p, int n, int m, int sms, cudaStream_t st) {
   const int cb = 4 * n / m;
-  if (n == m) return launch_tc<8, 4, true, ACC>(tm, p, st);
+  if (n == m) return launch_tc<8, 4, true, ACC>(tm, p, sms, st);
   switch (m * 8 + cb) {
-    case 4 * 8 + 1: return launch_tc<4, 1, false, ACC>(tm, p, st);
-    case 4 * 8 + 2: return launch_tc<4, 2, false, ACC>(tm, p, st);
-    case 4 * 8 + 3: return launch_tc<4, 3, false, ACC>(tm, p, st);
-    case 8 * 8 + 1: return launch_tc<8, 1, false, ACC>(tm, p, st);
-    case 8 * 8 + 2: return launch_tc<8, 2, false, ACC>(tm, p, st);
-    case 8 * 8 + 3: return launch_tc<8, 3, false, ACC>(tm, p, st);
-    case 16 * 8 + 1: return launch_tc<16, 1, false, ACC>(tm, p, st);
-    case 16 * 8 + 2: return launch_tc<16, 2, false, ACC>(tm, p, st);
-    case 16 * 8 + 3: return launch_tc<16, 3, false, ACC>(tm, p, st);
+    case 4 * 8 + 1: return launch_tc<4, 1, false, ACC>(tm, p, sms, st);
+    case 4 * 8 + 2: return launch_tc<4, 2, false, ACC>(tm, p, sms, st);
+    case 4 * 8 + 3: return launch_tc<4, 3, false, ACC>(tm, p, sms, st);
+    case 8 * 8 + 1: return launch_tc<8, 1, false, ACC>(tm, p, sms, st);
+    case 8 * 8 + 2: return launch_tc<8, 2, false, ACC>(tm, p, sms, st);
+    case 8 * 8 + 3: return launch_tc<8, 3, false, ACC>(tm, p, sms, st);
+    case 16 * 8 + 1: return launch_tc<16, 1, false, ACC>(tm, p, sms, st);
+    case 16 * 8 + 2: return launch_tc<16, 2, false, ACC>(tm, p, sms, st);
+    case 16 * 8 + 3: return launch_tc<16, 3, false, ACC>(tm, p, sms, st);
   }
   return SBN_ERR_PATTERN;
 }
@@ -247,7 +241,7 @@ sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k
   TcParams p;
   p.codes = codes; p.meta = meta; p.xs = xs; p.gamma = gamma; p.y = y; p.acc_out = acc;
   p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
-  return dispatch_tc<ACC_OUT>(tm, p, n, m, st);
+  return dispatch_tc<ACC_OUT>(tm, p, n, m, sms, st);
 }
 
 sbn_status validate_bitlinear(const int8_t* xq, int32_t t, int32_t k, int32_t n_out, int32_t n,

@@ -210,3 +210,33 @@ def test_bitlinear_module_matches_calls():
     ref = oracle.dequant_bf16(oracle.bitlinear_acc(q, dense), s, gamma)
     assert y.shape == (2, 8, 256)
     assert_y_close(bf16_tensor_bits(y.reshape(16, 256)), ref)
+
+
+def test_gamma_fp32_midpoint_exact_path():
+    """2^24 weights, all 1.0 but one 2.0: the exact mean 1 + 2^-24 lies exactly
+    halfway between two fp32 values, so no approximate sum can decide the
+    rounding and the kernel must take its exact path; ties go to even (1.0)."""
+    w = np.full((4096, 4096), 0x3F80, np.uint16)
+    w[123, 456] = 0x4000
+    x = synth.activations(2, 4096, seed=9)
+    g = run_layer(w, x, 6, 8, want_acc=False)
+    cb, mb, gamma, _, _ = oracle.quantize_weights(w, 6, 8)
+    assert gamma == np.float32(1.0)
+    assert_weights_exact(g, cb, mb, gamma)
+
+
+def test_gamma_midpoint_plus_tiny_follows_fp64_rounding():
+    """S = 2^24 + 1 + 2^-30 over 2^24 weights (all 1.0 except 2.0, 1.5, 1.5 and
+    2^-30): the fp64 rounding of S drops the 2^-30 (half an ulp of 2^24 is
+    2^-29), leaving the exact midpoint 1 + 2^-24 again, which goes to even.
+    This pins the defined order fl32(fl64(fl64(S) / N)) on the exact path."""
+    w = np.full((4096, 4096), 0x3F80, np.uint16)
+    w[7, 9] = 0x4000          # 2.0
+    w[8, 10] = 0x3FC0         # 1.5
+    w[9, 11] = 0x3FC0         # 1.5
+    w[10, 12] = 0x3080        # 2^-30
+    x = synth.activations(2, 4096, seed=10)
+    g = run_layer(w, x, 6, 8, want_acc=False)
+    cb, mb, gamma, _, _ = oracle.quantize_weights(w, 6, 8)
+    assert gamma == np.float32(1.0)
+    assert_weights_exact(g, cb, mb, gamma)
