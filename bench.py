@@ -108,6 +108,30 @@ def step_ops(layers):
 
 
 # ---------------------------------------------------------------------------
+# across ranks (one process per GPU, each on its own independent layer)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own and gets the max."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(workload: str, steps: int, world: int, ms_max: float) -> float:
+    """Units processed by all ranks (weak scaling: each rank runs a full step
+    on its own layer) over the slowest rank's time, in the workload's unit."""
+    layers = WORKLOADS[workload]["layers"]
+    if WORKLOADS[workload]["unit"] == "TOPS":
+        return step_ops(layers) * steps * world / (ms_max * 1e-3) / 1e12
+    return step_bytes(layers) * steps * world / (ms_max * 1e-3) / 1e9
+
+
+# ---------------------------------------------------------------------------
 # helpers
 # ---------------------------------------------------------------------------
 
@@ -301,6 +325,7 @@ def run_ours(args, rank, world, local_rank):
 
     # R rotation slots of inputs, packed weights, activations and outputs
     slots = []
+    layer_bws = {}
     for _ in range(R):
         sl = []
         for (w, xs, n, m), (n_out, k, _, _, ts) in zip(data, layers):
@@ -311,7 +336,12 @@ def run_ours(args, rank, world, local_rank):
             qs = [(torch.empty((t, k), dtype=torch.int8, device=dev),
                    torch.empty((t,), dtype=torch.float32, device=dev)) for t in ts]
             ys = [torch.empty((t, n_out), dtype=torch.bfloat16, device=dev) for t in ts]
-            sl.append(dict(w=wd, xs=xds, pw=pw, ws=ws, qs=qs, ys=ys, n=n, m=m))
+            # the contraction's workspace (expanded weights, T > 16); written
+            # and read within one call, so one per layer serves every slot
+            bws = layer_bws.setdefault((n_out, k), torch.empty(
+                (max(1, max(sbn.bitlinear_workspace_bytes(t, k, n_out) for t in ts)),),
+                dtype=torch.uint8, device=dev))
+            sl.append(dict(w=wd, xs=xds, pw=pw, ws=ws, bws=bws, qs=qs, ys=ys, n=n, m=m))
         slots.append(sl)
 
     # per-call events inside each slot's graph: names of the calls in order
@@ -335,7 +365,7 @@ def run_ours(args, rank, world, local_rank):
                 if evs: evs[i][1].record(stream)
                 i += 1
                 if evs: evs[i][0].record(stream)
-                sbn.bitlinear(q, s, L["pw"], out=y, stream=stream)
+                sbn.bitlinear(q, s, L["pw"], out=y, workspace=L["bws"], stream=stream)
                 if evs: evs[i][1].record(stream)
                 i += 1
 
@@ -351,7 +381,10 @@ def run_ours(args, rank, world, local_rank):
             enqueue_step(slots[r], evs)
         graphs.append(g)
         slot_events.append(evs)
-    launches_per_step = sum(3 + 2 * len(ts) for (_, _, _, _, ts) in layers)
+    # our kernels per step: quantize_weights 1 per layer; quantize_acts 1 and
+    # bitlinear 1 (+1 weight expansion when T > 16) per token set
+    launches_per_step = sum(1 + sum(2 + (1 if t > 16 else 0) for t in ts)
+                            for (_, _, _, _, ts) in layers)
 
     def barrier():
         if world > 1:
@@ -387,17 +420,11 @@ def run_ours(args, rank, world, local_rank):
         for (name, li, t), (a, b) in zip(call_names, slot_events[r]):
             per_call.setdefault((name, li, t), []).append(a.elapsed_time(b))
 
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
 
     sb = step_bytes(layers)
     ms_per_step = ms / args.steps
-    if WORKLOADS[args.workload]["unit"] == "TOPS":
-        value = step_ops(layers) * args.steps * world / (ms * 1e-3) / 1e12
-    else:
-        value = sb * args.steps * world / (ms * 1e-3) / 1e9
+    value = whole_job_value(args.workload, args.steps, world, ms)
 
     # dominant call by total time in a step
     totals = {}
@@ -540,16 +567,8 @@ def run_e2e(args, data, layers, dev, stream, world):
             step()
         ev1.record(stream)
     stream.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    sb = step_bytes(layers)
-    if WORKLOADS[args.workload]["unit"] == "TOPS":
-        ev = step_ops(layers) * steps * world / (ms * 1e-3) / 1e12
-    else:
-        ev = sb * steps * world / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    ev = whole_job_value(args.workload, steps, world, ms)
     return {"value": round(ev, 3), "unit": WORKLOADS[args.workload]["unit"],
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4)}

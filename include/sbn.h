@@ -177,23 +177,38 @@ sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k,
  *   y_bf16        device, [t, n_out] bf16, written:
  *                 y = bf16_rne(acc * gamma * s_t / 127) evaluated in fp32, where
  *                 acc[t, o] = sum over kept k of xq[t, k] * code[o, k] (exact int32).
- * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN;
- * SBN_ERR_CUDA.
+ *   workspace,    optional device scratch owned by the caller (the pages have
+ *   ws_bytes      no counterpart). NULL: the packed weights are expanded
+ *                 inside the contraction kernel. Non-NULL (16-byte aligned,
+ *                 ws_bytes >= sbn_bitlinear_workspace_bytes(t, k, n_out)):
+ *                 for t > 16 the packed weights are first expanded once into
+ *                 it as a dense int8 [n_out, k] matrix, which the tensor-core
+ *                 kernel then loads by TMA like the activations. Ignored for
+ *                 t <= 16. Its contents are unspecified afterwards. Both
+ *                 routes give the same acc and y.
+ * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN,
+ * SBN_ERR_WORKSPACE (before anything is enqueued); SBN_ERR_CUDA.
  */
 sbn_status sbn_bitlinear(const int8_t* xq, const float* x_scale, int32_t t,
                          int32_t k, int32_t n_out, int32_t n, int32_t m,
                          const uint8_t* codes, const uint8_t* meta,
-                         const float* gamma, void* y_bf16, void* stream);
+                         const float* gamma, void* y_bf16, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* Bytes of sbn_bitlinear's optional workspace: n_out * k when t > 16, else 0. */
+size_t sbn_bitlinear_workspace_bytes(int32_t t, int32_t k, int32_t n_out);
 
 /*
  * sbn_bitlinear_acc32 -- the same contraction, writing the exact int32
  * accumulators acc [t, n_out] (device, row-major) instead of y. Meant for
- * verification; same arguments and errors as sbn_bitlinear.
+ * verification; same arguments (workspace included) and errors as
+ * sbn_bitlinear.
  */
 sbn_status sbn_bitlinear_acc32(const int8_t* xq, int32_t t, int32_t k,
                                int32_t n_out, int32_t n, int32_t m,
                                const uint8_t* codes, const uint8_t* meta,
-                               int32_t* acc, void* stream);
+                               int32_t* acc, void* workspace, size_t ws_bytes,
+                               void* stream);
 
 /*
  * sbn_get_device_error -- synchronizes `stream`, then reads and clears the

@@ -30,6 +30,7 @@
 
 #include <cuda.h>
 
+#include "async.cuh"
 #include "common.cuh"
 #include "expand.cuh"
 
@@ -50,7 +51,6 @@ constexpr uint32_t kTcTmemCols = 512; // two 256-column accumulators
 // N = 256 (bits 17-22 hold N >> 3), M = 128 (bits 24-28 hold M >> 4)
 constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcBN >> 3) << 17) |
                               ((uint32_t)(kTcBM >> 4) << 24);
-constexpr unsigned long long kTcWaitNs = 250000000ull;  // a wait gives up after 0.25 s
 
 // dynamic shared memory: stages (1024-aligned), then barriers and tables
 constexpr int kTcSelCopies = 8;       // selector table copies (fewer bank conflicts)
@@ -67,43 +67,6 @@ struct TcParams {
   int T, K, N;
   int cstride, mstride;
 };
-
-SBN_DEVFN uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-SBN_DEVFN void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-SBN_DEVFN void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
-}
-SBN_DEVFN void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-// Wait for the phase of the given parity, bounded in time (kTcWaitNs); false
-// (and SBN_ERR_TIMEOUT in the device error word) if it gave up. Polls with the
-// non-blocking test_wait so the thread sees the phase change at once.
-SBN_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  unsigned long long t0 = 0;
-  for (uint32_t i = 0;; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((i & 63u) == 0u) {
-      const unsigned long long t = global_ns();
-      if (i == 0u) t0 = t;
-      else if (t - t0 > kTcWaitNs) break;
-    }
-  }
-  atomicOr(&g_dev_error, kDevErrTimeout);
-  return false;
-}
 
 SBN_DEVFN uint64_t sw128_kmajor_desc(uint32_t saddr) {
   uint64_t d = 0;
@@ -160,9 +123,12 @@ SBN_DEVFN uint32_t code_bits(const uint32_t (&cw)[NW], int bit) {
   return s ? ((lo >> s) | (hi << (32 - s))) : lo;
 }
 
-template <int MM, int CB, bool DENSE, bool ACC>
+// TMA_A: the weights come expanded (dense int8 [N_out, K], expand_dense.cuh)
+// and warp 0 loads their tiles by TMA as well; the producer warps stay idle.
+template <int MM, int CB, bool DENSE, bool ACC, bool TMA_A>
 __global__ void __launch_bounds__(kTcThreads, 1)
-bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
+bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+             const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kTcStages * kTcStageBytes);
@@ -179,7 +145,8 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
 
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], kTcProducers / 32 + 1);   // one arrival per producer warp + TMA
+      // one arrival per producer warp + the TMA thread's (or the TMA thread's alone)
+      mbar_init(&full[s], TMA_A ? 1 : kTcProducers / 32 + 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -194,7 +161,7 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  if (!DENSE) {
+  if (!DENSE && !TMA_A) {
     for (int i = tid; i < 256 * kTcSelCopies; i += blockDim.x) s_sel[i] = expand_selector((uint32_t)(i / kTcSelCopies));
   }
   tc_fence_before();
@@ -208,12 +175,14 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
       int it = 0;
       for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         const int tok0 = (tile / row_tiles) * kTcBN;
+        const int row0 = (tile % row_tiles) * kTcBM;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kTcStages;
           const uint32_t ph = (it / kTcStages) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[s], kTcBBytes);
+          mbar_arrive_expect_tx(&full[s], TMA_A ? kTcABytes + kTcBBytes : kTcBBytes);
+          if (TMA_A) tma_load_2d(smem + (size_t)s * kTcStageBytes, &tmap_w, kb * kTcBK, row0, &full[s]);
           tma_load_2d(smem + (size_t)s * kTcStageBytes + kTcABytes, &tmap_x, kb * kTcBK, tok0, &full[s]);
         }
         if (!ok) break;
@@ -246,7 +215,7 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
         tc_commit(&acc_full[b]);  // arrives once every MMA of this tile has completed
       }
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (!TMA_A && warp >= 4 && warp < 12) {
     // ---- producers: thread (i, h) expands units 4h..4h+3 of row i ----
     const int pi = tid - 128;
     const int i = pi & (kTcBM - 1), h = pi >> 7;

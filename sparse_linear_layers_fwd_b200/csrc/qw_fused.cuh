@@ -27,6 +27,7 @@
 // The launch is cooperative, so all CTAs are resident and the barriers end.
 #pragma once
 
+#include "async.cuh"
 #include "common.cuh"
 #include "qw.cuh"
 
@@ -200,19 +201,96 @@ SBN_DEVFN void fill_remove_table(uint32_t* s_rm) {
   }
 }
 
+// Launch shape and dynamic shared memory of qw_fused_kernel. Every CTA owns a
+// contiguous range of units (16 consecutive weights of one row, 32 bytes),
+// i.e. one contiguous byte range of W, and streams it through a ring of
+// 16 KB stages filled by bulk copies: one stage is 512 units, one per thread.
+constexpr int kQwThreads = 512;
+constexpr int kQwWarps = kQwThreads / 32;
+constexpr int kQwChunk = 16384;       // bytes per stage
+constexpr int kQwStages = 8;          // 128 KB in flight per SM
+constexpr int kQwKeepCap = 16384;     // units whose keep bits stay in shared memory
+constexpr size_t kQwSmKeep = (size_t)kQwStages * kQwChunk;
+constexpr size_t kQwSmRm = kQwSmKeep + (size_t)kQwKeepCap * 2;
+constexpr size_t kQwSmBins = kQwSmRm + 256 * 4;
+constexpr size_t kQwSmBars = kQwSmBins + (size_t)kQwBins * 8;
+constexpr size_t kQwSmemBytes = kQwSmBars + (size_t)kQwStages * 8;
+
+// Stream ring over one CTA's byte range of W.
+struct QwRing {
+  const uint8_t* src;   // first byte of the range
+  long long bytes;      // length (a multiple of 32)
+  int nch;              // chunks in the range
+  uint8_t* buf;         // kQwStages x kQwChunk
+  uint64_t* full;       // one mbarrier per stage
+  uint32_t seq;         // chunks consumed so far, over all passes (uniform)
+};
+
+SBN_DEVFN void qw_issue(const QwRing& r, int c, uint32_t q) {
+  const int st = (int)(q % kQwStages);
+  const long long off = (long long)c * kQwChunk;
+  const uint32_t nb = (uint32_t)min((long long)kQwChunk, r.bytes - off);
+  mbar_arrive_expect_tx(&r.full[st], nb);
+  bulk_g2s(r.buf + (size_t)st * kQwChunk, r.src + off, nb, &r.full[st]);
+}
+
+// Issues the first stages of the next pass (thread 0).
+SBN_DEVFN void qw_prologue(const QwRing& r) {
+  if (threadIdx.x == 0)
+    for (int c = 0; c < min(r.nch, kQwStages); ++c) qw_issue(r, c, r.seq + (uint32_t)c);
+}
+
+// One pass over the range, whose prologue is already issued: f(c, stage,
+// units_here) runs for every chunk on every thread, then the stage is
+// refilled with chunk c + kQwStages. If a wait gives up, the copies still in
+// flight are waited for (bounded) and false is returned on every thread.
+template <class F>
+SBN_DEVFN bool qw_pass(QwRing& r, F&& f) {
+  for (int c = 0; c < r.nch; ++c) {
+    const uint32_t q = r.seq + (uint32_t)c;
+    const int st = (int)(q % kQwStages);
+    const bool ok = mbar_wait(&r.full[st], (q / kQwStages) & 1u);
+    const int units_here = (int)(min((long long)kQwChunk, r.bytes - (long long)c * kQwChunk) >> 5);
+    if (ok) f(c, r.buf + (size_t)st * kQwChunk, units_here);
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) {
+        for (int d = c + 1; d < min(r.nch, c + kQwStages); ++d) {
+          const uint32_t qd = r.seq + (uint32_t)d;
+          if (!mbar_wait(&r.full[qd % kQwStages], (qd / kQwStages) & 1u)) break;
+        }
+      }
+      __syncthreads();
+      return false;
+    }
+    if (threadIdx.x == 0 && c + kQwStages < r.nch) qw_issue(r, c + kQwStages, q + kQwStages);
+  }
+  r.seq += (uint32_t)r.nch;
+  return true;
+}
+
+// This thread's unit of a stage, read without bank conflicts: lanes 4-7 of
+// every quarter-warp fetch their upper half first.
+SBN_DEVFN void qw_load_unit(const uint8_t* stage, int t, uint32_t (&wd)[8]) {
+  const uint4* p = reinterpret_cast<const uint4*>(stage) + 2 * t;
+  const int sw = (t >> 2) & 1;
+  const uint4 a = p[sw], b = p[sw ^ 1];
+  const uint4 lo = sw ? b : a, hi = sw ? a : b;
+  wd[0] = lo.x; wd[1] = lo.y; wd[2] = lo.z; wd[3] = lo.w;
+  wd[4] = hi.x; wd[5] = hi.y; wd[6] = hi.z; wd[7] = hi.w;
+}
+
 template <int M>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(kQwThreads, 1)
 qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
                 uint8_t* __restrict__ codes, int codes_stride, uint8_t* __restrict__ meta,
                 int meta_stride, float* __restrict__ gamma_out, unsigned char* __restrict__ ws) {
-  constexpr int kSeg = 256;  // units per staged code segment
-  constexpr int kWarps = 16;
-  constexpr int kAhead = 4;  // units in flight per lane in phase 1
-  __shared__ unsigned long long sbins[kQwBins];
-  __shared__ double swarp_d[kWarps];
-  __shared__ unsigned long long swarp[kWarps];
-  __shared__ __align__(16) uint8_t s_codes[kWarps][kSeg * 4];
-  __shared__ uint32_t s_rm[256];
+  extern __shared__ __align__(128) uint8_t qw_smem[];
+  uint16_t* s_keep = reinterpret_cast<uint16_t*>(qw_smem + kQwSmKeep);
+  uint32_t* s_rm = reinterpret_cast<uint32_t*>(qw_smem + kQwSmRm);
+  unsigned long long* sbins = reinterpret_cast<unsigned long long*>(qw_smem + kQwSmBins);
+  uint64_t* full = reinterpret_cast<uint64_t*>(qw_smem + kQwSmBars);
+  __shared__ double swarp_d[kQwWarps];
+  __shared__ unsigned long long swarp[kQwWarps];
   __shared__ uint32_t s_tau;
   __shared__ int s_abort, s_exact;
 
@@ -220,34 +298,52 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   uint32_t* arrive = reinterpret_cast<uint32_t*>(ws + kQwArriveOffset);
   double* gsum = reinterpret_cast<double*>(ws + kQwSumOffset);
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int units = k >> 4;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int upr = k >> 4;                       // units per row
+  const long long total_units = (long long)n_out * upr;
+  const long long u_begin = (long long)blockIdx.x * total_units / gridDim.x;
+  const long long u_end = (long long)(blockIdx.x + 1) * total_units / gridDim.x;
   const bool has_meta = (n != M);
-  const int rows_per_cta = (n_out + gridDim.x - 1) / gridDim.x;
-  const int r_begin = min(n_out, (int)blockIdx.x * rows_per_cta);
-  const int r_end = min(n_out, r_begin + rows_per_cta);
+  const int cb = 4 * n / M;                     // code bytes per unit
+  const int row_step = kQwThreads / upr, u_step = kQwThreads % upr;
 
+  QwRing ring;
+  ring.src = reinterpret_cast<const uint8_t*>(w) + u_begin * 32;
+  ring.bytes = (u_end - u_begin) * 32;
+  ring.nch = (int)((ring.bytes + kQwChunk - 1) / kQwChunk);
+  ring.buf = qw_smem;
+  ring.full = full;
+  ring.seq = 0u;
+
+  if (t == 0) {
+    for (int s = 0; s < kQwStages; ++s) mbar_init(&full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
   if (M == 8 && n == 6) fill_remove_table(s_rm);
+  __syncthreads();
+  qw_prologue(ring);
+
+  // (row, u) of this thread's unit in chunk c, advanced chunk by chunk
+  int row0, u0;
+  {
+    const long long g = u_begin + t;
+    row0 = (int)(g / upr);
+    u0 = (int)(g - (long long)row0 * upr);
+  }
+  auto advance = [&](int& row, int& u) {
+    row += row_step;
+    u += u_step;
+    if (u >= upr) { u -= upr; ++row; }
+  };
 
   // ---- phase 1: fp64 sum and keep masks -------------------------------------
   double d0 = 0.0, d1 = 0.0;
-  for (int row = r_begin + warp; row < r_end; row += kWarps) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(w + (size_t)row * k);
-    for (int u0 = lane; u0 < units; u0 += 32 * kAhead) {
-      uint4 va[kAhead], vb[kAhead];
-#pragma unroll
-      for (int j = 0; j < kAhead; ++j) {
-        const int u = u0 + 32 * j;
-        if (u < units) {
-          va[j] = __ldg(wrow + 2 * u);
-          vb[j] = __ldg(wrow + 2 * u + 1);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < kAhead; ++j) {
-        const int u = u0 + 32 * j;
-        if (u >= units) break;
-        const uint32_t wd[8] = {va[j].x, va[j].y, va[j].z, va[j].w, vb[j].x, vb[j].y, vb[j].z, vb[j].w};
+  {
+    int row = row0, u = u0;
+    const bool ok = qw_pass(ring, [&](int c, const uint8_t* stage, int units_here) {
+      if (t < units_here) {
+        uint32_t wd[8];
+        qw_load_unit(stage, t, wd);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           d0 += __hiloint2double((int)(((wd[i] & 0x7FFFu) << 13) + kF64Rebias), 0);
@@ -262,30 +358,41 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
           }
           const uint32_t keep = unit_keep_bits<M>(h, n);
           *reinterpret_cast<uint16_t*>(meta + (size_t)row * meta_stride + 2 * u) = (uint16_t)keep;
+          const int li = c * kQwThreads + t;
+          if (li < kQwKeepCap) s_keep[li] = (uint16_t)keep;
         }
       }
-    }
+      advance(row, u);
+    });
+    if (!ok) return;
   }
   double dsum = d0 + d1;
 #pragma unroll
   for (int o = 16; o; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
   if (lane == 0) swarp_d[warp] = dsum;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (t == 0) {
     double a = 0.0;
-    for (int i = 0; i < kWarps; ++i) a += swarp_d[i];
+    for (int i = 0; i < kQwWarps; ++i) a += swarp_d[i];
     atomicAdd(gsum, a);
   }
-  if (!grid_barrier(arrive, gridDim.x, &s_abort)) return;
+  // the second pass re-reads the same range (now mostly in L2): start it
+  // before the grid barrier
+  qw_prologue(ring);
+  if (!grid_barrier(arrive, gridDim.x, &s_abort)) {
+    qw_pass(ring, [](int, const uint8_t*, int) {});   // drain the prefetched stages
+    return;
+  }
 
   // ---- gamma: certified from the fp64 total, else exact ---------------------
-  if (threadIdx.x == 0) {
+  if (t == 0) {
     const double S = __ldcg(gsum);
     const double nk = (double)n_out * (double)k;
-    // additions on the longest path: per-thread accumulator, 2 -> 1, warp
-    // tree, CTA sum, one global atomic per CTA
-    const int per_thread = ((rows_per_cta + kWarps - 1) / kWarps) * ((units + 31) / 32) * 8;
-    const double adds = (double)per_thread + 1.0 + 5.0 + kWarps + (double)gridDim.x;
+    // additions on the longest path: per-thread accumulator (8 per unit, one
+    // unit per chunk), d0 + d1, warp tree, CTA sum, one global atomic per CTA
+    const long long max_units = (total_units + gridDim.x - 1) / gridDim.x;
+    const double per_thread = 8.0 * (double)((max_units + kQwThreads - 1) / kQwThreads);
+    const double adds = per_thread + 1.0 + 5.0 + kQwWarps + (double)gridDim.x;
     const double err = S * adds * 0x1p-53 * 1.01 + nk * 0x1p-126 * 1.01;
     const double lo = (S - err) / nk * (1.0 - 0x1p-50);
     const double hi = (S + err) / nk * (1.0 + 0x1p-50);
@@ -299,30 +406,29 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   }
   __syncthreads();
   if (s_exact) {
-    // rare: exact integer bins over the same rows (from L2), second barrier
-    for (int i = threadIdx.x; i < kQwBins; i += blockDim.x) sbins[i] = 0ull;
+    // rare: exact integer bins over the same range, second barrier
+    for (int i = t; i < kQwBins; i += kQwThreads) sbins[i] = 0ull;
     __syncthreads();
     unsigned long long acc = 0ull;
-    for (int row = r_begin + warp; row < r_end; row += kWarps) {
-      const uint4* wrow = reinterpret_cast<const uint4*>(w + (size_t)row * k);
-      for (int u = lane; u < units; u += 32) {
-        const uint4 a = __ldg(wrow + 2 * u);
-        const uint4 b = __ldg(wrow + 2 * u + 1);
-        const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const bool ok = qw_pass(ring, [&](int, const uint8_t* stage, int units_here) {
+      if (t < units_here) {
+        uint32_t wd[8];
+        qw_load_unit(stage, t, wd);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           exact_accumulate(wd[i] & 0x7FFFu, acc, sbins);
           exact_accumulate((wd[i] >> 16) & 0x7FFFu, acc, sbins);
         }
       }
-    }
+    });
+    if (!ok) return;
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) swarp[warp] = acc;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (t == 0) {
       unsigned long long a = 0ull;
-      for (int i = 0; i < kWarps; ++i) a += swarp[i];
+      for (int i = 0; i < kQwWarps; ++i) a += swarp[i];
       // a counts units of 2^(kWinLo-134): file it under exponents kWinLo,
       // kWinLo+21 and kWinLo+42 in 21-bit pieces so every bin stays small
       const unsigned long long mask21 = (1ull << 21) - 1ull;
@@ -331,9 +437,13 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
       if (a1) atomicAdd(&gbins[kWinLo + 21], a1);
       if (a2) atomicAdd(&gbins[kWinLo + 42], a2);
     }
-    for (int i = threadIdx.x; i < kQwBins; i += blockDim.x)
+    for (int i = t; i < kQwBins; i += kQwThreads)
       if (sbins[i]) atomicAdd(&gbins[i], sbins[i]);
-    if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort)) return;
+    qw_prologue(ring);
+    if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort)) {
+      qw_pass(ring, [](int, const uint8_t*, int) {});
+      return;
+    }
     if (warp == 0) {
       float g;
       uint32_t tau;
@@ -348,30 +458,35 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   const uint32_t tau = s_tau;
 
   // ---- phase 2: codes of the kept positions ---------------------------------
-  const int cb = 4 * n / M;
-  uint4* sc4 = reinterpret_cast<uint4*>(s_codes[warp]);
-  for (int row = r_begin + warp; row < r_end; row += kWarps) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(w + (size_t)row * k);
-    const uint16_t* mrow = reinterpret_cast<const uint16_t*>(meta + (size_t)row * meta_stride);
-    for (int seg = 0; seg < units; seg += kSeg) {
-      const int seg_units = min(kSeg, units - seg);
-      for (int i = lane; i < kSeg * 4 / 16; i += 32) sc4[i] = make_uint4(0u, 0u, 0u, 0u);
-      __syncwarp();
-      for (int u = lane; u < seg_units; u += 32) {
-        const uint4 a = __ldg(wrow + 2 * (seg + u));
-        const uint4 b = __ldg(wrow + 2 * (seg + u) + 1);
-        const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        const uint32_t keep = has_meta ? (uint32_t)mrow[seg + u] : 0xFFFFu;
+  {
+    int row = row0, u = u0;
+    qw_pass(ring, [&](int c, const uint8_t* stage, int units_here) {
+      if (t < units_here) {
+        uint32_t wd[8];
+        qw_load_unit(stage, t, wd);
+        uint32_t keep = 0xFFFFu;
+        if (has_meta) {
+          const int li = c * kQwThreads + t;
+          keep = (li < kQwKeepCap)
+                     ? (uint32_t)s_keep[li]
+                     : (uint32_t) * reinterpret_cast<const uint16_t*>(meta + (size_t)row * meta_stride + 2 * u);
+        }
         const uint32_t packed = compact_codes16<M>(dense_codes16(wd, tau), keep, n, s_rm);
-        for (int bb = 0; bb < cb; ++bb) s_codes[warp][u * cb + bb] = (uint8_t)(packed >> (8 * bb));
+        uint8_t* dst = codes + (size_t)row * codes_stride + (size_t)u * cb;
+        if (cb == 4) {
+          *reinterpret_cast<uint32_t*>(dst) = packed;
+        } else if (cb == 2) {
+          *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+        } else {
+          for (int bb = 0; bb < cb; ++bb) dst[bb] = (uint8_t)(packed >> (8 * bb));
+        }
+        if (u == upr - 1) {
+          // zero padding at the end of the row
+          for (int i = upr * cb; i < codes_stride; ++i) codes[(size_t)row * codes_stride + i] = 0u;
+        }
       }
-      __syncwarp();
-      const int cstart = seg * cb;
-      const int cend = min(cstart + kSeg * cb, codes_stride);
-      uint4* cdst = reinterpret_cast<uint4*>(codes + (size_t)row * codes_stride + cstart);
-      for (int i = lane; i < (cend - cstart) / 16; i += 32) cdst[i] = sc4[i];
-      __syncwarp();
-    }
+      advance(row, u);
+    });
   }
 }
 

@@ -17,6 +17,8 @@
 #include "qw.cuh"
 #include "qw_fused.cuh"
 #include "bl_decode.cuh"
+#include "bl_decode_res.cuh"
+#include "expand_dense.cuh"
 #include "bl_tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -79,10 +81,24 @@ template <int M>
 sbn_status launch_qw_fused(const uint16_t* w, int n_out, int k, int n, uint8_t* codes, int cstride,
                            uint8_t* meta, int mstride, float* gamma, unsigned char* ws, int sms,
                            cudaStream_t st) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(qw_fused_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kQwSmemBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)sms);
-  cfg.blockDim = dim3(512);
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3(kQwThreads);
+  cfg.dynamicSmemBytes = kQwSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -154,6 +170,48 @@ sbn_status dispatch_decode(const DecodeParams& p, int n, int m, int sms, cudaStr
   return SBN_ERR_PATTERN;
 }
 
+// Resident decode kernel: grid = min(SMs, tiles), one CTA per SM holding the
+// packed rows of its tiles and all of Xq in shared memory.
+template <int MM, int CB, int NT, bool DENSE, bool ACC>
+sbn_status launch_decode_res(const DresParams& p, int grid, size_t smem, cudaStream_t st) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  auto kern = bl_decode_res_kernel<MM, CB, NT, DENSE, ACC>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDresSmemMax) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  kern<<<grid, kDresThreads, smem, st>>>(p);
+  return launch_status();
+}
+
+template <int NT, bool ACC>
+sbn_status dispatch_decode_res(const DresParams& p, int n, int m, int grid, size_t smem,
+                               cudaStream_t st) {
+  const int cb = 4 * n / m;
+  if (n == m) return launch_decode_res<8, 4, NT, true, ACC>(p, grid, smem, st);
+  switch (m * 8 + cb) {
+    case 4 * 8 + 1: return launch_decode_res<4, 1, NT, false, ACC>(p, grid, smem, st);
+    case 4 * 8 + 2: return launch_decode_res<4, 2, NT, false, ACC>(p, grid, smem, st);
+    case 4 * 8 + 3: return launch_decode_res<4, 3, NT, false, ACC>(p, grid, smem, st);
+    case 8 * 8 + 1: return launch_decode_res<8, 1, NT, false, ACC>(p, grid, smem, st);
+    case 8 * 8 + 2: return launch_decode_res<8, 2, NT, false, ACC>(p, grid, smem, st);
+    case 8 * 8 + 3: return launch_decode_res<8, 3, NT, false, ACC>(p, grid, smem, st);
+    case 16 * 8 + 1: return launch_decode_res<16, 1, NT, false, ACC>(p, grid, smem, st);
+    case 16 * 8 + 2: return launch_decode_res<16, 2, NT, false, ACC>(p, grid, smem, st);
+    case 16 * 8 + 3: return launch_decode_res<16, 3, NT, false, ACC>(p, grid, smem, st);
+  }
+  return SBN_ERR_PATTERN;
+}
+
 // cuTensorMapEncodeTiled from the driver, looked up once (no libcuda link).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -170,37 +228,74 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-template <int MM, int CB, bool DENSE, bool ACC>
-sbn_status launch_tc(const CUtensorMap& tm, const TcParams& p, int sms, cudaStream_t st) {
-  static bool attr_set = false;
-  auto kern = bl_tc_kernel<MM, CB, DENSE, ACC>;
-  if (!attr_set) {
+template <int MM, int CB, bool DENSE, bool ACC, bool TMA_A>
+sbn_status launch_tc(const CUtensorMap& tm, const CUtensorMap& tw, const TcParams& p, int sms,
+                     cudaStream_t st) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  auto kern = bl_tc_kernel<MM, CB, DENSE, ACC, TMA_A>;
+  if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes) !=
         cudaSuccess) {
       cudaGetLastError();
       return SBN_ERR_CUDA;
     }
-    attr_set = true;
+    attr_set[dev] = true;
   }
   const int tiles = ((p.N + kTcBM - 1) / kTcBM) * ((p.T + kTcBN - 1) / kTcBN);
-  kern<<<std::min(tiles, sms), kTcThreads, kTcSmemBytes, st>>>(tm, p);
+  kern<<<std::min(tiles, sms), kTcThreads, kTcSmemBytes, st>>>(tm, tw, p);
   return launch_status();
 }
 
+// Packed weights, expanded in the kernel (no workspace).
 template <bool ACC>
 sbn_status dispatch_tc(const CUtensorMap& tm, const TcParams& p, int n, int m, int sms, cudaStream_t st) {
   const int cb = 4 * n / m;
-  if (n == m) return launch_tc<8, 4, true, ACC>(tm, p, sms, st);
+  const CUtensorMap& unused = tm;
+  if (n == m) return launch_tc<8, 4, true, ACC, false>(tm, unused, p, sms, st);
   switch (m * 8 + cb) {
-    case 4 * 8 + 1: return launch_tc<4, 1, false, ACC>(tm, p, sms, st);
-    case 4 * 8 + 2: return launch_tc<4, 2, false, ACC>(tm, p, sms, st);
-    case 4 * 8 + 3: return launch_tc<4, 3, false, ACC>(tm, p, sms, st);
-    case 8 * 8 + 1: return launch_tc<8, 1, false, ACC>(tm, p, sms, st);
-    case 8 * 8 + 2: return launch_tc<8, 2, false, ACC>(tm, p, sms, st);
-    case 8 * 8 + 3: return launch_tc<8, 3, false, ACC>(tm, p, sms, st);
-    case 16 * 8 + 1: return launch_tc<16, 1, false, ACC>(tm, p, sms, st);
-    case 16 * 8 + 2: return launch_tc<16, 2, false, ACC>(tm, p, sms, st);
-    case 16 * 8 + 3: return launch_tc<16, 3, false, ACC>(tm, p, sms, st);
+    case 4 * 8 + 1: return launch_tc<4, 1, false, ACC, false>(tm, unused, p, sms, st);
+    case 4 * 8 + 2: return launch_tc<4, 2, false, ACC, false>(tm, unused, p, sms, st);
+    case 4 * 8 + 3: return launch_tc<4, 3, false, ACC, false>(tm, unused, p, sms, st);
+    case 8 * 8 + 1: return launch_tc<8, 1, false, ACC, false>(tm, unused, p, sms, st);
+    case 8 * 8 + 2: return launch_tc<8, 2, false, ACC, false>(tm, unused, p, sms, st);
+    case 8 * 8 + 3: return launch_tc<8, 3, false, ACC, false>(tm, unused, p, sms, st);
+    case 16 * 8 + 1: return launch_tc<16, 1, false, ACC, false>(tm, unused, p, sms, st);
+    case 16 * 8 + 2: return launch_tc<16, 2, false, ACC, false>(tm, unused, p, sms, st);
+    case 16 * 8 + 3: return launch_tc<16, 3, false, ACC, false>(tm, unused, p, sms, st);
+  }
+  return SBN_ERR_PATTERN;
+}
+
+// Expansion of the packed weights into the dense int8 workspace [N_out, K].
+template <int MM, int CB, bool DENSE>
+sbn_status launch_expand(const uint8_t* codes, const uint8_t* meta, int n_out, int k, int cstride,
+                         int mstride, int8_t* wd, int sms, cudaStream_t st) {
+  const long long units = (long long)n_out * (k / 16);
+  const long long want = (units + kXdThreads - 1) / kXdThreads;
+  const int grid = (int)std::max(1LL, std::min(want, (long long)sms * 4));
+  expand_dense_kernel<MM, CB, DENSE><<<grid, kXdThreads, 0, st>>>(codes, meta, n_out, k, cstride, mstride, wd);
+  return launch_status();
+}
+
+sbn_status dispatch_expand(const uint8_t* codes, const uint8_t* meta, int n_out, int k, int n, int m,
+                           int cstride, int mstride, int8_t* wd, int sms, cudaStream_t st) {
+  const int cb = 4 * n / m;
+  if (n == m) return launch_expand<8, 4, true>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+  switch (m * 8 + cb) {
+    case 4 * 8 + 1: return launch_expand<4, 1, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 4 * 8 + 2: return launch_expand<4, 2, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 4 * 8 + 3: return launch_expand<4, 3, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 8 * 8 + 1: return launch_expand<8, 1, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 8 * 8 + 2: return launch_expand<8, 2, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 8 * 8 + 3: return launch_expand<8, 3, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 16 * 8 + 1: return launch_expand<16, 1, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 16 * 8 + 2: return launch_expand<16, 2, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
+    case 16 * 8 + 3: return launch_expand<16, 3, false>(codes, meta, n_out, k, cstride, mstride, wd, sms, st);
   }
   return SBN_ERR_PATTERN;
 }
@@ -220,17 +315,51 @@ sbn_status make_act_tensor_map(CUtensorMap* tm, const int8_t* xq, int t, int k) 
   return r == CUDA_SUCCESS ? SBN_OK : SBN_ERR_CUDA;
 }
 
+// TMA map of the expanded int8 weights [N_out, K]: boxes of 128 rows x 128
+// bytes, 128-byte swizzle (the layout the A descriptor describes).
+sbn_status make_weight_tensor_map(CUtensorMap* tm, const int8_t* wd, int n_out, int k) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return SBN_ERR_CUDA;
+  cuuint64_t gdim[2] = {(cuuint64_t)k, (cuuint64_t)n_out};
+  cuuint64_t gstride[1] = {(cuuint64_t)k};
+  cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBM};
+  cuuint32_t estride[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(wd), gdim, gstride, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SBN_OK : SBN_ERR_CUDA;
+}
+
+// Bytes of the optional workspace of the contraction: the expanded weights
+// when t selects the tensor-core kernel, else none.
+size_t bitlinear_ws_bytes(int32_t t, int32_t k, int32_t n_out) {
+  return t > 16 ? (size_t)n_out * (size_t)k : 0;
+}
+
 template <bool ACC_OUT>
 sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k, int32_t n_out,
                          int32_t n, int32_t m, const uint8_t* codes, const uint8_t* meta,
-                         const float* gamma, uint16_t* y, int32_t* acc, int sms, cudaStream_t st) {
+                         const float* gamma, uint16_t* y, int32_t* acc, void* ws, int sms,
+                         cudaStream_t st) {
   const int cstride = (int)sbn_codes_row_bytes(k, n, m);
   const int mstride = (int)sbn_meta_row_bytes(k, n, m);
   if (t <= 16) {
+    // resident kernel when the largest CTA's rows and Xq fit in shared memory
+    const int tiles = (n_out + 15) / 16;
+    const int grid = std::min(sms, tiles);
+    const int per_cta = (tiles + grid - 1) / grid;
+    const int nt = t <= 8 ? 8 : 16;
+    const DresLayout L = dres_layout(per_cta, nt, k, cstride, mstride, n == m);
+    if (per_cta <= kDresMaxTiles && L.total <= kDresSmemMax) {
+      DresParams q;
+      q.xq = xq; q.xs = xs; q.codes = codes; q.meta = meta; q.gamma = gamma; q.y = y; q.acc_out = acc;
+      q.T = t; q.K = k; q.N = n_out; q.cstride = cstride; q.mstride = mstride; q.tiles_per_cta = per_cta;
+      return t <= 8 ? dispatch_decode_res<8, ACC_OUT>(q, n, m, grid, L.total, st)
+                    : dispatch_decode_res<16, ACC_OUT>(q, n, m, grid, L.total, st);
+    }
     DecodeParams p;
     p.xq = xq; p.xs = xs; p.codes = codes; p.meta = meta; p.gamma = gamma; p.y = y; p.acc_out = acc;
     p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
-    const int tiles = (n_out + 15) / 16;
     p.rt = std::min(kDecMaxRT, std::max(1, (tiles + sms - 1) / sms));
     return t <= 8 ? dispatch_decode<8, ACC_OUT>(p, n, m, sms, st)
                   : dispatch_decode<16, ACC_OUT>(p, n, m, sms, st);
@@ -241,7 +370,30 @@ sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k
   TcParams p;
   p.codes = codes; p.meta = meta; p.xs = xs; p.gamma = gamma; p.y = y; p.acc_out = acc;
   p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
+  if (ws) {
+    // expand once into the workspace, then TMA both operands
+    int8_t* wd = reinterpret_cast<int8_t*>(ws);
+    sbn_status s2 = dispatch_expand(codes, meta, n_out, k, n, m, cstride, mstride, wd, sms, st);
+    if (s2 != SBN_OK) return s2;
+    CUtensorMap tw;
+    if ((s2 = make_weight_tensor_map(&tw, wd, n_out, k)) != SBN_OK) return s2;
+    return launch_tc<8, 4, true, ACC_OUT, true>(tm, tw, p, sms, st);
+  }
   return dispatch_tc<ACC_OUT>(tm, p, n, m, sms, st);
+}
+
+// The workspace argument of the contraction: NULL (no expansion buffer), or
+// 16-byte aligned and at least bitlinear_ws_bytes long. Unused (NULL) for t <= 16.
+sbn_status check_bitlinear_ws(int32_t t, int32_t k, int32_t n_out, void*& ws, size_t ws_bytes) {
+  if (!ws) return SBN_OK;
+  const size_t need = bitlinear_ws_bytes(t, k, n_out);
+  if (need == 0) {
+    ws = nullptr;
+    return SBN_OK;
+  }
+  if (!aligned16(ws)) return SBN_ERR_ALIGN;
+  if (ws_bytes < need) return SBN_ERR_WORKSPACE;
+  return SBN_OK;
 }
 
 sbn_status validate_bitlinear(const int8_t* xq, int32_t t, int32_t k, int32_t n_out, int32_t n,
@@ -355,31 +507,39 @@ sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k, int8_t* x
   return launch_status();
 }
 
+size_t sbn_bitlinear_workspace_bytes(int32_t t, int32_t k, int32_t n_out) {
+  if (t < 1 || k < 1 || n_out < 1) return 0;
+  return bitlinear_ws_bytes(t, k, n_out);
+}
+
 sbn_status sbn_bitlinear(const int8_t* xq, const float* x_scale, int32_t t, int32_t k, int32_t n_out,
                          int32_t n, int32_t m, const uint8_t* codes, const uint8_t* meta,
-                         const float* gamma, void* y_bf16, void* stream) {
+                         const float* gamma, void* y_bf16, void* workspace, size_t ws_bytes,
+                         void* stream) {
   if (!x_scale || !gamma || !y_bf16) return SBN_ERR_NULL;
   sbn_status st = validate_bitlinear(xq, t, k, n_out, n, m, codes, meta);
   if (st != SBN_OK) return st;
   if (!aligned16(y_bf16)) return SBN_ERR_ALIGN;
+  if ((st = check_bitlinear_ws(t, k, n_out, workspace, ws_bytes)) != SBN_OK) return st;
   int dev = 0, sms = 0;
   if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
   return run_bitlinear<false>(xq, x_scale, t, k, n_out, n, m, codes, meta, gamma,
-                              reinterpret_cast<uint16_t*>(y_bf16), nullptr, sms,
+                              reinterpret_cast<uint16_t*>(y_bf16), nullptr, workspace, sms,
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_bitlinear_acc32(const int8_t* xq, int32_t t, int32_t k, int32_t n_out, int32_t n,
                                int32_t m, const uint8_t* codes, const uint8_t* meta, int32_t* acc,
-                               void* stream) {
+                               void* workspace, size_t ws_bytes, void* stream) {
   if (!acc) return SBN_ERR_NULL;
   sbn_status st = validate_bitlinear(xq, t, k, n_out, n, m, codes, meta);
   if (st != SBN_OK) return st;
   if (!aligned16(acc)) return SBN_ERR_ALIGN;
+  if ((st = check_bitlinear_ws(t, k, n_out, workspace, ws_bytes)) != SBN_OK) return st;
   int dev = 0, sms = 0;
   if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
   return run_bitlinear<true>(xq, nullptr, t, k, n_out, n, m, codes, meta, nullptr, nullptr, acc,
-                             sms, reinterpret_cast<cudaStream_t>(stream));
+                             workspace, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // Allocation-free variant of sbn_quantize_weights. Its scratch is a fixed

@@ -44,9 +44,10 @@ PROTOTYPES = {
                                                     _c_p, _c_p, _c_p]),
     "sbn_quantize_acts": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p]),
     "sbn_bitlinear": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
-                                     _c_p, _c_p, _c_p, _c_p]),
+                                     _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "sbn_bitlinear_workspace_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32]),
     "sbn_bitlinear_acc32": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
-                                           _c_p, _c_p, _c_p]),
+                                           _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
 
@@ -183,8 +184,24 @@ def quantize_acts(x: torch.Tensor, out_q: Optional[torch.Tensor] = None,
     return out_q, out_s
 
 
+def bitlinear_workspace_bytes(t: int, k: int, n_out: int) -> int:
+    """Bytes of the contraction's optional workspace (0 when T <= 16)."""
+    return int(lib().sbn_bitlinear_workspace_bytes(t, k, n_out))
+
+
+def _bitlinear_ws(workspace, t: int, k: int, n_out: int, device):
+    """None: allocate the workspace (expanded-weights route); False: no
+    workspace (weights expanded inside the kernel); else the given tensor."""
+    if workspace is False:
+        return None
+    if workspace is None:
+        nb = bitlinear_workspace_bytes(t, k, n_out)
+        return torch.empty((nb,), dtype=torch.uint8, device=device) if nb else None
+    return workspace
+
+
 def bitlinear(xq: torch.Tensor, s: torch.Tensor, w: PackedWeights,
-              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+              out: Optional[torch.Tensor] = None, workspace=None, stream=None) -> torch.Tensor:
     """sbn_bitlinear: y[t, o] = bf16(acc * gamma * s_t / 127)."""
     _need(xq, torch.int8, "xq")
     _need(s, torch.float32, "s")
@@ -193,21 +210,25 @@ def bitlinear(xq: torch.Tensor, s: torch.Tensor, w: PackedWeights,
         raise ValueError("K mismatch between activations and weights")
     if out is None:
         out = torch.empty((t, w.n_out), dtype=torch.bfloat16, device=xq.device)
+    ws = _bitlinear_ws(workspace, t, k, w.n_out, xq.device)
     st = lib().sbn_bitlinear(_ptr(xq), _ptr(s), t, k, w.n_out, w.n, w.m, _ptr(w.codes),
-                             _ptr(w.meta), _ptr(w.gamma), _ptr(out), _stream_ptr(stream))
+                             _ptr(w.meta), _ptr(w.gamma), _ptr(out), _ptr(ws),
+                             0 if ws is None else ws.numel(), _stream_ptr(stream))
     _check(st, "sbn_bitlinear")
     return out
 
 
 def bitlinear_acc32(xq: torch.Tensor, w: PackedWeights, out: Optional[torch.Tensor] = None,
-                    stream=None) -> torch.Tensor:
+                    workspace=None, stream=None) -> torch.Tensor:
     """sbn_bitlinear_acc32: the exact int32 accumulators [T, N_out]."""
     _need(xq, torch.int8, "xq")
     t, k = xq.shape
     if out is None:
         out = torch.empty((t, w.n_out), dtype=torch.int32, device=xq.device)
+    ws = _bitlinear_ws(workspace, t, k, w.n_out, xq.device)
     st = lib().sbn_bitlinear_acc32(_ptr(xq), t, k, w.n_out, w.n, w.m, _ptr(w.codes),
-                                   _ptr(w.meta), _ptr(out), _stream_ptr(stream))
+                                   _ptr(w.meta), _ptr(out), _ptr(ws),
+                                   0 if ws is None else ws.numel(), _stream_ptr(stream))
     _check(st, "sbn_bitlinear_acc32")
     return out
 

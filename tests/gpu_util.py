@@ -33,13 +33,15 @@ def packed_to_numpy(pw):
     return codes, meta, gamma
 
 
-def run_layer(w_bits, x_bits, n, m, want_acc=True):
-    """All three calls; returns numpy copies of every intermediate."""
+def run_layer(w_bits, x_bits, n, m, want_acc=True, workspace=None):
+    """All three calls; returns numpy copies of every intermediate.
+    workspace=None: the contraction gets a workspace (for T > 16 the weights
+    are expanded into it first); workspace=False: none (expanded in-kernel)."""
     from sparse_linear_layers_fwd_b200 import sbn
     pw = run_quantize_weights(w_bits, n, m)
     xq, s = sbn.quantize_acts(to_dev_bf16(x_bits))
-    y = sbn.bitlinear(xq, s, pw)
-    acc = sbn.bitlinear_acc32(xq, pw) if want_acc else None
+    y = sbn.bitlinear(xq, s, pw, workspace=workspace)
+    acc = sbn.bitlinear_acc32(xq, pw, workspace=workspace) if want_acc else None
     torch.cuda.synchronize()
     assert sbn.get_device_error() == 0
     codes, meta, gamma = packed_to_numpy(pw)
@@ -63,8 +65,8 @@ def assert_weights_exact(g, ref_codes, ref_meta, ref_gamma):
     assert np.array_equal(g["codes"], ref_codes), "codes differ"
 
 
-def full_parity(w_bits, x_bits, n, m):
-    g = run_layer(w_bits, x_bits, n, m)
+def full_parity(w_bits, x_bits, n, m, workspace=None):
+    g = run_layer(w_bits, x_bits, n, m, workspace=workspace)
     cb, mb, gamma, mask, dense = oracle.quantize_weights(w_bits, n, m)
     assert_weights_exact(g, cb, mb, gamma)
     q, s = oracle.quantize_acts(x_bits)

@@ -97,7 +97,8 @@ def test_bitlinear_validation(sbn_lib):
     def bl(**kw):
         a = dict(ok, **kw)
         return lib.sbn_bitlinear(a["xq"], a["s"], a["t"], a["k"], a["n_out"], a["n"], a["m"],
-                                 a["codes"], a["meta"], a["g"], a["y"], None)
+                                 a["codes"], a["meta"], a["g"], a["y"], a.get("ws"),
+                                 a.get("ws_bytes", 0), None)
     assert bl(xq=None) == 1
     assert bl(y=None) == 1
     assert bl(meta=None) == 1
@@ -106,7 +107,15 @@ def test_bitlinear_validation(sbn_lib):
     assert bl(t=0) == 2
     assert bl(k=100) == 2
     assert bl(xq=MIS) == 4
-    assert lib.sbn_bitlinear_acc32(A, 4, 256, 64, 2, 4, A, A, None, None) == 1
+    # the optional workspace: used (and checked) only when T > 16
+    need = lib.sbn_bitlinear_workspace_bytes(64, 256, 64)
+    assert need == 64 * 256
+    assert lib.sbn_bitlinear_workspace_bytes(16, 256, 64) == 0
+    assert bl(t=64, ws=MIS, ws_bytes=need) == 4
+    assert bl(t=64, ws=A, ws_bytes=need - 1) == 5
+    assert bl(t=4, ws=MIS, ws_bytes=0) not in (4, 5)       # ignored for decode
+    assert lib.sbn_bitlinear_acc32(A, 4, 256, 64, 2, 4, A, A, None, None, 0, None) == 1
+    assert lib.sbn_bitlinear_acc32(A, 64, 256, 64, 2, 4, A, A, A, A, need - 1, None) == 5
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")

@@ -38,6 +38,26 @@ def test_patterns_and_ragged_shapes(nm, shape):
     full_parity(w, x, *nm)
 
 
+@pytest.mark.parametrize("nm", SUPPORTED)
+@pytest.mark.parametrize("shape", [s for s in SHAPES if s[0] > 16])
+def test_tensor_core_without_workspace(nm, shape):
+    """T > 16 without a workspace: the weights are expanded inside the
+    tensor-core kernel instead of into the workspace first."""
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=13, tag=f"nows{nm}{shape}")
+    x = synth.activations(t, k, seed=13, tag=f"nows{nm}{shape}", outlier_channels=2)
+    full_parity(w, x, *nm, workspace=False)
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_prefill_sampled_without_workspace(which):
+    d = synth.prefill(which)
+    g = run_layer(d["w"], d["x"], d["n"], d["m"], workspace=False)
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(d["w"], d["n"], d["m"])
+    q, s = oracle.quantize_acts(d["x"])
+    _sampled_check(g, q, s, dense, gamma, d["x"].shape[0], d["w"].shape[0], seed=21)
+
+
 @pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (8, 8)])
 def test_all_zero_weights(nm):
     w = np.zeros((40, 256), np.uint16)
@@ -113,6 +133,17 @@ def test_repeated_calls_reuse_workspace():
 # ---------------------------------------------------------------------------
 # the workloads at full size
 # ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape,nm", [((16, 11008, 40), (6, 8)), ((9, 11008, 17), (8, 16)),
+                                      ((12, 11008, 33), (8, 8))])
+def test_decode_streaming_kernel(shape, nm):
+    """Token counts and K whose activations do not fit next to the weights in
+    shared memory take the streaming decode kernel."""
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=12, tag=f"stream{shape}")
+    x = synth.activations(t, k, seed=12, tag=f"stream{shape}", outlier_channels=3)
+    full_parity(w, x, *nm)
+
 
 @pytest.fixture(scope="module")
 def decode_ref():
