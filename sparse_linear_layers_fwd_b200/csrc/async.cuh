@@ -6,6 +6,7 @@
 namespace sbn {
 
 constexpr unsigned long long kMbarWaitNs = 250000000ull;  // an mbarrier wait gives up after 0.25 s
+constexpr uint32_t kMbarSuspendNs = 20000;                 // suspend-time hint of one try_wait
 
 SBN_DEVFN uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -21,24 +22,26 @@ SBN_DEVFN void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 // Wait for the phase of the given parity, bounded in time (kMbarWaitNs); false
-// (and SBN_ERR_TIMEOUT in the device error word) if it gave up. Polls with the
-// non-blocking test_wait so the thread sees the phase change at once.
+// (and SBN_ERR_TIMEOUT in the device error word) if it gave up. try_wait
+// suspends the thread until the phase completes or the hinted time passes,
+// so a waiting thread does not spin. Kernels let one thread (or one lane
+// per warp) wait and the others meet it at a barrier: the phase completion
+// it observes, followed by the barrier, orders the arrived data before the
+// others' reads.
 SBN_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
   unsigned long long t0 = 0;
   for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
-        "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(done)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(kMbarSuspendNs)
         : "memory");
     if (done) return true;
-    if ((i & 63u) == 0u) {
-      const unsigned long long t = global_ns();
-      if (i == 0u) t0 = t;
-      else if (t - t0 > kMbarWaitNs) break;
-    }
+    const unsigned long long t = global_ns();
+    if (i == 0u) t0 = t;
+    else if (t - t0 > kMbarWaitNs) break;
   }
   atomicOr(&g_dev_error, kDevErrTimeout);
   return false;

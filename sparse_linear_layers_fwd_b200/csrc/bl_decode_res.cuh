@@ -7,12 +7,12 @@
 // unpacked there and contracted with 8-bit activations, so HBM carries only
 // the packed bytes. Decoding is bound by those bytes.
 //
-// A CTA owns a contiguous range of 16-row tiles. Thread 0 issues, at once:
-// one bulk copy per token row of Xq (into rows padded by 16 bytes against
-// bank conflicts), then per tile one copy of its code rows and one of its
-// keep-bit rows, each tile completing its own mbarrier. The 32 warps walk
-// the (tile, 128-position segment) items in tile-major order, so the first
-// tiles are contracted while later ones are still arriving. Per item a thread
+// A CTA owns a contiguous range of 16-row tiles. Thread 0 issues, at once,
+// a few large bulk copies (each copy has a fixed cost, so few and large beats
+// many and small): all of Xq in one, then the code rows and the keep-bit rows
+// of the tiles in at most two groups, each group completing its own mbarrier.
+// The 32 warps walk the (tile, 128-position segment) items in tile-major
+// order, so the first group is contracted while the second is arriving. Per item a thread
 // expands 32 positions of two rows (expand.cuh) straight into the A fragment
 // of `mma.sync.m16n8k32.s8` (weights as the 16-row operand, tokens as the 8
 // columns, a K permutation shared with the activation fragment). A warp adds
@@ -41,7 +41,7 @@ struct DresLayout {
 __host__ __device__ inline DresLayout dres_layout(int tiles, int nt, int k, int cstride, int mstride,
                                                   bool dense) {
   DresLayout L;
-  L.xstride = k + 16;
+  L.xstride = k;
   L.sel = 0;
   L.acc = 1024;
   L.x = L.acc + (size_t)tiles * 16 * nt * 4;
@@ -90,34 +90,41 @@ bl_decode_res_kernel(const DresParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int row0 = t_begin * 16;
+  // tiles [0, split) form copy group 0, [split, tiles) group 1 (if any)
+  const int ngrp = tiles > 1 ? 2 : 1;
+  const int split = ngrp == 2 ? tiles / 2 : tiles;
 
   if (tid == 0) {
+    // the copies start at once; the other threads meet the barriers after
+    // the block-wide sync below
     mbar_init(bar_x, 1);
-    for (int i = 0; i < tiles; ++i) mbar_init(&bar_t[i], 1);
+    for (int i = 0; i < ngrp; ++i) mbar_init(&bar_t[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
-  __syncthreads();
-  if (tid == 0) {
     mbar_arrive_expect_tx(bar_x, (uint32_t)(p.T * p.K));
-    for (int tok = 0; tok < p.T; ++tok)
-      bulk_g2s(s_x + (size_t)tok * L.xstride, p.xq + (size_t)tok * p.K, (uint32_t)p.K, bar_x);
-    for (int i = 0; i < tiles; ++i) {
-      const int r = row0 + 16 * i;
-      const int nrows = min(16, p.N - r);
+    bulk_g2s(s_x, p.xq, (uint32_t)(p.T * p.K), bar_x);
+    for (int gi = 0; gi < ngrp; ++gi) {
+      const int ta = gi ? split : 0, tb = gi ? tiles : split;
+      const int r = row0 + 16 * ta;
+      const int nrows = min(16 * (tb - ta), p.N - r);
       const uint32_t cbytes = (uint32_t)(nrows * p.cstride);
       const uint32_t mbytes = DENSE ? 0u : (uint32_t)(nrows * p.mstride);
-      mbar_arrive_expect_tx(&bar_t[i], cbytes + mbytes);
-      bulk_g2s(s_codes + (size_t)i * 16 * p.cstride, p.codes + (size_t)r * p.cstride, cbytes, &bar_t[i]);
+      mbar_arrive_expect_tx(&bar_t[gi], cbytes + mbytes);
+      bulk_g2s(s_codes + (size_t)ta * 16 * p.cstride, p.codes + (size_t)r * p.cstride, cbytes, &bar_t[gi]);
       if (!DENSE)
-        bulk_g2s(s_meta + (size_t)i * 16 * p.mstride, p.meta + (size_t)r * p.mstride, mbytes, &bar_t[i]);
+        bulk_g2s(s_meta + (size_t)ta * 16 * p.mstride, p.meta + (size_t)r * p.mstride, mbytes, &bar_t[gi]);
     }
   }
   if (!DENSE) fill_selector_table(s_sel);
   for (int i = tid; i < tiles * 16 * NT; i += kDresThreads) s_acc[i] = 0;
   __syncthreads();
 
-  // a wait's verdict is made warp-uniform (the MMAs need the whole warp)
-  bool ok = __all_sync(0xffffffffu, mbar_wait(bar_x, 0u));
+  // lane 0 waits, the warp follows it (the MMAs need the whole warp)
+  auto warp_wait = [&](uint64_t* bar) {
+    int got = 1;
+    if (lane == 0) got = mbar_wait(bar, 0u) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, got, 0) != 0;
+  };
+  bool ok = warp_wait(bar_x);
   const int ksegs = p.K / 128;
   const int items = tiles * ksegs;
   int cur_tile = -1;
@@ -144,7 +151,7 @@ bl_decode_res_kernel(const DresParams p) {
     if (tile != cur_tile) {
       if (cur_tile >= 0) flush(cur_tile);
       cur_tile = tile;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_t[tile], 0u))) { ok = false; break; }
+      if (!warp_wait(&bar_t[tile < split ? 0 : 1])) { ok = false; break; }
     }
     const uint8_t* ct = s_codes + (size_t)tile * 16 * p.cstride;
     const uint8_t* mt = s_meta + (size_t)tile * 16 * p.mstride;
@@ -192,7 +199,7 @@ bl_decode_res_kernel(const DresParams p) {
   if (tid == 0) {
     // every copy of this CTA has landed before the CTA may exit
     mbar_wait(bar_x, 0u);
-    for (int i = 0; i < tiles; ++i) mbar_wait(&bar_t[i], 0u);
+    for (int i = 0; i < ngrp; ++i) mbar_wait(&bar_t[i], 0u);
   }
   __syncthreads();
 

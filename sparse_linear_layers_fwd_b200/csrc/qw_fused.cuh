@@ -35,8 +35,9 @@ namespace sbn {
 
 // Workspace offsets beyond the bins and tau of qw.cuh.
 constexpr size_t kQwArriveOffset = kQwTauOffset + 16;   // u32 arrival counter
-constexpr size_t kQwSumOffset = kQwArriveOffset + 16;   // f64 total of |w|
-constexpr size_t kQwClearBytes = kQwSumOffset + 16;     // cleared before every launch
+constexpr size_t kQwClearBytes = kQwArriveOffset + 16;  // cleared before every launch
+constexpr size_t kQwPartOffset = 2304;                  // f64 partial sum of |w| per CTA
+constexpr int kQwMaxGrid = (int)((kQwWorkspaceBytes - kQwPartOffset) / 8);
 constexpr unsigned long long kQwWaitNs = 1000000000ull;  // the grid barrier gives up after 1 s
 
 SBN_DEVFN uint32_t ld_acquire_u32(const uint32_t* p) {
@@ -56,7 +57,7 @@ SBN_DEVFN bool grid_barrier(uint32_t* arrive, uint32_t target, int* s_abort) {
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    atomicAdd(arrive, 1u);
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;\n" ::"l"(arrive) : "memory");
     const unsigned long long t0 = global_ns();
     int abort = 0;
     while (ld_acquire_u32(arrive) < target) {
@@ -135,69 +136,122 @@ SBN_DEVFN uint32_t unit_keep_bits(const uint32_t (&h)[16], int n) {
   return keep;
 }
 
-// Dense 2-bit codes of 16 positions (code of position i in bits 2i..2i+1):
-// 01 where |w| > tau and w > 0, 11 where |w| > tau and w < 0, else 00. The
-// comparison is one bf16x2 compare per pair of magnitudes.
-SBN_DEVFN uint32_t dense_codes16(const uint32_t (&wd)[8], uint32_t tau) {
-  const __nv_bfloat162 t2 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)tau),
-                                               __ushort_as_bfloat16((unsigned short)tau));
-  uint32_t d = 0u;
+// Packed pairs of bf16 magnitudes (sign bits clear) as raw 32-bit words.
+// Their float order equals the order of their bit patterns.
+SBN_DEVFN __nv_bfloat162 as_bf2(uint32_t x) {
+  __nv_bfloat162 r;
+  memcpy(&r, &x, 4);
+  return r;
+}
+SBN_DEVFN uint32_t as_u32(__nv_bfloat162 x) {
+  uint32_t r;
+  memcpy(&r, &x, 4);
+  return r;
+}
+SBN_DEVFN uint32_t bmin2(uint32_t a, uint32_t b) { return as_u32(__hmin2(as_bf2(a), as_bf2(b))); }
+SBN_DEVFN uint32_t bmax2(uint32_t a, uint32_t b) { return as_u32(__hmax2(as_bf2(a), as_bf2(b))); }
+SBN_DEVFN uint32_t ble2(uint32_t a, uint32_t b) { return __hle2_mask(as_bf2(a), as_bf2(b)); }
+SBN_DEVFN uint32_t swap16(uint32_t a) { return __byte_perm(a, 0u, 0x1032u); }
+
+// Pruned positions (bit j = element j) of one group of 8 magnitudes held as
+// four pairs (w0 = elements 0,1; ...): the two smallest. The second
+// smallest a2 comes from a min/max network on the pairs; the elements with
+// magnitude <= a2 are exactly the two smallest unless the third smallest
+// equals a2 -- then false is returned and the caller ranks the group exactly.
+SBN_DEVFN bool prune_2of8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t& prune) {
+  const uint32_t m01 = bmin2(w0, w1), M01 = bmax2(w0, w1);
+  const uint32_t m23 = bmin2(w2, w3), M23 = bmax2(w2, w3);
+  const uint32_t s1 = bmin2(m01, m23);                               // smallest per half
+  const uint32_t s2 = bmin2(bmax2(m01, m23), bmin2(M01, M23));       // second per half
+  const uint32_t a2 = bmin2(bmax2(s1, swap16(s1)), bmin2(s2, swap16(s2)));
+  const uint32_t P = (ble2(w0, a2) & 0x00010001u) | ((ble2(w1, a2) & 0x00010001u) << 2) |
+                     ((ble2(w2, a2) & 0x00010001u) << 4) | ((ble2(w3, a2) & 0x00010001u) << 6);
+  prune = (P | (P >> 15)) & 0xFFu;
+  return __popc(prune) == 2;
+}
+
+// The same for one group of 4 magnitudes held as two pairs.
+SBN_DEVFN bool prune_2of4(uint32_t w0, uint32_t w1, uint32_t& prune) {
+  const uint32_t m = bmin2(w0, w1), M = bmax2(w0, w1);
+  const uint32_t a2 = bmin2(bmax2(m, swap16(m)), bmin2(M, swap16(M)));
+  const uint32_t P = (ble2(w0, a2) & 0x00010001u) | ((ble2(w1, a2) & 0x00010001u) << 2);
+  prune = (P | (P >> 15)) & 0xFu;
+  return __popc(prune) == 2;
+}
+
+// Keep bits of one unit (16 magnitudes as 8 pairs) for 6:8 and 2:4 through
+// the networks above; other patterns, and groups where the boundary ties,
+// go through the exact rank selection.
+template <int M>
+SBN_DEVFN uint32_t unit_keep_fast(const uint32_t (&mw)[8], int n) {
+  if (M == 8 && n == 6) {
+    uint32_t p0, p1;
+    const bool a = prune_2of8(mw[0], mw[1], mw[2], mw[3], p0);
+    const bool b = prune_2of8(mw[4], mw[5], mw[6], mw[7], p1);
+    if (a && b) return (~(p0 | (p1 << 8))) & 0xFFFFu;
+  } else if (M == 4 && n == 2) {
+    uint32_t keep = 0u;
+    bool ok = true;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint32_t pr;
+      ok &= prune_2of4(mw[2 * g], mw[2 * g + 1], pr);
+      keep |= ((~pr) & 0xFu) << (4 * g);
+    }
+    if (ok) return keep;
+  }
+  uint32_t h[16];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t mg = wd[i] & 0x7FFF7FFFu;
-    const uint32_t gt = __hgt2_mask(*reinterpret_cast<const __nv_bfloat162*>(&mg), t2);
-    // per half: bit 0 = nonzero, bit 1 = nonzero and negative
-    const uint32_t c = (gt & 0x00010001u) | ((gt & wd[i] & 0x80008000u) >> 14);
-    d |= ((c & 3u) | ((c >> 14) & 0xCu)) << (4 * i);
+    h[2 * i] = mw[i] & 0xFFFFu;
+    h[2 * i + 1] = mw[i] >> 16;
   }
-  return d;
+  return unit_keep_bits<M>(h, n);
 }
 
-// Remove one 2-bit field of x: fields below low_mask stay, higher ones move down.
-SBN_DEVFN uint32_t remove_field(uint32_t x, uint32_t low_mask) {
-  return (x & low_mask) | ((x >> 2) & ~low_mask);
-}
+// Four bytes with values in {0, 1, 3} -> their low two bits packed into 8
+// bits (byte i to bits 2i, 2i+1): one multiply collects the fields.
+SBN_DEVFN uint32_t pack4_2bit(uint32_t x) { return (x * 0x01041040u) >> 24; }
 
-// Kept codes, in order, of 16 positions from their dense codes and keep bits.
-template <int M>
-SBN_DEVFN uint32_t compact_codes16(uint32_t d, uint32_t keep, int n, const uint32_t* s_rm) {
-  if (n == M) return d;
-  if (M == 8 && n == 6) {
-    // per byte of keep bits, remove the two pruned fields (higher one first)
-    uint32_t out = 0u;
+// Kept codes of one unit, in order, from its 16 latent values (8 pairs), the
+// threshold tau and the keep bits: per element a code byte (0 for |w| <=
+// tau, else 1 or 3 by sign), then per 8 positions the kept bytes gathered
+// by a byte permute (selectors from s_csel) and packed to 2 bits each.
+SBN_DEVFN uint32_t unit_codes(const uint32_t (&wd)[8], uint32_t tau2, uint32_t keep,
+                              const uint32_t* s_csel) {
+  uint32_t B[4];
 #pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      const uint32_t r = s_rm[(keep >> (8 * g)) & 0xFFu];  // low masks: q in bits 0-15, p in 16-31
-      uint32_t x = (d >> (16 * g)) & 0xFFFFu;
-      x = remove_field(x, r & 0xFFFFu);
-      x = remove_field(x, r >> 16);
-      out |= (x & 0xFFFu) << (12 * g);
-    }
-    return out;
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t wa = wd[2 * j], wb = wd[2 * j + 1];
+    const uint32_t nza = __hgt2_mask(as_bf2(wa & 0x7FFF7FFFu), as_bf2(tau2));
+    const uint32_t nzb = __hgt2_mask(as_bf2(wb & 0x7FFF7FFFu), as_bf2(tau2));
+    const uint32_t nzB = __byte_perm(nza, nzb, 0x6420u);   // 0xFF per nonzero element
+    const uint32_t sB = __byte_perm(wa, wb, 0x7531u);      // high byte (sign in bit 7)
+    B[j] = nzB & (((sB >> 6) & 0x02020202u) | 0x01010101u);
   }
-  uint32_t out = 0u;
-  int j = 0;
+  uint32_t codes = 0u;
+  int sh = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if ((keep >> i) & 1u) {
-      out |= ((d >> (2 * i)) & 3u) << (2 * j);
-      ++j;
-    }
+  for (int b = 0; b < 2; ++b) {
+    const uint32_t kb = (keep >> (8 * b)) & 0xFFu;
+    const uint32_t sel = s_csel[kb];
+    const uint32_t r0 = __byte_perm(B[2 * b], B[2 * b + 1], sel & 0xFFFFu);
+    const uint32_t r1 = __byte_perm(B[2 * b], B[2 * b + 1], sel >> 16);
+    const int p = __popc(kb);
+    const uint32_t v = (pack4_2bit(r0) | (pack4_2bit(r1) << 8)) & ((1u << (2 * p)) - 1u);
+    codes |= v << sh;
+    sh += 2 * p;
   }
-  return out;
+  return codes;
 }
 
-// Removal masks of 6:8 groups: for keep byte k with pruned positions p < q,
-// entry = lowmask(q) | lowmask(p) << 16 where lowmask(j) = (1 << 2j) - 1.
-SBN_DEVFN void fill_remove_table(uint32_t* s_rm) {
+// Byte-gather selectors: nibble i of entry k = position of the i-th set bit of k.
+SBN_DEVFN void fill_compact_table(uint32_t* s_csel) {
   for (int k = threadIdx.x; k < 256; k += blockDim.x) {
-    uint32_t pr = (~(uint32_t)k) & 0xFFu, p = 0u, q = 0u;
-    if (__popc(pr) == 2) {
-      p = __ffs(pr) - 1;
-      pr &= pr - 1u;
-      q = __ffs(pr) - 1;
-    }
-    s_rm[k] = ((1u << (2 * q)) - 1u) | (((1u << (2 * p)) - 1u) << 16);
+    uint32_t s = 0u, i = 0u;
+    for (uint32_t pos = 0; pos < 8; ++pos)
+      if ((k >> pos) & 1) s |= pos << (4 * i++);
+    s_csel[k] = s;
   }
 }
 
@@ -211,8 +265,8 @@ constexpr int kQwChunk = 16384;       // bytes per stage
 constexpr int kQwStages = 8;          // 128 KB in flight per SM
 constexpr int kQwKeepCap = 16384;     // units whose keep bits stay in shared memory
 constexpr size_t kQwSmKeep = (size_t)kQwStages * kQwChunk;
-constexpr size_t kQwSmRm = kQwSmKeep + (size_t)kQwKeepCap * 2;
-constexpr size_t kQwSmBins = kQwSmRm + 256 * 4;
+constexpr size_t kQwSmCsel = kQwSmKeep + (size_t)kQwKeepCap * 2;
+constexpr size_t kQwSmBins = kQwSmCsel + 256 * 4;
 constexpr size_t kQwSmBars = kQwSmBins + (size_t)kQwBins * 8;
 constexpr size_t kQwSmemBytes = kQwSmBars + (size_t)kQwStages * 8;
 
@@ -241,18 +295,19 @@ SBN_DEVFN void qw_prologue(const QwRing& r) {
 }
 
 // One pass over the range, whose prologue is already issued: f(c, stage,
-// units_here) runs for every chunk on every thread, then the stage is
-// refilled with chunk c + kQwStages. If a wait gives up, the copies still in
-// flight are waited for (bounded) and false is returned on every thread.
+// units_here) runs for every chunk on every thread. Thread 0 alone waits for
+// a chunk; the block barrier after its wait publishes the chunk to the
+// others and frees the stage of the previous chunk, which thread 0 then
+// refills. If a wait gives up, the copies still in flight are waited for
+// (bounded) and false is returned on every thread.
 template <class F>
-SBN_DEVFN bool qw_pass(QwRing& r, F&& f) {
+SBN_DEVFN bool qw_pass(QwRing& r, int* s_ok, F&& f) {
   for (int c = 0; c < r.nch; ++c) {
     const uint32_t q = r.seq + (uint32_t)c;
     const int st = (int)(q % kQwStages);
-    const bool ok = mbar_wait(&r.full[st], (q / kQwStages) & 1u);
-    const int units_here = (int)(min((long long)kQwChunk, r.bytes - (long long)c * kQwChunk) >> 5);
-    if (ok) f(c, r.buf + (size_t)st * kQwChunk, units_here);
-    if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) *s_ok = mbar_wait(&r.full[st], (q / kQwStages) & 1u) ? 1 : 0;
+    __syncthreads();
+    if (!*s_ok) {
       if (threadIdx.x == 0) {
         for (int d = c + 1; d < min(r.nch, c + kQwStages); ++d) {
           const uint32_t qd = r.seq + (uint32_t)d;
@@ -262,8 +317,12 @@ SBN_DEVFN bool qw_pass(QwRing& r, F&& f) {
       __syncthreads();
       return false;
     }
-    if (threadIdx.x == 0 && c + kQwStages < r.nch) qw_issue(r, c + kQwStages, q + kQwStages);
+    if (threadIdx.x == 0 && c >= 1 && c - 1 + kQwStages < r.nch)
+      qw_issue(r, c - 1 + kQwStages, q - 1 + kQwStages);
+    const int units_here = (int)(min((long long)kQwChunk, r.bytes - (long long)c * kQwChunk) >> 5);
+    f(c, r.buf + (size_t)st * kQwChunk, units_here);
   }
+  __syncthreads();  // every thread is done with the last stages before they are reused
   r.seq += (uint32_t)r.nch;
   return true;
 }
@@ -286,17 +345,17 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
                 int meta_stride, float* __restrict__ gamma_out, unsigned char* __restrict__ ws) {
   extern __shared__ __align__(128) uint8_t qw_smem[];
   uint16_t* s_keep = reinterpret_cast<uint16_t*>(qw_smem + kQwSmKeep);
-  uint32_t* s_rm = reinterpret_cast<uint32_t*>(qw_smem + kQwSmRm);
+  uint32_t* s_csel = reinterpret_cast<uint32_t*>(qw_smem + kQwSmCsel);
   unsigned long long* sbins = reinterpret_cast<unsigned long long*>(qw_smem + kQwSmBins);
   uint64_t* full = reinterpret_cast<uint64_t*>(qw_smem + kQwSmBars);
   __shared__ double swarp_d[kQwWarps];
   __shared__ unsigned long long swarp[kQwWarps];
   __shared__ uint32_t s_tau;
-  __shared__ int s_abort, s_exact;
+  __shared__ int s_abort, s_exact, s_ok;
 
   unsigned long long* gbins = reinterpret_cast<unsigned long long*>(ws);
   uint32_t* arrive = reinterpret_cast<uint32_t*>(ws + kQwArriveOffset);
-  double* gsum = reinterpret_cast<double*>(ws + kQwSumOffset);
+  double* gpart = reinterpret_cast<double*>(ws + kQwPartOffset);
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int upr = k >> 4;                       // units per row
@@ -319,7 +378,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     for (int s = 0; s < kQwStages; ++s) mbar_init(&full[s], 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (M == 8 && n == 6) fill_remove_table(s_rm);
+  fill_compact_table(s_csel);
   __syncthreads();
   qw_prologue(ring);
 
@@ -340,23 +399,18 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   double d0 = 0.0, d1 = 0.0;
   {
     int row = row0, u = u0;
-    const bool ok = qw_pass(ring, [&](int c, const uint8_t* stage, int units_here) {
+    const bool ok = qw_pass(ring, &s_ok, [&](int c, const uint8_t* stage, int units_here) {
       if (t < units_here) {
-        uint32_t wd[8];
+        uint32_t wd[8], mw[8];
         qw_load_unit(stage, t, wd);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          d0 += __hiloint2double((int)(((wd[i] & 0x7FFFu) << 13) + kF64Rebias), 0);
-          d1 += __hiloint2double((int)(((wd[i] >> 3) & 0x0FFFE000u) + kF64Rebias), 0);
+          mw[i] = wd[i] & 0x7FFF7FFFu;
+          d0 += __hiloint2double((int)(((mw[i] & 0xFFFFu) << 13) + kF64Rebias), 0);
+          d1 += __hiloint2double((int)(((mw[i] >> 16) << 13) + kF64Rebias), 0);
         }
         if (has_meta) {
-          uint32_t h[16];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            h[2 * i] = wd[i] & 0xFFFFu;
-            h[2 * i + 1] = wd[i] >> 16;
-          }
-          const uint32_t keep = unit_keep_bits<M>(h, n);
+          const uint32_t keep = unit_keep_fast<M>(mw, n);
           *reinterpret_cast<uint16_t*>(meta + (size_t)row * meta_stride + 2 * u) = (uint16_t)keep;
           const int li = c * kQwThreads + t;
           if (li < kQwKeepCap) s_keep[li] = (uint16_t)keep;
@@ -374,25 +428,36 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   if (t == 0) {
     double a = 0.0;
     for (int i = 0; i < kQwWarps; ++i) a += swarp_d[i];
-    atomicAdd(gsum, a);
+    gpart[blockIdx.x] = a;
   }
   // the second pass re-reads the same range (now mostly in L2): start it
   // before the grid barrier
   qw_prologue(ring);
   if (!grid_barrier(arrive, gridDim.x, &s_abort)) {
-    qw_pass(ring, [](int, const uint8_t*, int) {});   // drain the prefetched stages
+    qw_pass(ring, &s_ok, [](int, const uint8_t*, int) {});   // drain the prefetched stages
     return;
   }
 
   // ---- gamma: certified from the fp64 total, else exact ---------------------
+  // the CTA partials, summed in the same fixed order by every CTA (one per
+  // thread, warp trees, then the warp sums in order), so all agree on S
+  {
+    double v = (t < (int)gridDim.x) ? __ldcg(gpart + t) : 0.0;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) swarp_d[warp] = v;
+  }
+  __syncthreads();
   if (t == 0) {
-    const double S = __ldcg(gsum);
+    double S = 0.0;
+    for (int i = 0; i < kQwWarps; ++i) S += swarp_d[i];
     const double nk = (double)n_out * (double)k;
     // additions on the longest path: per-thread accumulator (8 per unit, one
-    // unit per chunk), d0 + d1, warp tree, CTA sum, one global atomic per CTA
+    // unit per chunk), d0 + d1, warp tree, warp sums of the CTA, then the
+    // same two levels over the CTA partials (counted generously)
     const long long max_units = (total_units + gridDim.x - 1) / gridDim.x;
     const double per_thread = 8.0 * (double)((max_units + kQwThreads - 1) / kQwThreads);
-    const double adds = per_thread + 1.0 + 5.0 + kQwWarps + (double)gridDim.x;
+    const double adds = per_thread + 1.0 + 2.0 * (5.0 + kQwWarps) + (double)gridDim.x;
     const double err = S * adds * 0x1p-53 * 1.01 + nk * 0x1p-126 * 1.01;
     const double lo = (S - err) / nk * (1.0 - 0x1p-50);
     const double hi = (S + err) / nk * (1.0 + 0x1p-50);
@@ -410,7 +475,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     for (int i = t; i < kQwBins; i += kQwThreads) sbins[i] = 0ull;
     __syncthreads();
     unsigned long long acc = 0ull;
-    const bool ok = qw_pass(ring, [&](int, const uint8_t* stage, int units_here) {
+    const bool ok = qw_pass(ring, &s_ok, [&](int, const uint8_t* stage, int units_here) {
       if (t < units_here) {
         uint32_t wd[8];
         qw_load_unit(stage, t, wd);
@@ -441,7 +506,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
       if (sbins[i]) atomicAdd(&gbins[i], sbins[i]);
     qw_prologue(ring);
     if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort)) {
-      qw_pass(ring, [](int, const uint8_t*, int) {});
+      qw_pass(ring, &s_ok, [](int, const uint8_t*, int) {});
       return;
     }
     if (warp == 0) {
@@ -460,7 +525,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   // ---- phase 2: codes of the kept positions ---------------------------------
   {
     int row = row0, u = u0;
-    qw_pass(ring, [&](int c, const uint8_t* stage, int units_here) {
+    qw_pass(ring, &s_ok, [&](int c, const uint8_t* stage, int units_here) {
       if (t < units_here) {
         uint32_t wd[8];
         qw_load_unit(stage, t, wd);
@@ -471,7 +536,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
                      ? (uint32_t)s_keep[li]
                      : (uint32_t) * reinterpret_cast<const uint16_t*>(meta + (size_t)row * meta_stride + 2 * u);
         }
-        const uint32_t packed = compact_codes16<M>(dense_codes16(wd, tau), keep, n, s_rm);
+        const uint32_t packed = unit_codes(wd, tau | (tau << 16), keep, s_csel);
         uint8_t* dst = codes + (size_t)row * codes_stride + (size_t)u * cb;
         if (cb == 4) {
           *reinterpret_cast<uint32_t*>(dst) = packed;

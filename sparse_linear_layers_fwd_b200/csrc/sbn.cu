@@ -96,7 +96,7 @@ sbn_status launch_qw_fused(const uint16_t* w, int n_out, int k, int n, uint8_t* 
     attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)sms);
+  cfg.gridDim = dim3((unsigned)std::min(sms, kQwMaxGrid));
   cfg.blockDim = dim3(kQwThreads);
   cfg.dynamicSmemBytes = kQwSmemBytes;
   cfg.stream = st;
@@ -118,7 +118,7 @@ sbn_status launch_quantize_weights(const uint16_t* w, int n_out, int k, int n, i
                                    cudaStream_t st) {
   // Each CTA's exact sum counts units of 2^-37 of values below 8 in a u64:
   // at most 2^24 elements per CTA (always true for N_out*K < 2^31 on 128+ SMs).
-  if ((long long)n_out * k > ((long long)sms << 24)) return SBN_ERR_SHAPE;
+  if ((long long)n_out * k > ((long long)std::min(sms, kQwMaxGrid) << 24)) return SBN_ERR_SHAPE;
   if (cudaMemsetAsync(ws, 0, kQwClearBytes, st) != cudaSuccess) {
     cudaGetLastError();
     return SBN_ERR_CUDA;
