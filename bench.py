@@ -74,6 +74,12 @@ def bl_bytes(t, k, n_out, n, m):
     return packed_bytes(n_out, k, n, m) + t * k + 4 * t + 4 + 2 * t * n_out
 
 
+def blx_bytes(t, k, n_out, n, m):
+    """sbn_bitlinear_x (act-quant fused into the contraction): bf16 X + packed W
+    + gamma + bf16 Y (the INT8 activations stay on chip)."""
+    return 2 * t * k + packed_bytes(n_out, k, n, m) + 4 + 2 * t * n_out
+
+
 def bl_ops(t, k, n_out, n, m):
     """Algorithmic ops (2 per kept multiply-add)."""
     return 2 * t * k * n_out * n // m
@@ -82,20 +88,28 @@ def bl_ops(t, k, n_out, n, m):
 WORKLOADS = {
     # name: list of layers (n_out, k, n, m, [token counts]) in one step
     "decode": dict(desc="decode GEMV sweep: K=2560, N_out=6912, 6:8, T in {1,4,16}; value = "
-                        "algorithmic bytes of the step / step time",
-                   unit="GB/s", layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
+                        "algorithmic bytes of the step / step time; activation quantization "
+                        "fused into the contraction (sbn_bitlinear_x)",
+                   unit="GB/s", fused=True, layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
     "prefill": dict(desc="prefill GEMM: T=4096, (K,N_out)=(2560,6912) and (6912,2560), 2:4; value = "
                          "algorithmic ops (2 per kept multiply-add) of the step / step time",
                     unit="TOPS", layers=[(6912, 2560, 2, 4, [4096]), (2560, 6912, 2, 4, [4096])]),
 }
 
 
-def step_bytes(layers):
+def act_bytes(t, k, n_out, n, m, fused):
+    """Bytes of one token set after the weights are packed."""
+    if fused:
+        return blx_bytes(t, k, n_out, n, m)
+    return qa_bytes(t, k) + bl_bytes(t, k, n_out, n, m)
+
+
+def step_bytes(layers, fused=False):
     b = 0
     for (n_out, k, n, m, ts) in layers:
         b += qw_bytes(n_out, k, n, m)
         for t in ts:
-            b += qa_bytes(t, k) + bl_bytes(t, k, n_out, n, m)
+            b += act_bytes(t, k, n_out, n, m, fused)
     return b
 
 
@@ -110,6 +124,11 @@ def step_ops(layers):
 # ---------------------------------------------------------------------------
 # across ranks (one process per GPU, each on its own independent layer)
 # ---------------------------------------------------------------------------
+
+def is_fused(workload: str) -> bool:
+    """Whether the workload's steps use sbn_bitlinear_x (act-quant fused)."""
+    return bool(WORKLOADS[workload].get("fused", False))
+
 
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's time: every rank contributes its own and gets the max."""
@@ -128,7 +147,7 @@ def whole_job_value(workload: str, steps: int, world: int, ms_max: float) -> flo
     layers = WORKLOADS[workload]["layers"]
     if WORKLOADS[workload]["unit"] == "TOPS":
         return step_ops(layers) * steps * world / (ms_max * 1e-3) / 1e12
-    return step_bytes(layers) * steps * world / (ms_max * 1e-3) / 1e9
+    return step_bytes(layers, is_fused(workload)) * steps * world / (ms_max * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -253,13 +272,13 @@ def oracle_step(layers_data, rows):
             oracle.dequant_bf16(acc, s, gamma)
 
 
-def oracle_sample_bytes(layers, rows_frac):
+def oracle_sample_bytes(layers, rows_frac, fused=False):
     tot = 0
     for (n_out, k, n, m, ts) in layers:
         r = max(1, int(n_out * rows_frac))
         tot += qw_bytes(r, k, n, m)
         for t in ts:
-            tot += qa_bytes(t, k) + bl_bytes(t, k, r, n, m)
+            tot += act_bytes(t, k, r, n, m, fused)
     return tot
 
 
@@ -271,7 +290,7 @@ def oracle_sample_metric(workload, layers, rows_frac):
             r = max(1, int(n_out * rows_frac))
             tot += sum(bl_ops(t, k, r, n, m) for t in ts)
         return tot / 1e12
-    return oracle_sample_bytes(layers, rows_frac) / 1e9
+    return oracle_sample_bytes(layers, rows_frac, is_fused(workload)) / 1e9
 
 
 def make_layers_data(workload, rank=0):
@@ -339,18 +358,23 @@ def run_ours(args, rank, world, local_rank):
             # the contraction's workspace (expanded weights, T > 16); written
             # and read within one call, so one per layer serves every slot
             bws = layer_bws.setdefault((n_out, k), torch.empty(
-                (max(1, max(sbn.bitlinear_workspace_bytes(t, k, n_out) for t in ts)),),
+                (max(1, max(max(sbn.bitlinear_workspace_bytes(t, k, n_out),
+                                sbn.bitlinear_x_workspace_bytes(t, k, n_out)) for t in ts)),),
                 dtype=torch.uint8, device=dev))
             sl.append(dict(w=wd, xs=xds, pw=pw, ws=ws, bws=bws, qs=qs, ys=ys, n=n, m=m))
         slots.append(sl)
 
     # per-call events inside each slot's graph: names of the calls in order
+    fused = is_fused(args.workload)
     call_names = []
     for li, (n_out, k, n, m, ts) in enumerate(layers):
         call_names.append(("quantize_weights", li, None))
         for t in ts:
-            call_names.append(("quantize_acts", li, t))
-            call_names.append(("bitlinear", li, t))
+            if fused:
+                call_names.append(("bitlinear_x", li, t))
+            else:
+                call_names.append(("quantize_acts", li, t))
+                call_names.append(("bitlinear", li, t))
 
     def enqueue_step(sl, evs=None):
         i = 0
@@ -360,6 +384,12 @@ def run_ours(args, rank, world, local_rank):
             if evs: evs[i][1].record(stream)
             i += 1
             for x, (q, s), y in zip(L["xs"], L["qs"], L["ys"]):
+                if fused:
+                    if evs: evs[i][0].record(stream)
+                    sbn.bitlinear_x(x, L["pw"], out=y, workspace=L["bws"], stream=stream)
+                    if evs: evs[i][1].record(stream)
+                    i += 1
+                    continue
                 if evs: evs[i][0].record(stream)
                 sbn.quantize_acts(x, out_q=q, out_s=s, stream=stream)
                 if evs: evs[i][1].record(stream)
@@ -383,7 +413,9 @@ def run_ours(args, rank, world, local_rank):
         slot_events.append(evs)
     # our kernels per step: quantize_weights 1 per layer; quantize_acts 1 and
     # bitlinear 1 (+1 weight expansion when T > 16) per token set
-    launches_per_step = sum(1 + sum(2 + (1 if t > 16 else 0) for t in ts)
+    # (fused: one kernel per token set for T <= 16)
+    launches_per_step = sum(1 + sum((1 if fused and t <= 16 else 2 + (1 if t > 16 else 0))
+                                    for t in ts)
                             for (_, _, _, _, ts) in layers)
 
     def barrier():
@@ -422,7 +454,7 @@ def run_ours(args, rank, world, local_rank):
 
     ms = max_over_ranks(ms, world, dev)
 
-    sb = step_bytes(layers)
+    sb = step_bytes(layers, fused)
     ms_per_step = ms / args.steps
     value = whole_job_value(args.workload, args.steps, world, ms)
 
@@ -458,6 +490,8 @@ def run_ours(args, rank, world, local_rank):
             dom_bytes = sum(qw_bytes(n_out, k, n, m) for (n_out, k, n, m, ts) in layers)
         elif dom == "quantize_acts":
             dom_bytes = sum(qa_bytes(t, k) for (n_out, k, n, m, ts) in layers for t in ts)
+        elif dom == "bitlinear_x":
+            dom_bytes = sum(blx_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
         else:
             dom_bytes = sum(bl_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
         achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -477,11 +511,14 @@ def run_ours(args, rank, world, local_rank):
             b = qw_bytes(n_out, k, n, m)
         elif name == "quantize_acts":
             b = qa_bytes(t, k)
+        elif name == "bitlinear_x":
+            b = blx_bytes(t, k, n_out, n, m)
         else:
             b = bl_bytes(t, k, n_out, n, m)
         e = {"us": round(us, 3), "GB/s": round(b / (us * 1e-6) / 1e9, 1),
              "hbm_frac": round(b / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
-        if name == "bitlinear":
+        if name in ("bitlinear", "bitlinear_x"):
+            e["weight_GB/s"] = round(packed_bytes(n_out, k, n, m) / (us * 1e-6) / 1e9, 1)
             ops = bl_ops(t, k, n_out, n, m)
             e["TOPS"] = round(ops / (us * 1e-6) / 1e12, 3)
             e["dense_eq_TOPS"] = round(2 * t * k * n_out / (us * 1e-6) / 1e12, 3)
@@ -542,14 +579,19 @@ def run_e2e(args, data, layers, dev, stream, world):
     ws = [torch.empty(sbn.workspace_bytes(*h[0].shape), dtype=torch.uint8, device=dev) for h in host]
     pws = [sbn.alloc_packed(h[0].shape[0], h[0].shape[1], h[2], h[3], dev) for h in host]
 
+    fused = is_fused(args.workload)
+
     def step():
         for li, (hw, hxs, n, m) in enumerate(host):
             dw[li].copy_(hw, non_blocking=True)
             sbn.quantize_weights(dw[li], n, m, out=pws[li], workspace=ws[li], stream=stream)
             for j, hx in enumerate(hxs):
                 dxs[li][j].copy_(hx, non_blocking=True)
-                q, s = sbn.quantize_acts(dxs[li][j], stream=stream)
-                y = sbn.bitlinear(q, s, pws[li], stream=stream)
+                if fused:
+                    y = sbn.bitlinear_x(dxs[li][j], pws[li], stream=stream)
+                else:
+                    q, s = sbn.quantize_acts(dxs[li][j], stream=stream)
+                    y = sbn.bitlinear(q, s, pws[li], stream=stream)
                 ys_host[li][j].copy_(y, non_blocking=True)
 
     steps = max(3, min(args.steps, args.e2e_steps))
@@ -604,7 +646,8 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, bf16 io",
         "data": "synthetic (seeded: W ~ N(0,0.02) bf16, X ~ N(0,1) bf16)",
         "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]["desc"],
-                   "bytes_per_step": step_bytes(layers), "tokens_per_step": step_tokens(layers)},
+                   "bytes_per_step": step_bytes(layers, is_fused(args.workload)),
+                   "tokens_per_step": step_tokens(layers)},
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores_used(),
                          "kind": "oracle",
                          "sample": f"each step: {frac:.3f} of the output features of every "

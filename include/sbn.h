@@ -199,6 +199,39 @@ sbn_status sbn_bitlinear(const int8_t* xq, const float* x_scale, int32_t t,
 size_t sbn_bitlinear_workspace_bytes(int32_t t, int32_t k, int32_t n_out);
 
 /*
+ * sbn_bitlinear_x -- sbn_quantize_acts and sbn_bitlinear in one call, from
+ * the bf16 activations. For t <= 16 (when the layer's rows and X fit in
+ * shared memory) it is one kernel: every CTA quantizes X per token with the
+ * arithmetic of sbn_quantize_acts and contracts straight away, so the INT8
+ * activations never go through HBM ("The BitLinear Layer" (octagono page),
+ * second to fifth operations, run back to back). Otherwise it runs the two
+ * calls in sequence.
+ *
+ *   x_bf16        device, [t, k] bf16.
+ *   codes, meta,  as for sbn_bitlinear.
+ *   gamma, y_bf16
+ *   xq, x_scale   optional (NULL allowed) device outputs, [t, k] int8 and [t]
+ *                 fp32: the INT8 activations and scales, bit-identical to
+ *                 sbn_quantize_acts.
+ *   workspace,    device scratch owned by the caller, 16-byte aligned, at
+ *   ws_bytes      least sbn_bitlinear_x_workspace_bytes(t, k, n_out) bytes;
+ *                 may be NULL when the one-kernel route applies (t <= 16 on
+ *                 the configurations of this library's workloads), else
+ *                 SBN_ERR_WORKSPACE. Contents unspecified afterwards.
+ * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN,
+ * SBN_ERR_WORKSPACE (before anything is enqueued); SBN_ERR_CUDA.
+ */
+sbn_status sbn_bitlinear_x(const void* x_bf16, int32_t t, int32_t k,
+                           int32_t n_out, int32_t n, int32_t m,
+                           const uint8_t* codes, const uint8_t* meta,
+                           const float* gamma, void* y_bf16, int8_t* xq,
+                           float* x_scale, void* workspace, size_t ws_bytes,
+                           void* stream);
+
+/* Bytes of sbn_bitlinear_x's workspace (enough for its two-step route). */
+size_t sbn_bitlinear_x_workspace_bytes(int32_t t, int32_t k, int32_t n_out);
+
+/*
  * sbn_bitlinear_acc32 -- the same contraction, writing the exact int32
  * accumulators acc [t, n_out] (device, row-major) instead of y. Meant for
  * verification; same arguments (workspace included) and errors as
@@ -209,6 +242,24 @@ sbn_status sbn_bitlinear_acc32(const int8_t* xq, int32_t t, int32_t k,
                                const uint8_t* codes, const uint8_t* meta,
                                int32_t* acc, void* workspace, size_t ws_bytes,
                                void* stream);
+
+/*
+ * sbn_mask_flips -- number of positions whose keep bit differs between two
+ * keep masks of the same layer (two versions of sbn_quantize_weights' meta
+ * for the same n_out, k, n, m), e.g. consecutive training steps.
+ *
+ * Defining passage: Sparse-BitNet page, Figure 3(b), the mask flip rate r_t
+ * (its equation is missing from the page; read as the fraction of mask
+ * positions that changed): r_t = flips / (n_out * k).
+ *
+ *   meta_a, meta_b  device, [n_out, sbn_meta_row_bytes] each, 16-byte aligned.
+ *   flips           device, one uint64, 8-byte aligned, written (exact count).
+ * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN (also for n == m:
+ * a dense layer has no mask), SBN_ERR_ALIGN; SBN_ERR_CUDA.
+ */
+sbn_status sbn_mask_flips(const uint8_t* meta_a, const uint8_t* meta_b,
+                          int32_t n_out, int32_t k, int32_t n, int32_t m,
+                          unsigned long long* flips, void* stream);
 
 /*
  * sbn_get_device_error -- synchronizes `stream`, then reads and clears the

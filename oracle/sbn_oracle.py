@@ -77,6 +77,8 @@ __all__ = [
     "bitlinear",
     "bitlinear_acc_at",
     "bitlinear_at",
+    "mask_flips",
+    "mask_flip_rate",
 ]
 
 #: floor on gamma and on the per-token activation scale (not on the pages)
@@ -374,3 +376,27 @@ def bitlinear_at(xq, s, dense_codes, gamma, t_idx, n_idx):
     acc = bitlinear_acc_at(xq, dense_codes, t_idx, n_idx)
     y = acc.astype(np.float64) * float(gamma) * (s.astype(np.float64)[np.asarray(t_idx)] / Q_ACT)
     return bf16_bits_from_f64_rne(y), acc
+
+
+# --------------------------------------------------------------------------
+# mask flip rate between two steps
+# --------------------------------------------------------------------------
+
+def mask_flips(mask_a: np.ndarray, mask_b: np.ndarray) -> int:
+    """Number of positions whose keep/prune state differs between two masks.
+
+    Sparse-BitNet page, Figure 3(b): the mask flip rate r_t measures how
+    stable the dynamic N:M pattern is between training steps; its equation is
+    not in the extracted page, so it is read as the fraction of positions
+    whose mask entry changed.
+    """
+    mask_a = np.asarray(mask_a, dtype=bool)
+    mask_b = np.asarray(mask_b, dtype=bool)
+    if mask_a.shape != mask_b.shape:
+        raise ValueError("masks of different shapes")
+    return int(np.count_nonzero(mask_a != mask_b))
+
+
+def mask_flip_rate(mask_a: np.ndarray, mask_b: np.ndarray) -> float:
+    """r_t = mask_flips / number of positions."""
+    return mask_flips(mask_a, mask_b) / float(np.asarray(mask_a).size)

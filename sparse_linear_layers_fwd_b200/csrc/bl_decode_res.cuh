@@ -18,12 +18,19 @@
 // columns, a K permutation shared with the activation fragment). A warp adds
 // its partial sums into the tile's shared accumulator when it moves to
 // another tile; the epilogue dequantizes y = acc * gamma * s_t / 127.
+//
+// XBF: the kernel takes the bf16 activations instead and quantizes them
+// itself (the per-token absmax INT8 step fused into the contraction's
+// prologue): every CTA copies X, one warp per token computes s_t and the
+// INT8 row in shared memory with the arithmetic of sbn_quantize_acts
+// (qa.cuh), and CTA 0 optionally writes Xq and s to global memory.
 #pragma once
 
 #include "async.cuh"
 #include "bl_decode.cuh"
 #include "common.cuh"
 #include "expand.cuh"
+#include "qa.cuh"
 
 namespace sbn {
 
@@ -33,13 +40,13 @@ constexpr int kDresMaxTiles = 16;        // tiles per CTA at most
 constexpr size_t kDresSmemMax = 227 * 1024;
 
 struct DresLayout {
-  size_t sel, acc, x, codes, meta, bars, total;
+  size_t sel, acc, x, codes, meta, xbf, scale, bars, total;
   int xstride;
 };
 
 // Shared-memory layout of one CTA holding `tiles` tiles.
 __host__ __device__ inline DresLayout dres_layout(int tiles, int nt, int k, int cstride, int mstride,
-                                                  bool dense) {
+                                                  bool dense, bool xbf = false) {
   DresLayout L;
   L.xstride = k;
   L.sel = 0;
@@ -49,7 +56,10 @@ __host__ __device__ inline DresLayout dres_layout(int tiles, int nt, int k, int 
   L.codes = L.x + (size_t)nt * L.xstride;
   L.codes = (L.codes + 127) & ~(size_t)127;
   L.meta = L.codes + (size_t)tiles * 16 * cstride;
-  L.bars = L.meta + (dense ? 0 : (size_t)tiles * 16 * mstride);
+  L.xbf = L.meta + (dense ? 0 : (size_t)tiles * 16 * mstride);
+  L.xbf = (L.xbf + 127) & ~(size_t)127;
+  L.scale = L.xbf + (xbf ? (size_t)nt * k * 2 : 0);
+  L.bars = L.scale + (xbf ? 16 * 4 : 0);
   L.bars = (L.bars + 15) & ~(size_t)15;
   L.total = L.bars + (size_t)(tiles + 1) * 8;
   return L;
@@ -58,6 +68,9 @@ __host__ __device__ inline DresLayout dres_layout(int tiles, int nt, int k, int 
 struct DresParams {
   const int8_t* xq;
   const float* xs;
+  const uint16_t* xbf;   // XBF: bf16 activations [T, K]
+  int8_t* xq_out;        // XBF: optional copies of Xq and s (written by CTA 0)
+  float* xs_out;
   const uint8_t* codes;
   const uint8_t* meta;
   const float* gamma;
@@ -70,7 +83,7 @@ struct DresParams {
 
 // MM: group size m; CB: code bytes per 16 positions (= 4n/m); NT: token
 // columns (8 or 16); DENSE: n == m (no keep bits); ACC: write int32 acc.
-template <int MM, int CB, int NT, bool DENSE, bool ACC>
+template <int MM, int CB, int NT, bool DENSE, bool ACC, bool XBF>
 __global__ void __launch_bounds__(kDresThreads, 1)
 bl_decode_res_kernel(const DresParams p) {
   extern __shared__ __align__(128) uint8_t dres_smem[];
@@ -78,12 +91,14 @@ bl_decode_res_kernel(const DresParams p) {
   const int t_begin = (int)((long long)blockIdx.x * n_tiles / gridDim.x);
   const int t_end = (int)((long long)(blockIdx.x + 1) * n_tiles / gridDim.x);
   const int tiles = t_end - t_begin;
-  const DresLayout L = dres_layout(p.tiles_per_cta, NT, p.K, p.cstride, p.mstride, DENSE);
+  const DresLayout L = dres_layout(p.tiles_per_cta, NT, p.K, p.cstride, p.mstride, DENSE, XBF);
   uint32_t* s_sel = reinterpret_cast<uint32_t*>(dres_smem + L.sel);
   int32_t* s_acc = reinterpret_cast<int32_t*>(dres_smem + L.acc);
   uint8_t* s_x = dres_smem + L.x;
   uint8_t* s_codes = dres_smem + L.codes;
   uint8_t* s_meta = dres_smem + L.meta;
+  uint16_t* s_xbf = reinterpret_cast<uint16_t*>(dres_smem + L.xbf);
+  float* s_scale = reinterpret_cast<float*>(dres_smem + L.scale);
   uint64_t* bar_x = reinterpret_cast<uint64_t*>(dres_smem + L.bars);
   uint64_t* bar_t = bar_x + 1;
 
@@ -100,8 +115,13 @@ bl_decode_res_kernel(const DresParams p) {
     mbar_init(bar_x, 1);
     for (int i = 0; i < ngrp; ++i) mbar_init(&bar_t[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    mbar_arrive_expect_tx(bar_x, (uint32_t)(p.T * p.K));
-    bulk_g2s(s_x, p.xq, (uint32_t)(p.T * p.K), bar_x);
+    if (XBF) {
+      mbar_arrive_expect_tx(bar_x, (uint32_t)(p.T * p.K * 2));
+      bulk_g2s(s_xbf, p.xbf, (uint32_t)(p.T * p.K * 2), bar_x);
+    } else {
+      mbar_arrive_expect_tx(bar_x, (uint32_t)(p.T * p.K));
+      bulk_g2s(s_x, p.xq, (uint32_t)(p.T * p.K), bar_x);
+    }
     for (int gi = 0; gi < ngrp; ++gi) {
       const int ta = gi ? split : 0, tb = gi ? tiles : split;
       const int r = row0 + 16 * ta;
@@ -125,6 +145,31 @@ bl_decode_res_kernel(const DresParams p) {
     return __shfl_sync(0xffffffffu, got, 0) != 0;
   };
   bool ok = warp_wait(bar_x);
+  if (XBF) {
+    // warp `warp` quantizes token row `warp` (T <= 16 <= warps)
+    if (ok && warp < p.T) {
+      const uint4* xr = reinterpret_cast<const uint4*>(s_xbf + (size_t)warp * p.K);
+      const int kc = p.K / 8;
+      uint32_t amax = 0u;
+      for (int c = lane; c < kc; c += 32) amax = max(amax, mag_max8(xr[c]));
+      amax = __reduce_max_sync(0xffffffffu, amax);
+      const float sc = fmaxf(__uint_as_float(amax << 16), 1e-5f);
+      const float mult = __fdiv_rn(127.0f, sc);
+      uint2* qr = reinterpret_cast<uint2*>(s_x + (size_t)warp * L.xstride);
+      const bool out = blockIdx.x == 0 && p.xq_out != nullptr;
+      uint2* gq = out ? reinterpret_cast<uint2*>(p.xq_out + (size_t)warp * p.K) : nullptr;
+      for (int c = lane; c < kc; c += 32) {
+        const uint2 q = quant8(xr[c], mult);
+        qr[c] = q;
+        if (out) gq[c] = q;
+      }
+      if (lane == 0) {
+        s_scale[warp] = sc;
+        if (blockIdx.x == 0 && p.xs_out) p.xs_out[warp] = sc;
+      }
+    }
+    ok = __syncthreads_and(ok) != 0;
+  }
   const int ksegs = p.K / 128;
   const int items = tiles * ksegs;
   int cur_tile = -1;
@@ -212,7 +257,8 @@ bl_decode_res_kernel(const DresParams p) {
     if (ACC) {
       p.acc_out[(size_t)tok * p.N + grow] = a;
     } else {
-      const float sc = __fdiv_rn(__fmul_rn(gm, __ldg(p.xs + tok)), 127.0f);
+      const float st = XBF ? s_scale[tok] : __ldg(p.xs + tok);
+      const float sc = __fdiv_rn(__fmul_rn(gm, st), 127.0f);
       p.y[(size_t)tok * p.N + grow] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a, sc)));
     }
   }

@@ -19,6 +19,7 @@
 #include "bl_decode.cuh"
 #include "bl_decode_res.cuh"
 #include "expand_dense.cuh"
+#include "flip.cuh"
 #include "bl_tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -172,7 +173,7 @@ sbn_status dispatch_decode(const DecodeParams& p, int n, int m, int sms, cudaStr
 
 // Resident decode kernel: grid = min(SMs, tiles), one CTA per SM holding the
 // packed rows of its tiles and all of Xq in shared memory.
-template <int MM, int CB, int NT, bool DENSE, bool ACC>
+template <int MM, int CB, int NT, bool DENSE, bool ACC, bool XBF>
 sbn_status launch_decode_res(const DresParams& p, int grid, size_t smem, cudaStream_t st) {
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
@@ -180,7 +181,7 @@ sbn_status launch_decode_res(const DresParams& p, int grid, size_t smem, cudaStr
     cudaGetLastError();
     return SBN_ERR_CUDA;
   }
-  auto kern = bl_decode_res_kernel<MM, CB, NT, DENSE, ACC>;
+  auto kern = bl_decode_res_kernel<MM, CB, NT, DENSE, ACC, XBF>;
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDresSmemMax) !=
         cudaSuccess) {
@@ -193,21 +194,21 @@ sbn_status launch_decode_res(const DresParams& p, int grid, size_t smem, cudaStr
   return launch_status();
 }
 
-template <int NT, bool ACC>
+template <int NT, bool ACC, bool XBF>
 sbn_status dispatch_decode_res(const DresParams& p, int n, int m, int grid, size_t smem,
                                cudaStream_t st) {
   const int cb = 4 * n / m;
-  if (n == m) return launch_decode_res<8, 4, NT, true, ACC>(p, grid, smem, st);
+  if (n == m) return launch_decode_res<8, 4, NT, true, ACC, XBF>(p, grid, smem, st);
   switch (m * 8 + cb) {
-    case 4 * 8 + 1: return launch_decode_res<4, 1, NT, false, ACC>(p, grid, smem, st);
-    case 4 * 8 + 2: return launch_decode_res<4, 2, NT, false, ACC>(p, grid, smem, st);
-    case 4 * 8 + 3: return launch_decode_res<4, 3, NT, false, ACC>(p, grid, smem, st);
-    case 8 * 8 + 1: return launch_decode_res<8, 1, NT, false, ACC>(p, grid, smem, st);
-    case 8 * 8 + 2: return launch_decode_res<8, 2, NT, false, ACC>(p, grid, smem, st);
-    case 8 * 8 + 3: return launch_decode_res<8, 3, NT, false, ACC>(p, grid, smem, st);
-    case 16 * 8 + 1: return launch_decode_res<16, 1, NT, false, ACC>(p, grid, smem, st);
-    case 16 * 8 + 2: return launch_decode_res<16, 2, NT, false, ACC>(p, grid, smem, st);
-    case 16 * 8 + 3: return launch_decode_res<16, 3, NT, false, ACC>(p, grid, smem, st);
+    case 4 * 8 + 1: return launch_decode_res<4, 1, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 4 * 8 + 2: return launch_decode_res<4, 2, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 4 * 8 + 3: return launch_decode_res<4, 3, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 1: return launch_decode_res<8, 1, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 2: return launch_decode_res<8, 2, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 3: return launch_decode_res<8, 3, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 16 * 8 + 1: return launch_decode_res<16, 1, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 16 * 8 + 2: return launch_decode_res<16, 2, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 16 * 8 + 3: return launch_decode_res<16, 3, NT, false, ACC, XBF>(p, grid, smem, st);
   }
   return SBN_ERR_PATTERN;
 }
@@ -354,8 +355,9 @@ sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k
       DresParams q;
       q.xq = xq; q.xs = xs; q.codes = codes; q.meta = meta; q.gamma = gamma; q.y = y; q.acc_out = acc;
       q.T = t; q.K = k; q.N = n_out; q.cstride = cstride; q.mstride = mstride; q.tiles_per_cta = per_cta;
-      return t <= 8 ? dispatch_decode_res<8, ACC_OUT>(q, n, m, grid, L.total, st)
-                    : dispatch_decode_res<16, ACC_OUT>(q, n, m, grid, L.total, st);
+      q.xbf = nullptr; q.xq_out = nullptr; q.xs_out = nullptr;
+      return t <= 8 ? dispatch_decode_res<8, ACC_OUT, false>(q, n, m, grid, L.total, st)
+                    : dispatch_decode_res<16, ACC_OUT, false>(q, n, m, grid, L.total, st);
     }
     DecodeParams p;
     p.xq = xq; p.xs = xs; p.codes = codes; p.meta = meta; p.gamma = gamma; p.y = y; p.acc_out = acc;
@@ -404,6 +406,44 @@ sbn_status validate_bitlinear(const int8_t* xq, int32_t t, int32_t k, int32_t n_
   if (!prod_lt_2_31(t, k) || !prod_lt_2_31(n_out, k) || !prod_lt_2_31(t, n_out)) return SBN_ERR_SHAPE;
   if (!aligned16(xq) || !aligned16(codes) || (meta && !aligned16(meta))) return SBN_ERR_ALIGN;
   return SBN_OK;
+}
+
+// Fused decode (activation quantization inside the contraction): used when
+// t <= 16 and the layout with the bf16 activations fits in shared memory.
+bool fused_decode_fits(int32_t t, int32_t k, int32_t n_out, int32_t n, int32_t m, int sms, int* grid,
+                       int* per_cta, size_t* smem) {
+  if (t > 16) return false;
+  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
+  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
+  const int tiles = (n_out + 15) / 16;
+  *grid = std::min(sms, tiles);
+  *per_cta = (tiles + *grid - 1) / *grid;
+  const DresLayout L = dres_layout(*per_cta, t <= 8 ? 8 : 16, k, cstride, mstride, n == m, true);
+  *smem = L.total;
+  return *per_cta <= kDresMaxTiles && L.total <= kDresSmemMax;
+}
+
+// Workspace of sbn_bitlinear_x when it runs as two steps: Xq and s, then
+// the contraction's own workspace (the same size whatever the device).
+size_t bitlinear_x_ws_bytes(int32_t t, int32_t k, int32_t n_out) {
+  return round_up16((size_t)t * k) + round_up16((size_t)t * 4) + bitlinear_ws_bytes(t, k, n_out);
+}
+
+// One CTA per token row (qa.cuh); rows up to 16 * 128 * 8 positions stay in registers.
+sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, float* x_scale,
+                                cudaStream_t s) {
+  const int kc = k / 8;
+  const uint4* x = reinterpret_cast<const uint4*>(x_bf16);
+  uint2* q = reinterpret_cast<uint2*>(xq);
+  const int need = (kc + kQaThreads - 1) / kQaThreads;
+  if (need <= 1) qa_kernel<1><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  else if (need <= 2) qa_kernel<2><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  else if (need <= 4) qa_kernel<4><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  else if (need <= 8) qa_kernel<8><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  else if (need <= 12) qa_kernel<12><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  else if (need <= 16) qa_kernel<16><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  else qa_kernel_long<<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  return launch_status();
 }
 
 // Fixed scratch of sbn_quantize_weights_noalloc (see include/sbn.h).
@@ -492,19 +532,79 @@ sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k, int8_t* x
   int dev = 0, sms = 0;
   sbn_status st = check_device(&dev, &sms);
   if (st != SBN_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int kc = k / 8;
-  const uint4* x = reinterpret_cast<const uint4*>(x_bf16);
-  uint2* q = reinterpret_cast<uint2*>(xq);
-  const int need = (kc + kQaThreads - 1) / kQaThreads;
-  if (need <= 1) qa_kernel<1><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 2) qa_kernel<2><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 4) qa_kernel<4><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 8) qa_kernel<8><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 12) qa_kernel<12><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 16) qa_kernel<16><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else qa_kernel_long<<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  return launch_quantize_acts(x_bf16, t, k, xq, x_scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_mask_flips(const uint8_t* meta_a, const uint8_t* meta_b, int32_t n_out, int32_t k,
+                          int32_t n, int32_t m, unsigned long long* flips, void* stream) {
+  if (!meta_a || !meta_b || !flips) return SBN_ERR_NULL;
+  if (!pattern_ok(n, m) || n == m) return SBN_ERR_PATTERN;
+  if (n_out < 1 || k < 128 || (k % 128) != 0 || !prod_lt_2_31(n_out, k)) return SBN_ERR_SHAPE;
+  if (!aligned16(meta_a) || !aligned16(meta_b) || (reinterpret_cast<uintptr_t>(flips) & 7u))
+    return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(flips, 0, sizeof(unsigned long long), cs) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  // rows are padded with zero bytes in both masks, so the padding never counts
+  const long long n16 = (long long)n_out * (long long)sbn_meta_row_bytes(k, n, m) / 16;
+  const long long want = (n16 + kFlipThreads - 1) / kFlipThreads;
+  const int grid = (int)std::max(1LL, std::min(want, (long long)sms * 8));
+  flip_count_kernel<<<grid, kFlipThreads, 0, cs>>>(reinterpret_cast<const uint4*>(meta_a),
+                                                   reinterpret_cast<const uint4*>(meta_b), n16, flips);
   return launch_status();
+}
+
+size_t sbn_bitlinear_x_workspace_bytes(int32_t t, int32_t k, int32_t n_out) {
+  if (t < 1 || k < 1 || n_out < 1) return 0;
+  return bitlinear_x_ws_bytes(t, k, n_out);
+}
+
+sbn_status sbn_bitlinear_x(const void* x_bf16, int32_t t, int32_t k, int32_t n_out, int32_t n,
+                           int32_t m, const uint8_t* codes, const uint8_t* meta, const float* gamma,
+                           void* y_bf16, int8_t* xq, float* x_scale, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  if (!x_bf16 || !gamma || !y_bf16 || !codes || (n != m && !meta)) return SBN_ERR_NULL;
+  if (!pattern_ok(n, m)) return SBN_ERR_PATTERN;
+  if (t < 1 || n_out < 1 || k < 128 || (k % 128) != 0) return SBN_ERR_SHAPE;
+  if (!prod_lt_2_31(t, k) || !prod_lt_2_31(n_out, k) || !prod_lt_2_31(t, n_out)) return SBN_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(codes) || (meta && !aligned16(meta)) || !aligned16(y_bf16) ||
+      (xq && !aligned16(xq)) || (reinterpret_cast<uintptr_t>(x_scale) & 3u) ||
+      (workspace && !aligned16(workspace)))
+    return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int grid = 0, per_cta = 0;
+  size_t smem = 0;
+  if (fused_decode_fits(t, k, n_out, n, m, sms, &grid, &per_cta, &smem)) {
+    DresParams q;
+    q.xq = nullptr; q.xs = nullptr; q.xbf = reinterpret_cast<const uint16_t*>(x_bf16);
+    q.xq_out = xq; q.xs_out = x_scale;
+    q.codes = codes; q.meta = meta; q.gamma = gamma; q.y = reinterpret_cast<uint16_t*>(y_bf16);
+    q.acc_out = nullptr;
+    q.T = t; q.K = k; q.N = n_out;
+    q.cstride = (int)sbn_codes_row_bytes(k, n, m); q.mstride = (int)sbn_meta_row_bytes(k, n, m);
+    q.tiles_per_cta = per_cta;
+    return t <= 8 ? dispatch_decode_res<8, false, true>(q, n, m, grid, smem, cs)
+                  : dispatch_decode_res<16, false, true>(q, n, m, grid, smem, cs);
+  }
+  // two steps: quantize_acts into the given buffers or the workspace, then
+  // the contraction (which expands the weights into the rest of it)
+  if (!workspace || ws_bytes < bitlinear_x_ws_bytes(t, k, n_out)) return SBN_ERR_WORKSPACE;
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(workspace);
+  int8_t* q8 = xq ? xq : reinterpret_cast<int8_t*>(w8);
+  float* sc = x_scale ? x_scale : reinterpret_cast<float*>(w8 + round_up16((size_t)t * k));
+  void* rest = w8 + round_up16((size_t)t * k) + round_up16((size_t)t * 4);
+  if ((st = launch_quantize_acts(x_bf16, t, k, q8, sc, cs)) != SBN_OK) return st;
+  return run_bitlinear<false>(q8, sc, t, k, n_out, n, m, codes, meta, gamma,
+                              reinterpret_cast<uint16_t*>(y_bf16), nullptr,
+                              bitlinear_ws_bytes(t, k, n_out) ? rest : nullptr, sms, cs);
 }
 
 size_t sbn_bitlinear_workspace_bytes(int32_t t, int32_t k, int32_t n_out) {

@@ -48,6 +48,10 @@ PROTOTYPES = {
     "sbn_bitlinear_workspace_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32]),
     "sbn_bitlinear_acc32": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
                                            _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "sbn_bitlinear_x": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p,
+                                       _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "sbn_bitlinear_x_workspace_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32]),
+    "sbn_mask_flips": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
 
@@ -233,6 +237,45 @@ def bitlinear_acc32(xq: torch.Tensor, w: PackedWeights, out: Optional[torch.Tens
     return out
 
 
+def bitlinear_x_workspace_bytes(t: int, k: int, n_out: int) -> int:
+    return int(lib().sbn_bitlinear_x_workspace_bytes(t, k, n_out))
+
+
+def bitlinear_x(x: torch.Tensor, w: PackedWeights, out: Optional[torch.Tensor] = None,
+                out_q: Optional[torch.Tensor] = None, out_s: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """sbn_bitlinear_x: y = bitlinear(quantize_acts(x)) in one call (one kernel
+    for T <= 16). out_q / out_s, if given, receive Xq and s."""
+    _need(x, torch.bfloat16, "x")
+    t, k = x.shape
+    if k != w.k:
+        raise ValueError("K mismatch between activations and weights")
+    if out is None:
+        out = torch.empty((t, w.n_out), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((bitlinear_x_workspace_bytes(t, k, w.n_out),), dtype=torch.uint8,
+                                device=x.device)
+    st = lib().sbn_bitlinear_x(_ptr(x), t, k, w.n_out, w.n, w.m, _ptr(w.codes), _ptr(w.meta),
+                               _ptr(w.gamma), _ptr(out), _ptr(out_q), _ptr(out_s), _ptr(workspace),
+                               workspace.numel(), _stream_ptr(stream))
+    _check(st, "sbn_bitlinear_x")
+    return out
+
+
+def mask_flips(a: PackedWeights, b: PackedWeights, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """sbn_mask_flips: positions whose keep bit differs between two packed
+    versions of one layer (device int64 scalar); flip rate = count / (N_out*K)."""
+    if (a.n_out, a.k, a.n, a.m) != (b.n_out, b.k, b.n, b.m):
+        raise ValueError("the two packed weights describe different layers")
+    if out is None:
+        out = torch.empty((1,), dtype=torch.int64, device=a.codes.device)
+    st = lib().sbn_mask_flips(_ptr(a.meta), _ptr(b.meta), a.n_out, a.k, a.n, a.m, _ptr(out),
+                              _stream_ptr(stream))
+    _check(st, "sbn_mask_flips")
+    return out
+
+
 def get_device_error(stream=None) -> int:
     """sbn_get_device_error: sync the stream, read and clear the device error word."""
     return int(lib().sbn_get_device_error(_stream_ptr(stream)))
@@ -269,6 +312,5 @@ class BitLinear(torch.nn.Module):
         lead = x.shape[:-1]
         x2 = x.reshape(-1, x.shape[-1]).contiguous()
         packed = self.pack()
-        xq, s = quantize_acts(x2)
-        y = bitlinear(xq, s, packed)
+        y = bitlinear_x(x2, packed)   # activation quantization fused for T <= 16
         return y.reshape(*lead, packed.n_out)

@@ -118,6 +118,39 @@ def test_bitlinear_validation(sbn_lib):
     assert lib.sbn_bitlinear_acc32(A, 64, 256, 64, 2, 4, A, A, A, A, need - 1, None) == 5
 
 
+def test_bitlinear_x_validation(sbn_lib):
+    lib = sbn_lib
+    ok = dict(x=A, t=4, k=256, n_out=64, n=2, m=4, codes=A, meta=A, g=A, y=A, q=None, s=None,
+              ws=None, wsb=0)
+
+    def blx(**kw):
+        a = dict(ok, **kw)
+        return lib.sbn_bitlinear_x(a["x"], a["t"], a["k"], a["n_out"], a["n"], a["m"], a["codes"],
+                                   a["meta"], a["g"], a["y"], a["q"], a["s"], a["ws"], a["wsb"], None)
+    assert blx(x=None) == 1
+    assert blx(y=None) == 1
+    assert blx(meta=None) == 1
+    assert blx(n=5, m=8) == 3
+    assert blx(t=0) == 2
+    assert blx(k=100) == 2
+    assert blx(x=MIS) == 4
+    assert blx(q=MIS) == 4
+    assert blx(ws=MIS, wsb=1 << 20) == 4
+    need = lib.sbn_bitlinear_x_workspace_bytes(64, 256, 64)
+    assert need == 64 * 256 + 64 * 4 + 64 * 256          # Xq, s, expanded weights
+    assert lib.sbn_bitlinear_x_workspace_bytes(4, 256, 64) == 4 * 256 + 16
+
+
+def test_mask_flips_validation(sbn_lib):
+    lib = sbn_lib
+    assert lib.sbn_mask_flips(None, A, 8, 256, 2, 4, A, None) == 1
+    assert lib.sbn_mask_flips(A, A, 8, 256, 2, 4, None, None) == 1
+    assert lib.sbn_mask_flips(A, A, 8, 256, 4, 4, A, None) == 3     # dense: no mask
+    assert lib.sbn_mask_flips(A, A, 8, 100, 2, 4, A, None) == 2
+    assert lib.sbn_mask_flips(MIS, A, 8, 256, 2, 4, A, None) == 4
+    assert lib.sbn_mask_flips(A, A, 8, 256, 2, 4, A + 4, None) == 4
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")
 def test_valid_arguments_without_gpu_fail_cleanly(sbn_lib):
     # every argument is valid, so the call reaches the device check and stops there

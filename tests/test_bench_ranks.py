@@ -63,7 +63,7 @@ def test_max_over_ranks_and_whole_job_value_gloo():
     for rank, ms, value, _ in out:
         assert ms == 15.0                                   # max over ranks on every rank
         layers = b.WORKLOADS["decode"]["layers"]
-        expect = b.step_bytes(layers) * 100 * world / (15.0e-3) / 1e9
+        expect = b.step_bytes(layers, b.is_fused("decode")) * 100 * world / (15.0e-3) / 1e9
         assert value == pytest.approx(expect, rel=1e-12)    # all ranks' bytes / slowest time
     # independent inputs per rank
     assert not np.array_equal(out[0][3], out[1][3])

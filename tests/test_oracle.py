@@ -125,3 +125,36 @@ def test_layer_small_zero_fraction_reported():
     g = oracle.absmean_gamma(w)
     c = oracle.ternary_codes(w, g, np.ones(w.shape, bool))
     assert 0.29 < float(np.mean(c == 0)) < 0.33
+
+
+# ---- mask flip rate --------------------------------------------------------
+
+def test_mask_flips_brute_force_and_invariants():
+    rng = np.random.default_rng(31)
+    for (n, m) in [(2, 4), (6, 8), (8, 16), (1, 4)]:
+        w1 = rng.integers(0, 0x4000, size=(7, 64)).astype(np.uint16)
+        w2 = w1.copy()
+        sel = rng.random(w2.shape) < 0.2
+        w2[sel] = rng.integers(0, 0x4000, size=int(sel.sum())).astype(np.uint16)
+        a, b = oracle.nm_mask(w1, n, m), oracle.nm_mask(w2, n, m)
+        # brute force: a plain loop over positions
+        brute = 0
+        for i in range(a.shape[0]):
+            for j in range(a.shape[1]):
+                brute += 1 if bool(a[i, j]) != bool(b[i, j]) else 0
+        assert oracle.mask_flips(a, b) == brute
+        # every group keeps exactly n in both masks: flips come in pairs per group
+        per_group = (a != b).reshape(a.shape[0], -1, m).sum(axis=2)
+        assert np.all(per_group % 2 == 0)
+        assert np.all(per_group <= 2 * min(n, m - n))
+        assert oracle.mask_flips(a, a) == 0
+        assert oracle.mask_flip_rate(a, b) == brute / a.size
+
+
+def test_mask_flips_complement_within_2of4_groups():
+    # keep {0,1} vs keep {2,3} in every group of four: every position flips
+    w1 = np.tile(np.array([0x3F80, 0x3F80, 0x3C00, 0x3C00], np.uint16), (3, 32))
+    w2 = np.tile(np.array([0x3C00, 0x3C00, 0x3F80, 0x3F80], np.uint16), (3, 32))
+    a, b = oracle.nm_mask(w1, 2, 4), oracle.nm_mask(w2, 2, 4)
+    assert oracle.mask_flips(a, b) == a.size
+    assert oracle.mask_flip_rate(a, b) == 1.0

@@ -58,6 +58,54 @@ def test_prefill_sampled_without_workspace(which):
     _sampled_check(g, q, s, dense, gamma, d["x"].shape[0], d["w"].shape[0], seed=21)
 
 
+def _fused_check(w, x, n, m):
+    """sbn_bitlinear_x against the oracle: Xq and s bit-exact, y within tolerance."""
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    pw = run_quantize_weights(w, n, m)
+    xd = to_dev_bf16(x)
+    t, k = x.shape
+    oq = torch.empty((t, k), dtype=torch.int8, device="cuda")
+    os_ = torch.empty((t,), dtype=torch.float32, device="cuda")
+    y = sbn.bitlinear_x(xd, pw, out_q=oq, out_s=os_)
+    torch.cuda.synchronize()
+    assert sbn.get_device_error() == 0
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, n, m)
+    q, s = oracle.quantize_acts(x)
+    assert np.array_equal(oq.cpu().numpy(), q) and np.array_equal(os_.cpu().numpy(), s)
+    acc = oracle.bitlinear_acc(q, dense)
+    assert_y_close(bf16_tensor_bits(y), oracle.dequant_bf16(acc, s, gamma))
+    # without the optional outputs
+    y2 = sbn.bitlinear_x(xd, pw)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_tensor_bits(y2), bf16_tensor_bits(y))
+
+
+@pytest.mark.parametrize("nm", SUPPORTED)
+@pytest.mark.parametrize("shape", SHAPES)
+def test_fused_act_quant_contraction(nm, shape):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=14, tag=f"fx{nm}{shape}")
+    x = synth.activations(t, k, seed=14, tag=f"fx{nm}{shape}", outlier_channels=2)
+    _fused_check(w, x, *nm)
+
+
+@pytest.mark.parametrize("t", synth.DECODE_TOKENS)
+def test_fused_decode_full(t):
+    _fused_check(synth.decode_weights(), synth.decode_acts(t), 6, 8)
+
+
+def test_fused_zero_rows_and_streaming_fallback():
+    w = synth.latent_weights(40, 11008, seed=15)
+    x = synth.activations(16, 11008, seed=15)       # X does not fit: two-step route
+    x[3] = 0
+    _fused_check(w, x, 6, 8)
+    x2 = synth.activations(5, 512, seed=16)
+    x2[0] = 0
+    x2[1] = 0x8000
+    _fused_check(synth.latent_weights(64, 512, seed=16), x2, 2, 4)
+
+
 @pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (8, 8)])
 def test_all_zero_weights(nm):
     w = np.zeros((40, 256), np.uint16)
@@ -271,3 +319,21 @@ def test_gamma_midpoint_plus_tiny_follows_fp64_rounding():
     cb, mb, gamma, _, _ = oracle.quantize_weights(w, 6, 8)
     assert gamma == np.float32(1.0)
     assert_weights_exact(g, cb, mb, gamma)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (1, 4), (12, 16)])
+@pytest.mark.parametrize("shape", [(7, 128), (130, 1024), (6912, 2560)])
+def test_mask_flips(nm, shape):
+    """Keep-bit flips between two versions of a layer (a perturbed copy)."""
+    n_out, k = shape
+    w1 = synth.latent_weights(n_out, k, seed=17, tag=f"flip{shape}")
+    rng = np.random.default_rng(17)
+    w2 = w1.copy()
+    sel = rng.random(w1.shape) < 0.05
+    w2[sel] = synth.latent_weights(n_out, k, seed=18, tag=f"flip{shape}")[sel]
+    from sparse_linear_layers_fwd_b200 import sbn
+    p1 = run_quantize_weights(w1, *nm)
+    p2 = run_quantize_weights(w2, *nm)
+    got = int(sbn.mask_flips(p1, p2).cpu().item())
+    assert got == oracle.mask_flips(oracle.nm_mask(w1, *nm), oracle.nm_mask(w2, *nm))
+    assert int(sbn.mask_flips(p1, p1).cpu().item()) == 0
