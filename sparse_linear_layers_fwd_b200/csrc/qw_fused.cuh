@@ -51,13 +51,16 @@ SBN_DEVFN uint32_t ld_acquire_u32(const uint32_t* p) {
 // normal magnitudes, near 2^-127 for zero and subnormals.
 constexpr uint32_t kF64Rebias = 896u << 20;
 
-// Bounded grid barrier: thread 0 of every CTA arrives and waits until the
+// Bounded grid barrier: thread 0 of every CTA arrives, runs `between` (work
+// that needs no other CTA, e.g. issuing prefetches) and waits until the
 // counter reaches target. Returns false (and records a timeout) on give-up.
-SBN_DEVFN bool grid_barrier(uint32_t* arrive, uint32_t target, int* s_abort) {
+template <class B>
+SBN_DEVFN bool grid_barrier(uint32_t* arrive, uint32_t target, int* s_abort, B&& between) {
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;\n" ::"l"(arrive) : "memory");
+    between();
     const unsigned long long t0 = global_ns();
     int abort = 0;
     while (ld_acquire_u32(arrive) < target) {
@@ -258,11 +261,13 @@ SBN_DEVFN void fill_compact_table(uint32_t* s_csel) {
 // Launch shape and dynamic shared memory of qw_fused_kernel. Every CTA owns a
 // contiguous range of units (16 consecutive weights of one row, 32 bytes),
 // i.e. one contiguous byte range of W, and streams it through a ring of
-// 16 KB stages filled by bulk copies: one stage is 512 units, one per thread.
+// 32 KB stages filled by bulk copies: one stage is 1024 units, two per
+// thread (units t and t + 512), whose instruction chains are independent.
 constexpr int kQwThreads = 512;
 constexpr int kQwWarps = kQwThreads / 32;
-constexpr int kQwChunk = 16384;       // bytes per stage
-constexpr int kQwStages = 8;          // 128 KB in flight per SM
+constexpr int kQwUpt = 2;             // units per thread per stage (two independent chains)
+constexpr int kQwChunk = 32 * kQwThreads * kQwUpt;   // bytes per stage (32 KB)
+constexpr int kQwStages = 4;          // 128 KB in flight per SM
 constexpr int kQwKeepCap = 16384;     // units whose keep bits stay in shared memory
 constexpr size_t kQwSmKeep = (size_t)kQwStages * kQwChunk;
 constexpr size_t kQwSmCsel = kQwSmKeep + (size_t)kQwKeepCap * 2;
@@ -360,11 +365,17 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int upr = k >> 4;                       // units per row
   const long long total_units = (long long)n_out * upr;
-  const long long u_begin = (long long)blockIdx.x * total_units / gridDim.x;
-  const long long u_end = (long long)(blockIdx.x + 1) * total_units / gridDim.x;
+  // CTA ranges start on 128-byte boundaries (4 units), so every bulk copy
+  // reads whole 128-byte lines
+  auto range_start = [&](long long b) {
+    return b >= (long long)gridDim.x ? total_units : (b * total_units / gridDim.x) & ~3LL;
+  };
+  const long long u_begin = range_start(blockIdx.x);
+  const long long u_end = range_start(blockIdx.x + 1);
   const bool has_meta = (n != M);
   const int cb = 4 * n / M;                     // code bytes per unit
-  const int row_step = kQwThreads / upr, u_step = kQwThreads % upr;
+  constexpr int kUnitsPerChunk = kQwThreads * kQwUpt;
+  const int row_step = kUnitsPerChunk / upr, u_step = kUnitsPerChunk % upr;
 
   QwRing ring;
   ring.src = reinterpret_cast<const uint8_t*>(w) + u_begin * 32;
@@ -382,12 +393,14 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   __syncthreads();
   qw_prologue(ring);
 
-  // (row, u) of this thread's unit in chunk c, advanced chunk by chunk
-  int row0, u0;
-  {
-    const long long g = u_begin + t;
-    row0 = (int)(g / upr);
-    u0 = (int)(g - (long long)row0 * upr);
+  // (row, u) of this thread's units in chunk c (slots j: unit t + 512 j of
+  // the chunk), advanced chunk by chunk
+  int row0[kQwUpt], u0[kQwUpt];
+#pragma unroll
+  for (int j = 0; j < kQwUpt; ++j) {
+    const long long g = u_begin + t + (long long)kQwThreads * j;
+    row0[j] = (int)(g / upr);
+    u0[j] = (int)(g - (long long)row0[j] * upr);
   }
   auto advance = [&](int& row, int& u) {
     row += row_step;
@@ -396,31 +409,43 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   };
 
   // ---- phase 1: fp64 sum and keep masks -------------------------------------
-  double d0 = 0.0, d1 = 0.0;
-  {
-    int row = row0, u = u0;
-    const bool ok = qw_pass(ring, &s_ok, [&](int c, const uint8_t* stage, int units_here) {
-      if (t < units_here) {
-        uint32_t wd[8], mw[8];
-        qw_load_unit(stage, t, wd);
+  // fp64 accumulators: four per unit slot (short dependency chains)
+  double dacc[kQwUpt][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          mw[i] = wd[i] & 0x7FFF7FFFu;
-          d0 += __hiloint2double((int)(((mw[i] & 0xFFFFu) << 13) + kF64Rebias), 0);
-          d1 += __hiloint2double((int)(((mw[i] >> 16) << 13) + kF64Rebias), 0);
+  for (int j = 0; j < kQwUpt; ++j)
+#pragma unroll
+    for (int a = 0; a < 4; ++a) dacc[j][a] = 0.0;
+  {
+    int row[kQwUpt], u[kQwUpt];
+#pragma unroll
+    for (int j = 0; j < kQwUpt; ++j) { row[j] = row0[j]; u[j] = u0[j]; }
+    const bool ok = qw_pass(ring, &s_ok, [&](int c, const uint8_t* stage, int units_here) {
+#pragma unroll
+      for (int j = 0; j < kQwUpt; ++j) {
+        const int ui = t + kQwThreads * j;
+        if (ui < units_here) {
+          uint32_t wd[8], mw[8];
+          qw_load_unit(stage, ui, wd);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            mw[i] = wd[i] & 0x7FFF7FFFu;
+            dacc[j][(2 * i) & 3] += __hiloint2double((int)(((mw[i] & 0xFFFFu) << 13) + kF64Rebias), 0);
+            dacc[j][(2 * i + 1) & 3] += __hiloint2double((int)(((mw[i] >> 16) << 13) + kF64Rebias), 0);
+          }
+          if (has_meta) {
+            const uint32_t keep = unit_keep_fast<M>(mw, n);
+            *reinterpret_cast<uint16_t*>(meta + (size_t)row[j] * meta_stride + 2 * u[j]) = (uint16_t)keep;
+            const int li = c * kUnitsPerChunk + ui;
+            if (li < kQwKeepCap) s_keep[li] = (uint16_t)keep;
+          }
         }
-        if (has_meta) {
-          const uint32_t keep = unit_keep_fast<M>(mw, n);
-          *reinterpret_cast<uint16_t*>(meta + (size_t)row * meta_stride + 2 * u) = (uint16_t)keep;
-          const int li = c * kQwThreads + t;
-          if (li < kQwKeepCap) s_keep[li] = (uint16_t)keep;
-        }
+        advance(row[j], u[j]);
       }
-      advance(row, u);
     });
     if (!ok) return;
   }
-  double dsum = d0 + d1;
+  double dsum = ((dacc[0][0] + dacc[0][1]) + (dacc[0][2] + dacc[0][3])) +
+                ((dacc[1][0] + dacc[1][1]) + (dacc[1][2] + dacc[1][3]));
 #pragma unroll
   for (int o = 16; o; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
   if (lane == 0) swarp_d[warp] = dsum;
@@ -430,10 +455,9 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     for (int i = 0; i < kQwWarps; ++i) a += swarp_d[i];
     gpart[blockIdx.x] = a;
   }
-  // the second pass re-reads the same range (now mostly in L2): start it
-  // before the grid barrier
-  qw_prologue(ring);
-  if (!grid_barrier(arrive, gridDim.x, &s_abort)) {
+  // the second pass re-reads the same range (now mostly in L2): its first
+  // copies are issued while the grid barrier is pending
+  if (!grid_barrier(arrive, gridDim.x, &s_abort, [&] { qw_prologue(ring); })) {
     qw_pass(ring, &s_ok, [](int, const uint8_t*, int) {});   // drain the prefetched stages
     return;
   }
@@ -452,12 +476,13 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     double S = 0.0;
     for (int i = 0; i < kQwWarps; ++i) S += swarp_d[i];
     const double nk = (double)n_out * (double)k;
-    // additions on the longest path: per-thread accumulator (8 per unit, one
-    // unit per chunk), d0 + d1, warp tree, warp sums of the CTA, then the
-    // same two levels over the CTA partials (counted generously)
-    const long long max_units = (total_units + gridDim.x - 1) / gridDim.x;
-    const double per_thread = 8.0 * (double)((max_units + kQwThreads - 1) / kQwThreads);
-    const double adds = per_thread + 1.0 + 2.0 * (5.0 + kQwWarps) + (double)gridDim.x;
+    // additions on the longest path: one accumulator (4 per unit, one unit
+    // per slot and chunk), the 3-level tree over the 8 accumulators, warp
+    // tree, warp sums of the CTA, then the same two levels over the CTA
+    // partials (counted generously)
+    const long long max_units = (total_units + gridDim.x - 1) / gridDim.x + 4;  // aligned ranges
+    const double per_thread = 4.0 * (double)((max_units + kQwThreads - 1) / kQwThreads);
+    const double adds = per_thread + 3.0 + 2.0 * (5.0 + kQwWarps) + (double)gridDim.x;
     const double err = S * adds * 0x1p-53 * 1.01 + nk * 0x1p-126 * 1.01;
     const double lo = (S - err) / nk * (1.0 - 0x1p-50);
     const double hi = (S + err) / nk * (1.0 + 0x1p-50);
@@ -476,13 +501,16 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     __syncthreads();
     unsigned long long acc = 0ull;
     const bool ok = qw_pass(ring, &s_ok, [&](int, const uint8_t* stage, int units_here) {
-      if (t < units_here) {
-        uint32_t wd[8];
-        qw_load_unit(stage, t, wd);
+      for (int j = 0; j < kQwUpt; ++j) {
+        const int ui = t + kQwThreads * j;
+        if (ui < units_here) {
+          uint32_t wd[8];
+          qw_load_unit(stage, ui, wd);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          exact_accumulate(wd[i] & 0x7FFFu, acc, sbins);
-          exact_accumulate((wd[i] >> 16) & 0x7FFFu, acc, sbins);
+          for (int i = 0; i < 8; ++i) {
+            exact_accumulate(wd[i] & 0x7FFFu, acc, sbins);
+            exact_accumulate((wd[i] >> 16) & 0x7FFFu, acc, sbins);
+          }
         }
       }
     });
@@ -504,8 +532,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     }
     for (int i = t; i < kQwBins; i += kQwThreads)
       if (sbins[i]) atomicAdd(&gbins[i], sbins[i]);
-    qw_prologue(ring);
-    if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort)) {
+    if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort, [&] { qw_prologue(ring); })) {
       qw_pass(ring, &s_ok, [](int, const uint8_t*, int) {});
       return;
     }
@@ -524,33 +551,40 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
 
   // ---- phase 2: codes of the kept positions ---------------------------------
   {
-    int row = row0, u = u0;
+    int row[kQwUpt], u[kQwUpt];
+#pragma unroll
+    for (int j = 0; j < kQwUpt; ++j) { row[j] = row0[j]; u[j] = u0[j]; }
     qw_pass(ring, &s_ok, [&](int c, const uint8_t* stage, int units_here) {
-      if (t < units_here) {
-        uint32_t wd[8];
-        qw_load_unit(stage, t, wd);
-        uint32_t keep = 0xFFFFu;
-        if (has_meta) {
-          const int li = c * kQwThreads + t;
-          keep = (li < kQwKeepCap)
-                     ? (uint32_t)s_keep[li]
-                     : (uint32_t) * reinterpret_cast<const uint16_t*>(meta + (size_t)row * meta_stride + 2 * u);
+#pragma unroll
+      for (int j = 0; j < kQwUpt; ++j) {
+        const int ui = t + kQwThreads * j;
+        if (ui < units_here) {
+          uint32_t wd[8];
+          qw_load_unit(stage, ui, wd);
+          uint32_t keep = 0xFFFFu;
+          if (has_meta) {
+            const int li = c * kUnitsPerChunk + ui;
+            keep = (li < kQwKeepCap)
+                       ? (uint32_t)s_keep[li]
+                       : (uint32_t) * reinterpret_cast<const uint16_t*>(meta + (size_t)row[j] * meta_stride +
+                                                                         2 * u[j]);
+          }
+          const uint32_t packed = unit_codes(wd, tau | (tau << 16), keep, s_csel);
+          uint8_t* dst = codes + (size_t)row[j] * codes_stride + (size_t)u[j] * cb;
+          if (cb == 4) {
+            *reinterpret_cast<uint32_t*>(dst) = packed;
+          } else if (cb == 2) {
+            *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+          } else {
+            for (int bb = 0; bb < cb; ++bb) dst[bb] = (uint8_t)(packed >> (8 * bb));
+          }
+          if (u[j] == upr - 1) {
+            // zero padding at the end of the row
+            for (int i = upr * cb; i < codes_stride; ++i) codes[(size_t)row[j] * codes_stride + i] = 0u;
+          }
         }
-        const uint32_t packed = unit_codes(wd, tau | (tau << 16), keep, s_csel);
-        uint8_t* dst = codes + (size_t)row * codes_stride + (size_t)u * cb;
-        if (cb == 4) {
-          *reinterpret_cast<uint32_t*>(dst) = packed;
-        } else if (cb == 2) {
-          *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
-        } else {
-          for (int bb = 0; bb < cb; ++bb) dst[bb] = (uint8_t)(packed >> (8 * bb));
-        }
-        if (u == upr - 1) {
-          // zero padding at the end of the row
-          for (int i = upr * cb; i < codes_stride; ++i) codes[(size_t)row * codes_stride + i] = 0u;
-        }
+        advance(row[j], u[j]);
       }
-      advance(row, u);
     });
   }
 }
