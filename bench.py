@@ -379,38 +379,45 @@ def run_ours(args, rank, world, local_rank):
     def enqueue_step(sl, evs=None):
         i = 0
         for li, L in enumerate(sl):
-            if evs: evs[i][0].record(stream)
+            if evs and evs[i]: evs[i][0].record(stream)
             sbn.quantize_weights(L["w"], L["n"], L["m"], out=L["pw"], workspace=L["ws"], stream=stream)
-            if evs: evs[i][1].record(stream)
+            if evs and evs[i]: evs[i][1].record(stream)
             i += 1
             for x, (q, s), y in zip(L["xs"], L["qs"], L["ys"]):
                 if fused:
-                    if evs: evs[i][0].record(stream)
+                    if evs and evs[i]: evs[i][0].record(stream)
                     sbn.bitlinear_x(x, L["pw"], out=y, workspace=L["bws"], stream=stream)
-                    if evs: evs[i][1].record(stream)
+                    if evs and evs[i]: evs[i][1].record(stream)
                     i += 1
                     continue
-                if evs: evs[i][0].record(stream)
+                if evs and evs[i]: evs[i][0].record(stream)
                 sbn.quantize_acts(x, out_q=q, out_s=s, stream=stream)
-                if evs: evs[i][1].record(stream)
+                if evs and evs[i]: evs[i][1].record(stream)
                 i += 1
-                if evs: evs[i][0].record(stream)
+                if evs and evs[i]: evs[i][0].record(stream)
                 sbn.bitlinear(q, s, L["pw"], out=y, workspace=L["bws"], stream=stream)
-                if evs: evs[i][1].record(stream)
+                if evs and evs[i]: evs[i][1].record(stream)
                 i += 1
 
-    graphs, slot_events = [], []
+    def capture(which):
+        """One graph per slot; events around the calls `which` selects."""
+        gs, evss = [], []
+        for r in range(R):
+            evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) if which(c) else None
+                   for c in call_names]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                enqueue_step(slots[r], evs)
+            gs.append(g)
+            evss.append(evs)
+        return gs, evss
+
     with torch.cuda.stream(stream):
         enqueue_step(slots[0])  # load kernels before capture
     stream.synchronize()
-    for r in range(R):
-        evs = [(torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) for _ in call_names]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            enqueue_step(slots[r], evs)
-        graphs.append(g)
-        slot_events.append(evs)
+    # calibration graphs: every call bracketed by events (per-call breakdown)
+    cal_graphs, cal_events = capture(lambda c: True)
     # our kernels per step: quantize_weights 1 per layer; quantize_acts 1 and
     # bitlinear 1 (+1 weight expansion when T > 16) per token set
     # (fused: one kernel per token set for T <= 16)
@@ -422,10 +429,27 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    # warm-up
+    # warm-up, then one calibration replay per slot (untimed)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            graphs[i % R].replay()
+            cal_graphs[i % R].replay()
+        for r in range(R):
+            cal_graphs[r].replay()
+    stream.synchronize()
+    per_call = {}
+    for r in range(R):
+        for (name, li, t), ab in zip(call_names, cal_events[r]):
+            per_call.setdefault((name, li, t), []).append(ab[0].elapsed_time(ab[1]))
+    cal_totals = {}
+    for (name, li, t), v in per_call.items():
+        cal_totals[name] = cal_totals.get(name, 0.0) + statistics.mean(v)
+    dom = max(cal_totals, key=cal_totals.get)
+    # timed graphs: events only around the dominant call (its live launch
+    # durations for the roofline), so the other calls run back to back
+    graphs, slot_events = capture(lambda c: c[0] == dom)
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            graphs[r].replay()
     stream.synchronize()
 
     clocks = ClockSampler(local_rank)
@@ -445,12 +469,13 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1)
 
-    # per-call durations of the last replay of every slot (inside the timed region)
+    # the dominant call's durations in the last timed replay of every slot
     used = min(R, args.steps)
-    per_call = {}
+    dom_calls = {}
     for r in range(used):
-        for (name, li, t), (a, b) in zip(call_names, slot_events[r]):
-            per_call.setdefault((name, li, t), []).append(a.elapsed_time(b))
+        for (name, li, t), ab in zip(call_names, slot_events[r]):
+            if ab:
+                dom_calls.setdefault((name, li, t), []).append(ab[0].elapsed_time(ab[1]))
 
     ms = max_over_ranks(ms, world, dev)
 
@@ -458,13 +483,9 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = ms / args.steps
     value = whole_job_value(args.workload, args.steps, world, ms)
 
-    # dominant call by total time in a step
-    totals = {}
-    for (name, li, t), v in per_call.items():
-        totals.setdefault(name, 0.0)
-        totals[name] += statistics.mean(v)
-    dom = max(totals, key=totals.get)
-    dom_ms = totals[dom]
+    # dominant call (by total time in a calibration step): its time per step
+    # in the timed region
+    dom_ms = sum(statistics.mean(v) for v in dom_calls.values())
     peaks = load_peaks()
     n_dom_launches = len([c for c in call_names if c[0] == dom])
     traffic = ncu_traffic(dom, args.workload)
@@ -552,6 +573,9 @@ def run_ours(args, rank, world, local_rank):
                        "parallelism": f"replicas x{world} (independent layers per rank)"},
             "tokens_per_s": round(step_tokens(layers) * args.steps * world / (ms * 1e-3), 1),
             "roofline": roofline, "breakdown": breakdown,
+            "breakdown_note": "per-call means from one untimed replay per rotation slot with "
+                              "events around every call; the timed replays bracket only the "
+                              "dominant call (roofline.launch_us)",
             "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": clk, "cpu_baseline": cpu,
         }

@@ -151,7 +151,7 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kTcEpilogue / 32);
+      mbar_init(&acc_empty[b], TMA_A ? 2 * kTcEpilogue / 32 : kTcEpilogue / 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -299,9 +299,14 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
         if (lane == 0) mbar_arrive(&full[s]);
       }
     }
-  } else if (warp >= 12) {
+  } else if (TMA_A ? (warp >= 4 && warp < 12) : warp >= 12) {
     // ---- epilogue: TMEM -> registers -> y (or acc) ----
+    // warp w reads TMEM lane quadrant w % 4; with TMA_A the idle producer
+    // warps 4-11 drain the accumulator, two per quadrant, each half of the
+    // columns; otherwise warps 12-15 drain all of them
     const int q = warp & 3;
+    const int c_first = TMA_A ? ((warp - 4) >> 2) * (kTcBN / 64) : 0;
+    const int c_count = TMA_A ? kTcBN / 64 : kTcBN / 32;
     const int row_in_tile = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const float g = ACC ? 0.f : __ldg(p.gamma);
@@ -316,7 +321,7 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
       if (!got) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < kTcBN / 32; ++c) {
+      for (int c = c_first; c < c_first + c_count; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + (uint32_t)(b * kTcBN + 32 * c), r);
         // lane jj holds the scale gamma * s_t / 127 of token tok0 + 32c + jj
