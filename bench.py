@@ -2,17 +2,23 @@
 """Benchmark of the Sparse-BitNet BitLinear forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|qwen|ffn3b]
+                    [--workload decode|prefill]
 
 One step is one pass of the whole path over one batch of synthetic input:
 sbn_quantize_weights on the latent weights (the dynamic N:M mask is
-recomputed every forward), then sbn_quantize_acts + sbn_bitlinear for the
-step's activations. The default workload is the decode GEMV sweep:
-W [6912, 2560] bf16 ~ N(0, 0.02), 6:8, activations of T = 1, 4 and 16 tokens.
+recomputed every forward), then, for every token set, the activation
+quantization and the contraction: sbn_bitlinear_x (fused) for the decode
+workload, sbn_quantize_acts + sbn_bitlinear for prefill. The default workload
+is the decode GEMV sweep: W [6912, 2560] bf16 ~ N(0, 0.02), 6:8, activations
+of T = 1, 4 and 16 tokens. The prefill workload is T = 4096 through
+(K, N_out) = (2560, 6912) and (6912, 2560) at 2:4. The other shapes of the
+pages' workloads are covered by the parity tests.
 
 Timing: each step is a captured CUDA graph; steps rotate over enough
 distinct copies of the inputs and outputs that their total exceeds 3x the
-L2 cache, so no step reads another step's data from L2. The timed region is
+L2 cache, so no step reads another step's data from L2. An untimed
+calibration replay with events around every call gives the per-call
+breakdown; the timed replays bracket only the dominant call. The timed region is
 K graph replays bracketed by barrier + synchronize, timed with CUDA events;
 for N > 1 the max over ranks is taken and every rank runs its own
 independent layer (weak scaling, no collective on the data path).
