@@ -51,16 +51,32 @@ SBN_DEVFN uint32_t ld_acquire_u32(const uint32_t* p) {
 // normal magnitudes, near 2^-127 for zero and subnormals.
 constexpr uint32_t kF64Rebias = 896u << 20;
 
-// Bounded grid barrier: thread 0 of every CTA arrives, runs `between` (work
-// that needs no other CTA, e.g. issuing prefetches) and waits until the
-// counter reaches target. Returns false (and records a timeout) on give-up.
-template <class B>
-SBN_DEVFN bool grid_barrier(uint32_t* arrive, uint32_t target, int* s_abort, B&& between) {
+// Barrier of the 512 consumer threads of qw_fused_kernel (named barrier 1;
+// the producer warp never takes part).
+constexpr int kQwConsumerThreads = 512;
+SBN_DEVFN void qw_cons_sync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(kQwConsumerThreads) : "memory");
+}
+
+// True on every consumer thread if v is true on any (barrier 1, with reduction).
+SBN_DEVFN bool qw_cons_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, 1, %2, p;\nselp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kQwConsumerThreads)
+      : "memory");
+  return r != 0u;
+}
+
+// Bounded grid barrier among the consumers: thread 0 of every CTA arrives and
+// waits until the counter reaches target. Returns false (and records a
+// timeout) on give-up.
+SBN_DEVFN bool grid_barrier(uint32_t* arrive, uint32_t target, int* s_abort) {
   __threadfence();
-  __syncthreads();
+  qw_cons_sync();
   if (threadIdx.x == 0) {
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;\n" ::"l"(arrive) : "memory");
-    between();
     const unsigned long long t0 = global_ns();
     int abort = 0;
     while (ld_acquire_u32(arrive) < target) {
@@ -73,7 +89,7 @@ SBN_DEVFN bool grid_barrier(uint32_t* arrive, uint32_t target, int* s_abort, B&&
     }
     *s_abort = abort;
   }
-  __syncthreads();
+  qw_cons_sync();
   const bool ok = !*s_abort;
   __threadfence();
   return ok;
@@ -263,7 +279,7 @@ SBN_DEVFN void fill_compact_table(uint32_t* s_csel) {
 // i.e. one contiguous byte range of W, and streams it through a ring of
 // 32 KB stages filled by bulk copies: one stage is 1024 units, two per
 // thread (units t and t + 512), whose instruction chains are independent.
-constexpr int kQwThreads = 512;
+constexpr int kQwThreads = kQwConsumerThreads;   // consumer threads; one producer warp more
 constexpr int kQwWarps = kQwThreads / 32;
 constexpr int kQwUpt = 2;             // units per thread per stage (two independent chains)
 constexpr int kQwChunk = 32 * kQwThreads * kQwUpt;   // bytes per stage (32 KB)
@@ -273,62 +289,52 @@ constexpr size_t kQwSmKeep = (size_t)kQwStages * kQwChunk;
 constexpr size_t kQwSmCsel = kQwSmKeep + (size_t)kQwKeepCap * 2;
 constexpr size_t kQwSmBins = kQwSmCsel + 256 * 4;
 constexpr size_t kQwSmBars = kQwSmBins + (size_t)kQwBins * 8;
-constexpr size_t kQwSmemBytes = kQwSmBars + (size_t)kQwStages * 8;
+constexpr size_t kQwSmemBytes = kQwSmBars + (size_t)(2 * kQwStages + 1) * 8;
 
-// Stream ring over one CTA's byte range of W.
+// Stream ring over one CTA's byte range of W. The producer warp copies the
+// range once per pass into a ring of stages; the consumer warps take each
+// stage when its `full` barrier completes (the copy's bytes) and release it
+// with one arrival per warp on its `empty` barrier. Chunks are numbered
+// across passes (q); chunk q uses stage q % kQwStages for the (q /
+// kQwStages)-th time, so its phase parity is (q / kQwStages) & 1.
 struct QwRing {
   const uint8_t* src;   // first byte of the range
   long long bytes;      // length (a multiple of 32)
   int nch;              // chunks in the range
   uint8_t* buf;         // kQwStages x kQwChunk
-  uint64_t* full;       // one mbarrier per stage
-  uint32_t seq;         // chunks consumed so far, over all passes (uniform)
+  uint64_t* full;       // per stage: the producer's arrival + the copied bytes
+  uint64_t* empty;      // per stage: one arrival per consumer warp
 };
 
-SBN_DEVFN void qw_issue(const QwRing& r, int c, uint32_t q) {
-  const int st = (int)(q % kQwStages);
-  const long long off = (long long)c * kQwChunk;
-  const uint32_t nb = (uint32_t)min((long long)kQwChunk, r.bytes - off);
-  mbar_arrive_expect_tx(&r.full[st], nb);
-  bulk_g2s(r.buf + (size_t)st * kQwChunk, r.src + off, nb, &r.full[st]);
-}
-
-// Issues the first stages of the next pass (thread 0).
-SBN_DEVFN void qw_prologue(const QwRing& r) {
-  if (threadIdx.x == 0)
-    for (int c = 0; c < min(r.nch, kQwStages); ++c) qw_issue(r, c, r.seq + (uint32_t)c);
-}
-
-// One pass over the range, whose prologue is already issued: f(c, stage,
-// units_here) runs for every chunk on every thread. Thread 0 alone waits for
-// a chunk; the block barrier after its wait publishes the chunk to the
-// others and frees the stage of the previous chunk, which thread 0 then
-// refills. If a wait gives up, the copies still in flight are waited for
-// (bounded) and false is returned on every thread.
-template <class F>
-SBN_DEVFN bool qw_pass(QwRing& r, int* s_ok, F&& f) {
-  for (int c = 0; c < r.nch; ++c) {
-    const uint32_t q = r.seq + (uint32_t)c;
+// Producer (one thread): one pass over the range, chunk numbers q onwards.
+SBN_DEVFN bool qw_produce_pass(const QwRing& r, uint32_t& q) {
+  for (int c = 0; c < r.nch; ++c, ++q) {
     const int st = (int)(q % kQwStages);
-    if (threadIdx.x == 0) *s_ok = mbar_wait(&r.full[st], (q / kQwStages) & 1u) ? 1 : 0;
-    __syncthreads();
-    if (!*s_ok) {
-      if (threadIdx.x == 0) {
-        for (int d = c + 1; d < min(r.nch, c + kQwStages); ++d) {
-          const uint32_t qd = r.seq + (uint32_t)d;
-          if (!mbar_wait(&r.full[qd % kQwStages], (qd / kQwStages) & 1u)) break;
-        }
-      }
-      __syncthreads();
-      return false;
-    }
-    if (threadIdx.x == 0 && c >= 1 && c - 1 + kQwStages < r.nch)
-      qw_issue(r, c - 1 + kQwStages, q - 1 + kQwStages);
+    if (q >= (uint32_t)kQwStages && !mbar_wait(&r.empty[st], ((q / kQwStages) - 1u) & 1u)) return false;
+    const long long off = (long long)c * kQwChunk;
+    const uint32_t nb = (uint32_t)min((long long)kQwChunk, r.bytes - off);
+    mbar_arrive_expect_tx(&r.full[st], nb);
+    bulk_g2s(r.buf + (size_t)st * kQwChunk, r.src + off, nb, &r.full[st]);
+  }
+  return true;
+}
+
+// Consumer warp: one pass; f(c, stage, units_here) runs on every consumer
+// thread for every chunk. Lane 0 waits, the warp follows; false if a wait
+// gave up.
+template <class F>
+SBN_DEVFN bool qw_consume_pass(const QwRing& r, uint32_t& q, F&& f) {
+  const int lane = threadIdx.x & 31;
+  for (int c = 0; c < r.nch; ++c, ++q) {
+    const int st = (int)(q % kQwStages);
+    int got = 1;
+    if (lane == 0) got = mbar_wait(&r.full[st], (q / kQwStages) & 1u) ? 1 : 0;
+    if (!__shfl_sync(0xffffffffu, got, 0)) return false;
     const int units_here = (int)(min((long long)kQwChunk, r.bytes - (long long)c * kQwChunk) >> 5);
     f(c, r.buf + (size_t)st * kQwChunk, units_here);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&r.empty[st]);
   }
-  __syncthreads();  // every thread is done with the last stages before they are reused
-  r.seq += (uint32_t)r.nch;
   return true;
 }
 
@@ -344,7 +350,7 @@ SBN_DEVFN void qw_load_unit(const uint8_t* stage, int t, uint32_t (&wd)[8]) {
 }
 
 template <int M>
-__global__ void __launch_bounds__(kQwThreads, 1)
+__global__ void __launch_bounds__(kQwThreads + 32, 1)
 qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
                 uint8_t* __restrict__ codes, int codes_stride, uint8_t* __restrict__ meta,
                 int meta_stride, float* __restrict__ gamma_out, unsigned char* __restrict__ ws) {
@@ -353,10 +359,12 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   uint32_t* s_csel = reinterpret_cast<uint32_t*>(qw_smem + kQwSmCsel);
   unsigned long long* sbins = reinterpret_cast<unsigned long long*>(qw_smem + kQwSmBins);
   uint64_t* full = reinterpret_cast<uint64_t*>(qw_smem + kQwSmBars);
+  uint64_t* empty = full + kQwStages;
+  uint64_t* decided = empty + kQwStages;     // thread 0: the pass count is known
   __shared__ double swarp_d[kQwWarps];
   __shared__ unsigned long long swarp[kQwWarps];
   __shared__ uint32_t s_tau;
-  __shared__ int s_abort, s_exact, s_ok;
+  __shared__ int s_abort, s_exact;
 
   unsigned long long* gbins = reinterpret_cast<unsigned long long*>(ws);
   uint32_t* arrive = reinterpret_cast<uint32_t*>(ws + kQwArriveOffset);
@@ -383,15 +391,33 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
   ring.nch = (int)((ring.bytes + kQwChunk - 1) / kQwChunk);
   ring.buf = qw_smem;
   ring.full = full;
-  ring.seq = 0u;
+  ring.empty = empty;
 
   if (t == 0) {
-    for (int s = 0; s < kQwStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < kQwStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kQwWarps);
+    }
+    mbar_init(decided, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   fill_compact_table(s_csel);
-  __syncthreads();
-  qw_prologue(ring);
+  __syncthreads();   // the only barrier of all 544 threads
+
+  if (warp == kQwWarps) {
+    // ---- producer warp: lane 0 streams the range for every pass ----------
+    if (lane == 0) {
+      uint32_t q = 0u;
+      bool ok = qw_produce_pass(ring, q) && qw_produce_pass(ring, q);   // pass 1, then pass 2
+      // a third pass when gamma needs the exact integer bins
+      if (ok && mbar_wait(decided, 0u) && s_exact) ok = qw_produce_pass(ring, q);
+      // no copy may still be in flight when the CTA exits
+      for (uint32_t d = q > (uint32_t)kQwStages ? q - kQwStages : 0u; d < q; ++d)
+        if (!mbar_wait(&full[d % kQwStages], (d / kQwStages) & 1u)) break;
+    }
+    return;
+  }
+  uint32_t cq = 0u;   // consumer chunk number (the same in every consumer warp)
 
   // (row, u) of this thread's units in chunk c (slots j: unit t + 512 j of
   // the chunk), advanced chunk by chunk
@@ -419,7 +445,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     int row[kQwUpt], u[kQwUpt];
 #pragma unroll
     for (int j = 0; j < kQwUpt; ++j) { row[j] = row0[j]; u[j] = u0[j]; }
-    const bool ok = qw_pass(ring, &s_ok, [&](int c, const uint8_t* stage, int units_here) {
+    const bool ok = qw_consume_pass(ring, cq, [&](int c, const uint8_t* stage, int units_here) {
 #pragma unroll
       for (int j = 0; j < kQwUpt; ++j) {
         const int ui = t + kQwThreads * j;
@@ -442,23 +468,28 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
         advance(row[j], u[j]);
       }
     });
-    if (!ok) return;
+    // a warp whose wait gave up stops here; the others finish the pass (their
+    // waits are bounded too), then all leave together
+    if (qw_cons_any(!ok)) {
+      if (t == 0) { s_exact = 0; mbar_arrive(decided); }
+      return;
+    }
   }
   double dsum = ((dacc[0][0] + dacc[0][1]) + (dacc[0][2] + dacc[0][3])) +
                 ((dacc[1][0] + dacc[1][1]) + (dacc[1][2] + dacc[1][3]));
 #pragma unroll
   for (int o = 16; o; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
   if (lane == 0) swarp_d[warp] = dsum;
-  __syncthreads();
+  qw_cons_sync();
   if (t == 0) {
     double a = 0.0;
     for (int i = 0; i < kQwWarps; ++i) a += swarp_d[i];
     gpart[blockIdx.x] = a;
   }
-  // the second pass re-reads the same range (now mostly in L2): its first
-  // copies are issued while the grid barrier is pending
-  if (!grid_barrier(arrive, gridDim.x, &s_abort, [&] { qw_prologue(ring); })) {
-    qw_pass(ring, &s_ok, [](int, const uint8_t*, int) {});   // drain the prefetched stages
+  // meanwhile the producer already streams pass 2 (the same range, now
+  // mostly in L2) into the stages pass 1 released
+  if (!grid_barrier(arrive, gridDim.x, &s_abort)) {
+    if (t == 0) { s_exact = 0; mbar_arrive(decided); }
     return;
   }
 
@@ -471,7 +502,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) swarp_d[warp] = v;
   }
-  __syncthreads();
+  qw_cons_sync();
   if (t == 0) {
     double S = 0.0;
     for (int i = 0; i < kQwWarps; ++i) S += swarp_d[i];
@@ -493,14 +524,15 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
       s_tau = code_threshold(glo);
       if (blockIdx.x == 0) *gamma_out = glo;
     }
+    mbar_arrive(decided);   // the producer learns whether a third pass follows
   }
-  __syncthreads();
+  qw_cons_sync();
   if (s_exact) {
     // rare: exact integer bins over the same range, second barrier
     for (int i = t; i < kQwBins; i += kQwThreads) sbins[i] = 0ull;
-    __syncthreads();
+    qw_cons_sync();
     unsigned long long acc = 0ull;
-    const bool ok = qw_pass(ring, &s_ok, [&](int, const uint8_t* stage, int units_here) {
+    const bool ok = qw_consume_pass(ring, cq, [&](int, const uint8_t* stage, int units_here) {
       for (int j = 0; j < kQwUpt; ++j) {
         const int ui = t + kQwThreads * j;
         if (ui < units_here) {
@@ -514,11 +546,11 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
         }
       }
     });
-    if (!ok) return;
+    if (qw_cons_any(!ok)) return;
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) swarp[warp] = acc;
-    __syncthreads();
+    qw_cons_sync();
     if (t == 0) {
       unsigned long long a = 0ull;
       for (int i = 0; i < kQwWarps; ++i) a += swarp[i];
@@ -532,10 +564,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     }
     for (int i = t; i < kQwBins; i += kQwThreads)
       if (sbins[i]) atomicAdd(&gbins[i], sbins[i]);
-    if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort, [&] { qw_prologue(ring); })) {
-      qw_pass(ring, &s_ok, [](int, const uint8_t*, int) {});
-      return;
-    }
+    if (!grid_barrier(arrive, 2u * gridDim.x, &s_abort)) return;
     if (warp == 0) {
       float g;
       uint32_t tau;
@@ -545,7 +574,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
         if (blockIdx.x == 0) *gamma_out = g;
       }
     }
-    __syncthreads();
+    qw_cons_sync();
   }
   const uint32_t tau = s_tau;
 
@@ -554,7 +583,7 @@ qw_fused_kernel(const uint16_t* __restrict__ w, int n_out, int k, int n,
     int row[kQwUpt], u[kQwUpt];
 #pragma unroll
     for (int j = 0; j < kQwUpt; ++j) { row[j] = row0[j]; u[j] = u0[j]; }
-    qw_pass(ring, &s_ok, [&](int c, const uint8_t* stage, int units_here) {
+    qw_consume_pass(ring, cq, [&](int c, const uint8_t* stage, int units_here) {
 #pragma unroll
       for (int j = 0; j < kQwUpt; ++j) {
         const int ui = t + kQwThreads * j;

@@ -98,7 +98,7 @@ sbn_status launch_qw_fused(const uint16_t* w, int n_out, int k, int n, uint8_t* 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)std::min(sms, kQwMaxGrid));
-  cfg.blockDim = dim3(kQwThreads);
+  cfg.blockDim = dim3(kQwThreads + 32);   // consumers + the producer warp
   cfg.dynamicSmemBytes = kQwSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
