@@ -7,12 +7,12 @@
 // unpacked there and contracted with 8-bit activations, so HBM carries only
 // the packed bytes. Decoding is bound by those bytes.
 //
-// A CTA owns a contiguous range of 16-row tiles. Thread 0 issues, at once,
-// a few large bulk copies (each copy has a fixed cost, so few and large beats
-// many and small): all of Xq in one, then the code rows and the keep-bit rows
-// of the tiles in at most two groups, each group completing its own mbarrier.
-// The 32 warps walk the (tile, 128-position segment) items in tile-major
-// order, so the first group is contracted while the second is arriving. Per item a thread
+// A CTA owns a contiguous range of 16-row tiles. At entry all 1024 threads
+// issue 16-byte asynchronous copies (cp.async) of the tiles' code rows and
+// keep-bit rows and of the activations, about seven per thread, all in
+// flight at once; one wait and one block barrier later everything is in
+// shared memory. The 32 warps then walk the (tile, 128-position segment)
+// items. Per item a thread
 // expands 32 positions of two rows (expand.cuh) straight into the A fragment
 // of `mma.sync.m16n8k32.s8` (weights as the 16-row operand, tokens as the 8
 // columns, a K permutation shared with the activation fragment). A warp adds
@@ -26,7 +26,6 @@
 // (qa.cuh), and CTA 0 optionally writes Xq and s to global memory.
 #pragma once
 
-#include "async.cuh"
 #include "bl_decode.cuh"
 #include "common.cuh"
 #include "expand.cuh"
@@ -99,55 +98,36 @@ bl_decode_res_kernel(const DresParams p) {
   uint8_t* s_meta = dres_smem + L.meta;
   uint16_t* s_xbf = reinterpret_cast<uint16_t*>(dres_smem + L.xbf);
   float* s_scale = reinterpret_cast<float*>(dres_smem + L.scale);
-  uint64_t* bar_x = reinterpret_cast<uint64_t*>(dres_smem + L.bars);
-  uint64_t* bar_t = bar_x + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int row0 = t_begin * 16;
-  // tiles [0, split) form copy group 0, [split, tiles) group 1 (if any)
-  const int ngrp = tiles > 1 ? 2 : 1;
-  const int split = ngrp == 2 ? tiles / 2 : tiles;
-
-  if (tid == 0) {
-    // the copies start at once; the other threads meet the barriers after
-    // the block-wide sync below
-    mbar_init(bar_x, 1);
-    for (int i = 0; i < ngrp; ++i) mbar_init(&bar_t[i], 1);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    if (XBF) {
-      mbar_arrive_expect_tx(bar_x, (uint32_t)(p.T * p.K * 2));
-      bulk_g2s(s_xbf, p.xbf, (uint32_t)(p.T * p.K * 2), bar_x);
-    } else {
-      mbar_arrive_expect_tx(bar_x, (uint32_t)(p.T * p.K));
-      bulk_g2s(s_x, p.xq, (uint32_t)(p.T * p.K), bar_x);
+  const int rows_valid = min(16 * tiles, p.N - row0);
+  {
+    // every thread issues its share of 16-byte asynchronous copies of this
+    // CTA's code rows, keep-bit rows and activations: all of them are in
+    // flight at once, with no per-copy cost of a bulk copy engine
+    const int nx = XBF ? p.T * p.K * 2 / 16 : p.T * p.K / 16;
+    const int nc = rows_valid * p.cstride / 16;
+    const int nm = DENSE ? 0 : rows_valid * p.mstride / 16;
+    const uint8_t* gx = XBF ? reinterpret_cast<const uint8_t*>(p.xbf) : reinterpret_cast<const uint8_t*>(p.xq);
+    uint8_t* sx = XBF ? reinterpret_cast<uint8_t*>(s_xbf) : s_x;
+    const uint8_t* gc = p.codes + (size_t)row0 * p.cstride;
+    for (int i = tid; i < nx; i += kDresThreads) cp_async16(sx + 16 * (size_t)i, gx + 16 * (size_t)i, true);
+    for (int i = tid; i < nc; i += kDresThreads) cp_async16(s_codes + 16 * (size_t)i, gc + 16 * (size_t)i, true);
+    if (!DENSE) {
+      const uint8_t* gm = p.meta + (size_t)row0 * p.mstride;
+      for (int i = tid; i < nm; i += kDresThreads) cp_async16(s_meta + 16 * (size_t)i, gm + 16 * (size_t)i, true);
     }
-    for (int gi = 0; gi < ngrp; ++gi) {
-      const int ta = gi ? split : 0, tb = gi ? tiles : split;
-      const int r = row0 + 16 * ta;
-      const int nrows = min(16 * (tb - ta), p.N - r);
-      const uint32_t cbytes = (uint32_t)(nrows * p.cstride);
-      const uint32_t mbytes = DENSE ? 0u : (uint32_t)(nrows * p.mstride);
-      mbar_arrive_expect_tx(&bar_t[gi], cbytes + mbytes);
-      bulk_g2s(s_codes + (size_t)ta * 16 * p.cstride, p.codes + (size_t)r * p.cstride, cbytes, &bar_t[gi]);
-      if (!DENSE)
-        bulk_g2s(s_meta + (size_t)ta * 16 * p.mstride, p.meta + (size_t)r * p.mstride, mbytes, &bar_t[gi]);
-    }
+    cp_async_commit();
   }
   if (!DENSE) fill_selector_table(s_sel);
   for (int i = tid; i < tiles * 16 * NT; i += kDresThreads) s_acc[i] = 0;
+  cp_async_wait<0>();
   __syncthreads();
-
-  // lane 0 waits, the warp follows it (the MMAs need the whole warp)
-  auto warp_wait = [&](uint64_t* bar) {
-    int got = 1;
-    if (lane == 0) got = mbar_wait(bar, 0u) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, got, 0) != 0;
-  };
-  bool ok = warp_wait(bar_x);
   if (XBF) {
     // warp `warp` quantizes token row `warp` (T <= 16 <= warps)
-    if (ok && warp < p.T) {
+    if (warp < p.T) {
       const uint4* xr = reinterpret_cast<const uint4*>(s_xbf + (size_t)warp * p.K);
       const int kc = p.K / 8;
       uint32_t amax = 0u;
@@ -168,7 +148,7 @@ bl_decode_res_kernel(const DresParams p) {
         if (blockIdx.x == 0 && p.xs_out) p.xs_out[warp] = sc;
       }
     }
-    ok = __syncthreads_and(ok) != 0;
+    __syncthreads();
   }
   const int ksegs = p.K / 128;
   const int items = tiles * ksegs;
@@ -191,12 +171,11 @@ bl_decode_res_kernel(const DresParams p) {
     for (int i = 0; i < 4; ++i) acc0[i] = acc1[i] = 0;
   };
 
-  for (int it = warp; ok && it < items; it += kDresWarps) {
+  for (int it = warp; it < items; it += kDresWarps) {
     const int tile = it / ksegs, kseg = it - tile * ksegs;
     if (tile != cur_tile) {
       if (cur_tile >= 0) flush(cur_tile);
       cur_tile = tile;
-      if (!warp_wait(&bar_t[tile < split ? 0 : 1])) { ok = false; break; }
     }
     const uint8_t* ct = s_codes + (size_t)tile * 16 * p.cstride;
     const uint8_t* mt = s_meta + (size_t)tile * 16 * p.mstride;
@@ -239,13 +218,7 @@ bl_decode_res_kernel(const DresParams p) {
       }
     }
   }
-  if (ok && cur_tile >= 0) flush(cur_tile);
-  __syncthreads();
-  if (tid == 0) {
-    // every copy of this CTA has landed before the CTA may exit
-    mbar_wait(bar_x, 0u);
-    for (int i = 0; i < ngrp; ++i) mbar_wait(&bar_t[i], 0u);
-  }
+  if (cur_tile >= 0) flush(cur_tile);
   __syncthreads();
 
   const float gm = ACC ? 0.f : __ldg(p.gamma);
