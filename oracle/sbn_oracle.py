@@ -79,6 +79,13 @@ __all__ = [
     "bitlinear_at",
     "mask_flips",
     "mask_flip_rate",
+    "mask_index_bits",
+    "colex_rank",
+    "colex_unrank",
+    "entropy_group_bits",
+    "entropy_row_bytes",
+    "entropy_pack",
+    "entropy_unpack",
 ]
 
 #: floor on gamma and on the per-token activation scale (not on the pages)
@@ -400,3 +407,88 @@ def mask_flips(mask_a: np.ndarray, mask_b: np.ndarray) -> int:
 def mask_flip_rate(mask_a: np.ndarray, mask_b: np.ndarray) -> float:
     """r_t = mask_flips / number of positions."""
     return mask_flips(mask_a, mask_b) / float(np.asarray(mask_a).size)
+
+
+# --------------------------------------------------------------------------
+# entropy-tight packed format
+# --------------------------------------------------------------------------
+#
+# "From 2:4 to 8:16 sparsity patterns in LLMs for Outliers and Weights with
+# Variance Correction", Abstract: the mask of 2:4 costs 0.75 and that of 8:16
+# 0.875 bits per element. Both equal ceil(log2 C(m, n)) / m, the size of an
+# index that numbers every keep pattern of a group. The format below stores,
+# per group of m positions, one integer word
+#     word = rank(kept positions) * 3**n + sum_i (code_i + 1) * 3**i
+# (kept codes in ascending position order, i from 0) in
+# ceil(log2(C(m, n) * 3**n)) bits; rank is the combinatorial number system
+# (colex) rank: for kept offsets c_1 < ... < c_n within the group,
+# rank = sum_i C(c_i, i). The words of a row are concatenated little-endian
+# (bit b of the row stream is bit b % 8 of byte b // 8) and the row is padded
+# with zero bytes to a multiple of 16.
+
+def mask_index_bits(n: int, m: int) -> int:
+    """Bits of an index that numbers the C(m, n) keep patterns of a group."""
+    c = math.comb(m, n)
+    return 0 if c == 1 else (c - 1).bit_length()
+
+
+def entropy_group_bits(n: int, m: int) -> int:
+    """Bits of one group word: keep pattern and kept ternary values jointly."""
+    return (math.comb(m, n) * 3 ** n - 1).bit_length()
+
+
+def entropy_row_bytes(k: int, n: int, m: int) -> int:
+    return _round_up((k // m * entropy_group_bits(n, m) + 7) // 8, 16)
+
+
+def colex_rank(offsets) -> int:
+    return sum(math.comb(c, i + 1) for i, c in enumerate(offsets))
+
+
+def colex_unrank(rank: int, n: int, m: int):
+    """Kept offsets (ascending) of the pattern with the given colex rank."""
+    out = []
+    for i in range(n, 0, -1):
+        c = i - 1
+        while math.comb(c + 1, i) <= rank:
+            c += 1
+        out.append(c)
+        rank -= math.comb(c, i)
+    return sorted(out)
+
+
+def entropy_pack(mask: np.ndarray, dense_codes: np.ndarray, n: int, m: int) -> np.ndarray:
+    """Rows of group words from the keep mask and the dense codes [rows, K]."""
+    rows, k = mask.shape
+    bits = entropy_group_bits(n, m)
+    out = np.zeros((rows, entropy_row_bytes(k, n, m)), np.uint8)
+    for r in range(rows):
+        stream = 0
+        for g in range(k // m):
+            offs = [j for j in range(m) if mask[r, g * m + j]]
+            if len(offs) != n:
+                raise ValueError("a group does not keep exactly n positions")
+            word = colex_rank(offs) * 3 ** n
+            for i, j in enumerate(offs):
+                word += (int(dense_codes[r, g * m + j]) + 1) * 3 ** i
+            stream |= word << (g * bits)
+        nbytes = (k // m * bits + 7) // 8
+        out[r, :nbytes] = np.frombuffer(stream.to_bytes(nbytes, "little"), np.uint8)
+    return out
+
+
+def entropy_unpack(packed: np.ndarray, k: int, n: int, m: int):
+    """Inverse of entropy_pack: (dense codes int8 [rows, K], keep mask)."""
+    rows = packed.shape[0]
+    bits = entropy_group_bits(n, m)
+    dense = np.zeros((rows, k), np.int8)
+    mask = np.zeros((rows, k), bool)
+    for r in range(rows):
+        stream = int.from_bytes(bytes(packed[r]), "little")
+        for g in range(k // m):
+            word = (stream >> (g * bits)) & ((1 << bits) - 1)
+            rank, v = divmod(word, 3 ** n)
+            for i, j in enumerate(colex_unrank(rank, n, m)):
+                mask[r, g * m + j] = True
+                dense[r, g * m + j] = (v // 3 ** i) % 3 - 1
+    return dense, mask

@@ -482,3 +482,47 @@ def check_layer_vs_float(impl, w_bits, x_bits, n, m):
     ref = xr @ wr.T
     noise = 1e-12 * float(np.abs(ref).max() + 1e-300)   # fp64 rounding of the float product
     assert np.all(np.abs(y - ref) <= np.abs(ref) * 2.0 ** -8 + noise)
+
+
+# ---- entropy-tight packed format -------------------------------------------
+
+def check_entropy_accounting(impl):
+    """'From 2:4 to 8:16 sparsity patterns ...', Abstract: the masks of 2:4 and
+    8:16 cost 0.75 and 0.875 bits per element, i.e. ceil(log2 C(m, n)) / m."""
+    assert impl.mask_index_bits(2, 4) / 4 == 0.75
+    assert impl.mask_index_bits(8, 16) / 16 == 0.875
+    for (n, m) in [(1, 4), (2, 4), (6, 8), (8, 16), (8, 8)]:
+        # a group word holds every (pattern, values) pair and no more bits than that needs
+        total = math.comb(m, n) * 3 ** n
+        assert (1 << impl.entropy_group_bits(n, m)) >= total
+        assert (1 << (impl.entropy_group_bits(n, m) - 1)) < total
+
+
+def check_entropy_hand(impl):
+    """The worked example of tests/golden/entropy_hand.txt (2:4, K = 8)."""
+    text = (Path(__file__).parent / "golden" / "entropy_hand.txt").read_text().splitlines()
+    rows = {ln.split(":")[0]: ln.split(":")[1].split() for ln in text if ln and not ln.startswith("#")}
+    dense = np.array([[int(v) for v in rows["codes"]]], np.int8)
+    mask = np.array([[v == "1" for v in rows["mask"]]])
+    want = [int(v, 16) for v in rows["bytes"]]
+    packed = impl.entropy_pack(mask, dense, 2, 4)
+    assert list(packed[0, :len(want)]) == want and not packed[0, len(want):].any()
+
+
+def check_entropy_bijection(impl, n=2, m=4):
+    """Every (keep pattern, kept values) of a group gets its own word below 2^bits."""
+    bits = impl.entropy_group_bits(n, m)
+    seen = set()
+    for offs in itertools.combinations(range(m), n):
+        for digits in itertools.product((-1, 0, 1), repeat=n):
+            mask = np.zeros((1, m), bool)
+            dense = np.zeros((1, m), np.int8)
+            for j, d in zip(offs, digits):
+                mask[0, j] = True
+                dense[0, j] = d
+            word = int.from_bytes(bytes(impl.entropy_pack(mask, dense, n, m)[0]), "little")
+            assert word < (1 << bits)
+            seen.add(word)
+            d2, m2 = impl.entropy_unpack(impl.entropy_pack(mask, dense, n, m), m, n, m)
+            assert np.array_equal(d2, dense) and np.array_equal(m2, mask)
+    assert len(seen) == math.comb(m, n) * 3 ** n

@@ -1,5 +1,8 @@
 """The CPU oracle against its pins (no GPU)."""
 
+import math
+from pathlib import Path
+
 import numpy as np
 import pytest
 
@@ -158,3 +161,63 @@ def test_mask_flips_complement_within_2of4_groups():
     a, b = oracle.nm_mask(w1, 2, 4), oracle.nm_mask(w2, 2, 4)
     assert oracle.mask_flips(a, b) == a.size
     assert oracle.mask_flip_rate(a, b) == 1.0
+
+
+# ---- entropy-tight packed format ---------------------------------------------
+
+def test_mask_index_bits_match_the_pages_accounting():
+    # "From 2:4 to 8:16 sparsity patterns ...", Abstract: 0.75 vs 0.875 bits/element
+    assert oracle.mask_index_bits(2, 4) / 4 == 0.75
+    assert oracle.mask_index_bits(8, 16) / 16 == 0.875
+    assert oracle.entropy_group_bits(6, 8) == 15           # 28 * 729 = 20412 < 2^15
+
+
+def testcolex_rank_order_for_2of4():
+    order = [(0, 1), (0, 2), (1, 2), (0, 3), (1, 3), (2, 3)]
+    for r, offs in enumerate(order):
+        assert oracle.colex_rank(list(offs)) == r
+        assert oracle.colex_unrank(r, 2, 4) == list(offs)
+
+
+@pytest.mark.parametrize("nm", [(1, 4), (2, 4), (3, 4), (4, 4), (2, 8), (6, 8)])
+def test_entropy_words_are_a_bijection(nm):
+    import itertools
+    n, m = nm
+    bits = oracle.entropy_group_bits(n, m)
+    seen = set()
+    for offs in itertools.combinations(range(m), n):
+        for digits in itertools.product((-1, 0, 1), repeat=n):
+            mask = np.zeros((1, m), bool)
+            dense = np.zeros((1, m), np.int8)
+            for j, d in zip(offs, digits):
+                mask[0, j] = True
+                dense[0, j] = d
+            packed = oracle.entropy_pack(mask, dense, n, m)
+            word = int.from_bytes(bytes(packed[0]), "little")
+            assert word < (1 << bits)
+            seen.add(word)
+            d2, m2 = oracle.entropy_unpack(packed, m, n, m)
+            assert np.array_equal(d2, dense) and np.array_equal(m2, mask)
+    assert len(seen) == math.comb(m, n) * 3 ** n
+
+
+def test_entropy_hand_example():
+    text = (Path(__file__).parent / "golden" / "entropy_hand.txt").read_text().splitlines()
+    rows = {ln.split(":")[0]: ln.split(":")[1].split() for ln in text if ln and not ln.startswith("#")}
+    dense = np.array([[int(v) for v in rows["codes"]]], np.int8)
+    mask = np.array([[v == "1" for v in rows["mask"]]])
+    want = [int(v, 16) for v in rows["bytes"]]
+    packed = oracle.entropy_pack(mask, dense, 2, 4)
+    assert list(packed[0, :len(want)]) == want and not packed[0, len(want):].any()
+    assert packed.shape[1] == 16
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (4, 8), (8, 8), (12, 16)])
+def test_entropy_round_trip_on_quantized_layers(nm):
+    n, m = nm
+    w = synth.latent_weights(9, 256, seed=41, tag=f"ent{nm}")
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, n, m)
+    packed = oracle.entropy_pack(mask, dense, n, m)
+    assert packed.shape == (9, oracle.entropy_row_bytes(256, n, m))
+    d2, m2 = oracle.entropy_unpack(packed, 256, n, m)
+    assert np.array_equal(d2, dense) and np.array_equal(m2, mask)

@@ -178,6 +178,32 @@ def dequant_truncate(acc, s, gamma):
     return (np.asarray(y, np.float32).view(np.uint32) >> 16).astype(np.uint16)
 
 
+def _entropy_pack_with(rank_fn=None, digit_order=1, bits_fn=None):
+    """entropy_pack with one step replaced (for the mutants below)."""
+    def pack(mask, dense, n, m):
+        rows, k = mask.shape
+        bits = (bits_fn or O.entropy_group_bits)(n, m)
+        out = np.zeros((rows, O.entropy_row_bytes(k, n, m)), np.uint8)
+        for r in range(rows):
+            stream = 0
+            for g in range(k // m):
+                offs = [j for j in range(m) if mask[r, g * m + j]]
+                word = (rank_fn or O.colex_rank)(offs) * 3 ** n
+                for i, j in enumerate(offs[::digit_order]):
+                    word += (int(dense[r, g * m + j]) + 1) * 3 ** i
+                stream |= word << (g * bits)
+            nbytes = (k // m * bits + 7) // 8
+            out[r, :nbytes] = np.frombuffer(stream.to_bytes(nbytes, "little"), np.uint8)
+        return out
+    return pack
+
+
+def _lex_rank(offs):
+    import itertools as it
+    m = 4 if max(offs, default=0) < 4 else 16
+    return list(it.combinations(range(m), len(offs))).index(tuple(offs))
+
+
 MUTANTS = {
     "gamma_no_subnormal": dict(absmean_gamma=gamma_no_subnormal, gamma_bins=bins_no_subnormal),
     "gamma_exponent_off_by_one": dict(absmean_gamma=gamma_exponent_off_by_one),
@@ -202,6 +228,9 @@ MUTANTS = {
     "acc_dropped_last_k": dict(bitlinear_acc=acc_dropped_last_k),
     "dequant_no_s": dict(dequant_bf16=dequant_no_s),
     "dequant_truncate": dict(dequant_bf16=dequant_truncate),
+    "entropy_lex_rank": dict(entropy_pack=_entropy_pack_with(rank_fn=_lex_rank)),
+    "entropy_digits_msb_first": dict(entropy_pack=_entropy_pack_with(digit_order=-1)),
+    "entropy_bits_undersized": dict(entropy_group_bits=lambda n, m: O.entropy_group_bits(n, m) - 1),
 }
 
 
@@ -231,6 +260,9 @@ def all_pins(impl):
         ("acc_extremes", lambda: pins.check_acc_extremes(impl)),
         ("dequant", lambda: pins.check_dequant(impl)),
         ("layer", lambda: pins.check_layer_vs_float(impl, small["w"], small["x"], 2, 4)),
+        ("entropy_accounting", lambda: pins.check_entropy_accounting(impl)),
+        ("entropy_hand", lambda: pins.check_entropy_hand(impl)),
+        ("entropy_bijection", lambda: pins.check_entropy_bijection(impl)),
     ]
     failed = []
     for name, fn in checks:
