@@ -2,7 +2,7 @@
 """Benchmark of the Sparse-BitNet BitLinear forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill]
+                    [--workload decode|prefill|decode_entropy]
 
 One step is one pass of the whole path over one batch of synthetic input:
 sbn_quantize_weights on the latent weights (the dynamic N:M mask is
@@ -11,8 +11,10 @@ quantization and the contraction: sbn_bitlinear_x (fused) for the decode
 workload, sbn_quantize_acts + sbn_bitlinear for prefill. The default workload
 is the decode GEMV sweep: W [6912, 2560] bf16 ~ N(0, 0.02), 6:8, activations
 of T = 1, 4 and 16 tokens. The prefill workload is T = 4096 through
-(K, N_out) = (2560, 6912) and (6912, 2560) at 2:4. The other shapes of the
-pages' workloads are covered by the parity tests.
+(K, N_out) = (2560, 6912) and (6912, 2560) at 2:4. decode_entropy is the
+decode sweep over the entropy-tight weight format (sbn_pack_entropy +
+sbn_bitlinear_entropy). The other shapes of the pages' workloads are
+covered by the parity tests.
 
 Timing: each step is a captured CUDA graph; steps rotate over enough
 distinct copies of the inputs and outputs that their total exceeds 3x the
@@ -86,6 +88,22 @@ def blx_bytes(t, k, n_out, n, m):
     return 2 * t * k + packed_bytes(n_out, k, n, m) + 4 + 2 * t * n_out
 
 
+def entropy_bytes(n_out, k, n, m):
+    """Entropy-tight packed weights (one word of ceil(log2(C(m,n) 3^n)) bits per group)."""
+    bits = (math.comb(m, n) * 3 ** n - 1).bit_length()
+    return n_out * ((((k // m) * bits + 7) // 8 + 15) // 16 * 16)
+
+
+def pe_bytes(n_out, k, n, m):
+    """sbn_pack_entropy: canonical packed weights read, entropy-tight written."""
+    return packed_bytes(n_out, k, n, m) + entropy_bytes(n_out, k, n, m)
+
+
+def ble_bytes(t, k, n_out, n, m):
+    """sbn_bitlinear_entropy: entropy-tight W + Xq + scales + gamma + bf16 Y."""
+    return entropy_bytes(n_out, k, n, m) + t * k + 4 * t + 4 + 2 * t * n_out
+
+
 def bl_ops(t, k, n_out, n, m):
     """Algorithmic ops (2 per kept multiply-add)."""
     return 2 * t * k * n_out * n // m
@@ -97,25 +115,34 @@ WORKLOADS = {
                         "algorithmic bytes of the step / step time; activation quantization "
                         "fused into the contraction (sbn_bitlinear_x)",
                    unit="GB/s", fused=True, layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
+    "decode_entropy": dict(desc="decode GEMV sweep over entropy-tight weights: K=2560, N_out=6912, "
+                                "6:8, T in {1,4,16}; each step packs the quantized layer into the "
+                                "entropy-tight format (1.875 bit/weight) and contracts from it",
+                           unit="GB/s", mode="entropy", layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
     "prefill": dict(desc="prefill GEMM: T=4096, (K,N_out)=(2560,6912) and (6912,2560), 2:4; value = "
                          "algorithmic ops (2 per kept multiply-add) of the step / step time",
                     unit="TOPS", layers=[(6912, 2560, 2, 4, [4096]), (2560, 6912, 2, 4, [4096])]),
 }
 
 
-def act_bytes(t, k, n_out, n, m, fused):
-    """Bytes of one token set after the weights are packed."""
-    if fused:
+def act_bytes(t, k, n_out, n, m, mode):
+    """Bytes of one token set after the weights are packed (mode: True or
+    "fused", False or "split", "entropy")."""
+    if mode is True or mode == "fused":
         return blx_bytes(t, k, n_out, n, m)
+    if mode == "entropy":
+        return qa_bytes(t, k) + ble_bytes(t, k, n_out, n, m)
     return qa_bytes(t, k) + bl_bytes(t, k, n_out, n, m)
 
 
-def step_bytes(layers, fused=False):
+def step_bytes(layers, mode=False):
     b = 0
     for (n_out, k, n, m, ts) in layers:
         b += qw_bytes(n_out, k, n, m)
+        if mode == "entropy":
+            b += pe_bytes(n_out, k, n, m)
         for t in ts:
-            b += act_bytes(t, k, n_out, n, m, fused)
+            b += act_bytes(t, k, n_out, n, m, mode)
     return b
 
 
@@ -136,6 +163,12 @@ def is_fused(workload: str) -> bool:
     return bool(WORKLOADS[workload].get("fused", False))
 
 
+def workload_mode(workload: str):
+    """"fused", "entropy" or "split" (quantize_acts + bitlinear)."""
+    w = WORKLOADS[workload]
+    return w.get("mode", "fused" if w.get("fused") else "split")
+
+
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's time: every rank contributes its own and gets the max."""
     if world <= 1:
@@ -153,7 +186,7 @@ def whole_job_value(workload: str, steps: int, world: int, ms_max: float) -> flo
     layers = WORKLOADS[workload]["layers"]
     if WORKLOADS[workload]["unit"] == "TOPS":
         return step_ops(layers) * steps * world / (ms_max * 1e-3) / 1e12
-    return step_bytes(layers, is_fused(workload)) * steps * world / (ms_max * 1e-3) / 1e9
+    return step_bytes(layers, workload_mode(workload)) * steps * world / (ms_max * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -171,17 +204,30 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def kernel_source_sha():
+# device sources each call's kernels are built from: a recorded DRAM figure
+# stays valid while these files are unchanged
+TRAFFIC_FILES = {
+    "quantize_weights": ["qw_fused.cuh", "qw.cuh", "async.cuh", "common.cuh"],
+    "bitlinear_x": ["bl_decode_res.cuh", "bl_decode.cuh", "expand.cuh", "qa.cuh", "common.cuh"],
+    "bitlinear": ["bl_tc.cuh", "expand_dense.cuh", "expand.cuh", "async.cuh", "common.cuh"],
+    "bitlinear_entropy": ["bl_decode_ent.cuh", "bl_decode_res.cuh", "bl_decode.cuh", "entropy.cuh",
+                          "expand.cuh", "common.cuh"],
+}
+
+
+def kernel_source_sha(call=None):
+    """Hash of the device sources of a call's kernels (all of csrc/ if unknown)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_linear_layers_fwd_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files = TRAFFIC_FILES.get(call) or sorted(os.listdir(csrc))
+    for f in sorted(files):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel_key, workload):
-    """Per-launch DRAM bytes from a committed ncu summary, if the kernel
+    """Per-launch DRAM bytes from a committed ncu summary, if the call's kernel
     sources have not changed since it was captured; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -189,7 +235,7 @@ def ncu_traffic(kernel_key, workload):
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{kernel_key}@{workload}")
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(kernel_key):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -285,6 +331,8 @@ def oracle_sample_bytes(layers, rows_frac, fused=False):
         tot += qw_bytes(r, k, n, m)
         for t in ts:
             tot += act_bytes(t, k, r, n, m, fused)
+        if fused == "entropy":
+            tot += pe_bytes(r, k, n, m)
     return tot
 
 
@@ -296,7 +344,7 @@ def oracle_sample_metric(workload, layers, rows_frac):
             r = max(1, int(n_out * rows_frac))
             tot += sum(bl_ops(t, k, r, n, m) for t in ts)
         return tot / 1e12
-    return oracle_sample_bytes(layers, rows_frac, is_fused(workload)) / 1e9
+    return oracle_sample_bytes(layers, rows_frac, workload_mode(workload)) / 1e9
 
 
 def make_layers_data(workload, rank=0):
@@ -367,16 +415,24 @@ def run_ours(args, rank, world, local_rank):
                 (max(1, max(max(sbn.bitlinear_workspace_bytes(t, k, n_out),
                                 sbn.bitlinear_x_workspace_bytes(t, k, n_out)) for t in ts)),),
                 dtype=torch.uint8, device=dev))
-            sl.append(dict(w=wd, xs=xds, pw=pw, ws=ws, bws=bws, qs=qs, ys=ys, n=n, m=m))
+            ent = (torch.empty((n_out, sbn.entropy_row_bytes(k, n, m)), dtype=torch.uint8, device=dev)
+                   if workload_mode(args.workload) == "entropy" else None)
+            sl.append(dict(w=wd, xs=xds, pw=pw, ws=ws, bws=bws, qs=qs, ys=ys, n=n, m=m, ent=ent))
         slots.append(sl)
 
     # per-call events inside each slot's graph: names of the calls in order
     fused = is_fused(args.workload)
+    mode = workload_mode(args.workload)
     call_names = []
     for li, (n_out, k, n, m, ts) in enumerate(layers):
         call_names.append(("quantize_weights", li, None))
+        if mode == "entropy":
+            call_names.append(("pack_entropy", li, None))
         for t in ts:
-            if fused:
+            if mode == "entropy":
+                call_names.append(("quantize_acts", li, t))
+                call_names.append(("bitlinear_entropy", li, t))
+            elif fused:
                 call_names.append(("bitlinear_x", li, t))
             else:
                 call_names.append(("quantize_acts", li, t))
@@ -389,7 +445,22 @@ def run_ours(args, rank, world, local_rank):
             sbn.quantize_weights(L["w"], L["n"], L["m"], out=L["pw"], workspace=L["ws"], stream=stream)
             if evs and evs[i]: evs[i][1].record(stream)
             i += 1
+            if mode == "entropy":
+                if evs and evs[i]: evs[i][0].record(stream)
+                sbn.pack_entropy(L["pw"], out=L["ent"], stream=stream)
+                if evs and evs[i]: evs[i][1].record(stream)
+                i += 1
             for x, (q, s), y in zip(L["xs"], L["qs"], L["ys"]):
+                if mode == "entropy":
+                    if evs and evs[i]: evs[i][0].record(stream)
+                    sbn.quantize_acts(x, out_q=q, out_s=s, stream=stream)
+                    if evs and evs[i]: evs[i][1].record(stream)
+                    i += 1
+                    if evs and evs[i]: evs[i][0].record(stream)
+                    sbn.bitlinear_entropy(q, s, L["ent"], L["pw"], out=y, stream=stream)
+                    if evs and evs[i]: evs[i][1].record(stream)
+                    i += 1
+                    continue
                 if fused:
                     if evs and evs[i]: evs[i][0].record(stream)
                     sbn.bitlinear_x(x, L["pw"], out=y, workspace=L["bws"], stream=stream)
@@ -427,8 +498,11 @@ def run_ours(args, rank, world, local_rank):
     # our kernels per step: quantize_weights 1 per layer; quantize_acts 1 and
     # bitlinear 1 (+1 weight expansion when T > 16) per token set
     # (fused: one kernel per token set for T <= 16)
-    launches_per_step = sum(1 + sum((1 if fused and t <= 16 else 2 + (1 if t > 16 else 0))
-                                    for t in ts)
+    # (entropy: + 1 pack per layer, then quantize_acts + the entropy contraction)
+    launches_per_step = sum(1 + (1 if mode == "entropy" else 0)
+                            + sum((2 if mode == "entropy" else
+                                   1 if fused and t <= 16 else 2 + (1 if t > 16 else 0))
+                                  for t in ts)
                             for (_, _, _, _, ts) in layers)
 
     def barrier():
@@ -485,7 +559,7 @@ def run_ours(args, rank, world, local_rank):
 
     ms = max_over_ranks(ms, world, dev)
 
-    sb = step_bytes(layers, fused)
+    sb = step_bytes(layers, mode)
     ms_per_step = ms / args.steps
     value = whole_job_value(args.workload, args.steps, world, ms)
 
@@ -519,6 +593,10 @@ def run_ours(args, rank, world, local_rank):
             dom_bytes = sum(qa_bytes(t, k) for (n_out, k, n, m, ts) in layers for t in ts)
         elif dom == "bitlinear_x":
             dom_bytes = sum(blx_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
+        elif dom == "bitlinear_entropy":
+            dom_bytes = sum(ble_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
+        elif dom == "pack_entropy":
+            dom_bytes = sum(pe_bytes(n_out, k, n, m) for (n_out, k, n, m, ts) in layers)
         else:
             dom_bytes = sum(bl_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
         achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -540,12 +618,17 @@ def run_ours(args, rank, world, local_rank):
             b = qa_bytes(t, k)
         elif name == "bitlinear_x":
             b = blx_bytes(t, k, n_out, n, m)
+        elif name == "bitlinear_entropy":
+            b = ble_bytes(t, k, n_out, n, m)
+        elif name == "pack_entropy":
+            b = pe_bytes(n_out, k, n, m)
         else:
             b = bl_bytes(t, k, n_out, n, m)
         e = {"us": round(us, 3), "GB/s": round(b / (us * 1e-6) / 1e9, 1),
              "hbm_frac": round(b / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
-        if name in ("bitlinear", "bitlinear_x"):
-            e["weight_GB/s"] = round(packed_bytes(n_out, k, n, m) / (us * 1e-6) / 1e9, 1)
+        if name in ("bitlinear", "bitlinear_x", "bitlinear_entropy"):
+            wb = entropy_bytes(n_out, k, n, m) if name == "bitlinear_entropy" else packed_bytes(n_out, k, n, m)
+            e["weight_GB/s"] = round(wb / (us * 1e-6) / 1e9, 1)
             ops = bl_ops(t, k, n_out, n, m)
             e["TOPS"] = round(ops / (us * 1e-6) / 1e12, 3)
             e["dense_eq_TOPS"] = round(2 * t * k * n_out / (us * 1e-6) / 1e12, 3)
@@ -610,14 +693,19 @@ def run_e2e(args, data, layers, dev, stream, world):
     pws = [sbn.alloc_packed(h[0].shape[0], h[0].shape[1], h[2], h[3], dev) for h in host]
 
     fused = is_fused(args.workload)
+    mode = workload_mode(args.workload)
 
     def step():
         for li, (hw, hxs, n, m) in enumerate(host):
             dw[li].copy_(hw, non_blocking=True)
             sbn.quantize_weights(dw[li], n, m, out=pws[li], workspace=ws[li], stream=stream)
+            ent = sbn.pack_entropy(pws[li], stream=stream) if mode == "entropy" else None
             for j, hx in enumerate(hxs):
                 dxs[li][j].copy_(hx, non_blocking=True)
-                if fused:
+                if mode == "entropy":
+                    q, s = sbn.quantize_acts(dxs[li][j], stream=stream)
+                    y = sbn.bitlinear_entropy(q, s, ent, pws[li], stream=stream)
+                elif fused:
                     y = sbn.bitlinear_x(dxs[li][j], pws[li], stream=stream)
                 else:
                     q, s = sbn.quantize_acts(dxs[li][j], stream=stream)
@@ -676,7 +764,7 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, bf16 io",
         "data": "synthetic (seeded: W ~ N(0,0.02) bf16, X ~ N(0,1) bf16)",
         "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]["desc"],
-                   "bytes_per_step": step_bytes(layers, is_fused(args.workload)),
+                   "bytes_per_step": step_bytes(layers, workload_mode(args.workload)),
                    "tokens_per_step": step_tokens(layers)},
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores_used(),
                          "kind": "oracle",

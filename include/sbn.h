@@ -262,6 +262,55 @@ sbn_status sbn_mask_flips(const uint8_t* meta_a, const uint8_t* meta_b,
                           unsigned long long* flips, void* stream);
 
 /*
+ * Entropy-tight packed weights (the pages have no such format; the size of
+ * its keep-pattern part follows "From 2:4 to 8:16 sparsity patterns in LLMs
+ * for Outliers and Weights with Variance Correction", Abstract: 0.75 and
+ * 0.875 bits per element for the 2:4 and 8:16 masks, i.e. ceil(log2 C(m, n))
+ * / m, an index over the keep patterns of a group).
+ *
+ * Per group of m positions one word
+ *     word = rank * 3^n + sum_i (code_i + 1) * 3^i
+ * in ceil(log2(C(m, n) * 3^n)) bits, where rank = sum_i C(c_i, i) for the
+ * kept offsets c_1 < ... < c_n (combinatorial number system, colex order)
+ * and code_i are the kept ternary codes in ascending position. Words are
+ * concatenated little-endian per row (bit b is bit b % 8 of byte b / 8);
+ * rows are padded with zero bytes to a multiple of 16. 6:8 takes 15 bits per
+ * 8 weights (1.875 bits/weight) instead of 2.5.
+ */
+size_t sbn_entropy_row_bytes(int32_t k, int32_t n, int32_t m);
+size_t sbn_entropy_bytes(int32_t n_out, int32_t k, int32_t n, int32_t m);
+
+/*
+ * sbn_pack_entropy -- the canonical packed weights (codes, meta) of a layer,
+ * as written by sbn_quantize_weights, into the entropy-tight format.
+ *   ent   device, [n_out, sbn_entropy_row_bytes(k, n, m)], written.
+ * Every supported pattern. Errors: SBN_ERR_NULL, SBN_ERR_SHAPE,
+ * SBN_ERR_PATTERN, SBN_ERR_ALIGN; SBN_ERR_CUDA.
+ */
+sbn_status sbn_pack_entropy(const uint8_t* codes, const uint8_t* meta,
+                            int32_t n_out, int32_t k, int32_t n, int32_t m,
+                            uint8_t* ent, void* stream);
+
+/*
+ * sbn_bitlinear_entropy -- the decode contraction (1 <= t <= 16) reading
+ * the entropy-tight weights: the same y as sbn_bitlinear on the canonical
+ * weights, bit for bit. Patterns with m = 4 or 8 and n < m; other patterns
+ * give SBN_ERR_PATTERN, t > 16 or rows that do not fit in shared memory
+ * SBN_ERR_SHAPE. Other arguments and errors as sbn_bitlinear.
+ */
+sbn_status sbn_bitlinear_entropy(const int8_t* xq, const float* x_scale,
+                                 int32_t t, int32_t k, int32_t n_out,
+                                 int32_t n, int32_t m, const uint8_t* ent,
+                                 const float* gamma, void* y_bf16,
+                                 void* stream);
+
+/* The same contraction writing the exact int32 accumulators (verification). */
+sbn_status sbn_bitlinear_entropy_acc32(const int8_t* xq, int32_t t,
+                                       int32_t k, int32_t n_out, int32_t n,
+                                       int32_t m, const uint8_t* ent,
+                                       int32_t* acc, void* stream);
+
+/*
  * sbn_get_device_error -- synchronizes `stream`, then reads and clears the
  * device error word of the current device. Returns SBN_OK, SBN_ERR_TIMEOUT
  * (a bounded device wait gave up; the affected outputs are unspecified) or

@@ -18,7 +18,9 @@
 #include "qw_fused.cuh"
 #include "bl_decode.cuh"
 #include "bl_decode_res.cuh"
+#include "bl_decode_ent.cuh"
 #include "expand_dense.cuh"
+#include "entropy.cuh"
 #include "flip.cuh"
 #include "bl_tc.cuh"
 
@@ -209,6 +211,42 @@ sbn_status dispatch_decode_res(const DresParams& p, int n, int m, int grid, size
     case 16 * 8 + 1: return launch_decode_res<16, 1, NT, false, ACC, XBF>(p, grid, smem, st);
     case 16 * 8 + 2: return launch_decode_res<16, 2, NT, false, ACC, XBF>(p, grid, smem, st);
     case 16 * 8 + 3: return launch_decode_res<16, 3, NT, false, ACC, XBF>(p, grid, smem, st);
+  }
+  return SBN_ERR_PATTERN;
+}
+
+// Decode contraction over entropy-tight weights (patterns with m = 4 or 8).
+template <int MM, int CB, int NT, bool ACC>
+sbn_status launch_decode_ent(const DresParams& p, int grid, size_t smem, cudaStream_t st) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  auto kern = bl_decode_ent_kernel<MM, CB, NT, ACC>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDresSmemMax) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  kern<<<grid, kDresThreads, smem, st>>>(p);
+  return launch_status();
+}
+
+template <int NT, bool ACC>
+sbn_status dispatch_decode_ent(const DresParams& p, int n, int m, int grid, size_t smem,
+                               cudaStream_t st) {
+  switch (m * 8 + 4 * n / m) {
+    case 4 * 8 + 1: return launch_decode_ent<4, 1, NT, ACC>(p, grid, smem, st);
+    case 4 * 8 + 2: return launch_decode_ent<4, 2, NT, ACC>(p, grid, smem, st);
+    case 4 * 8 + 3: return launch_decode_ent<4, 3, NT, ACC>(p, grid, smem, st);
+    case 8 * 8 + 1: return launch_decode_ent<8, 1, NT, ACC>(p, grid, smem, st);
+    case 8 * 8 + 2: return launch_decode_ent<8, 2, NT, ACC>(p, grid, smem, st);
+    case 8 * 8 + 3: return launch_decode_ent<8, 3, NT, ACC>(p, grid, smem, st);
   }
   return SBN_ERR_PATTERN;
 }
@@ -446,6 +484,35 @@ sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, fl
   return launch_status();
 }
 
+template <bool ACC>
+sbn_status run_bitlinear_entropy(const int8_t* xq, const float* xs, int32_t t, int32_t k, int32_t n_out,
+                                 int32_t n, int32_t m, const uint8_t* ent, const float* gamma, uint16_t* y,
+                                 int32_t* acc, void* stream) {
+  if (!pattern_ok(n, m)) return SBN_ERR_PATTERN;
+  if (n == m || (m != 4 && m != 8)) return SBN_ERR_PATTERN;
+  if (t < 1 || t > 16 || n_out < 1 || k < 128 || (k % 128) != 0 || !prod_lt_2_31(n_out, k))
+    return SBN_ERR_SHAPE;
+  if (!aligned16(xq) || !aligned16(ent)) return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  const int estride = (int)entropy_row_bytes(k, n, m);
+  const int tiles = (n_out + 15) / 16;
+  const int grid = std::min(sms, tiles);
+  const int per_cta = (tiles + grid - 1) / grid;
+  const int nt = t <= 8 ? 8 : 16;
+  const DresLayout L = dres_layout(per_cta, nt, k, estride, 0, true);
+  const size_t smem = ent_smem_bytes(L);
+  if (per_cta > kDresMaxTiles || smem > kDresSmemMax) return SBN_ERR_SHAPE;
+  DresParams q;
+  q.xq = xq; q.xs = xs; q.xbf = nullptr; q.xq_out = nullptr; q.xs_out = nullptr;
+  q.codes = ent; q.meta = nullptr; q.gamma = gamma; q.y = y; q.acc_out = acc;
+  q.T = t; q.K = k; q.N = n_out; q.cstride = estride; q.mstride = 0; q.tiles_per_cta = per_cta;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  return t <= 8 ? dispatch_decode_ent<8, ACC>(q, n, m, grid, smem, cs)
+                : dispatch_decode_ent<16, ACC>(q, n, m, grid, smem, cs);
+}
+
 // Fixed scratch of sbn_quantize_weights_noalloc (see include/sbn.h).
 constexpr size_t kNoAllocScratchBytes = SBN_NOALLOC_SCRATCH_BYTES;
 static_assert(kQwWorkspaceBytes <= kNoAllocScratchBytes, "workspace exceeds the fixed scratch");
@@ -557,6 +624,60 @@ sbn_status sbn_mask_flips(const uint8_t* meta_a, const uint8_t* meta_b, int32_t 
   flip_count_kernel<<<grid, kFlipThreads, 0, cs>>>(reinterpret_cast<const uint4*>(meta_a),
                                                    reinterpret_cast<const uint4*>(meta_b), n16, flips);
   return launch_status();
+}
+
+size_t sbn_entropy_row_bytes(int32_t k, int32_t n, int32_t m) {
+  if (!pattern_ok(n, m) || k < 1 || (k % m) != 0) return 0;
+  return entropy_row_bytes(k, n, m);
+}
+
+size_t sbn_entropy_bytes(int32_t n_out, int32_t k, int32_t n, int32_t m) {
+  if (n_out < 1) return 0;
+  return (size_t)n_out * sbn_entropy_row_bytes(k, n, m);
+}
+
+sbn_status sbn_pack_entropy(const uint8_t* codes, const uint8_t* meta, int32_t n_out, int32_t k,
+                            int32_t n, int32_t m, uint8_t* ent, void* stream) {
+  if (!codes || !ent || (n != m && !meta)) return SBN_ERR_NULL;
+  sbn_status st = validate_weights_shape(n_out, k, n, m);
+  if (st != SBN_OK) return st;
+  if (!aligned16(codes) || !aligned16(ent) || (meta && !aligned16(meta))) return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const size_t ebytes = sbn_entropy_bytes(n_out, k, n, m);
+  if (cudaMemsetAsync(ent, 0, ebytes, cs) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
+  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
+  const int estride = (int)sbn_entropy_row_bytes(k, n, m);
+  const long long groups = (long long)n_out * (k / m);
+  const int grid = (int)std::max(1LL, std::min((groups + kEntThreads - 1) / kEntThreads, (long long)sms * 8));
+  uint32_t* e32 = reinterpret_cast<uint32_t*>(ent);
+  switch (m) {
+    case 4: entropy_pack_kernel<4><<<grid, kEntThreads, 0, cs>>>(codes, meta, n_out, k, n, cstride, mstride, e32, estride); break;
+    case 8: entropy_pack_kernel<8><<<grid, kEntThreads, 0, cs>>>(codes, meta, n_out, k, n, cstride, mstride, e32, estride); break;
+    default: entropy_pack_kernel<16><<<grid, kEntThreads, 0, cs>>>(codes, meta, n_out, k, n, cstride, mstride, e32, estride); break;
+  }
+  return launch_status();
+}
+
+sbn_status sbn_bitlinear_entropy(const int8_t* xq, const float* x_scale, int32_t t, int32_t k,
+                                 int32_t n_out, int32_t n, int32_t m, const uint8_t* ent,
+                                 const float* gamma, void* y_bf16, void* stream) {
+  if (!xq || !x_scale || !ent || !gamma || !y_bf16) return SBN_ERR_NULL;
+  if (!aligned16(y_bf16)) return SBN_ERR_ALIGN;
+  return run_bitlinear_entropy<false>(xq, x_scale, t, k, n_out, n, m, ent, gamma,
+                                      reinterpret_cast<uint16_t*>(y_bf16), nullptr, stream);
+}
+
+sbn_status sbn_bitlinear_entropy_acc32(const int8_t* xq, int32_t t, int32_t k, int32_t n_out, int32_t n,
+                                       int32_t m, const uint8_t* ent, int32_t* acc, void* stream) {
+  if (!xq || !ent || !acc) return SBN_ERR_NULL;
+  if (!aligned16(acc)) return SBN_ERR_ALIGN;
+  return run_bitlinear_entropy<true>(xq, nullptr, t, k, n_out, n, m, ent, nullptr, nullptr, acc, stream);
 }
 
 size_t sbn_bitlinear_x_workspace_bytes(int32_t t, int32_t k, int32_t n_out) {

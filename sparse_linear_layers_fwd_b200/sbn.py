@@ -52,6 +52,13 @@ PROTOTYPES = {
                                        _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "sbn_bitlinear_x_workspace_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32]),
     "sbn_mask_flips": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p]),
+    "sbn_entropy_row_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32]),
+    "sbn_entropy_bytes": (_c_sz, [_c_i32, _c_i32, _c_i32, _c_i32]),
+    "sbn_pack_entropy": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p]),
+    "sbn_bitlinear_entropy": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
+                                             _c_p, _c_p, _c_p, _c_p]),
+    "sbn_bitlinear_entropy_acc32": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
+                                                   _c_p, _c_p, _c_p]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
 
@@ -273,6 +280,48 @@ def mask_flips(a: PackedWeights, b: PackedWeights, out: Optional[torch.Tensor] =
     st = lib().sbn_mask_flips(_ptr(a.meta), _ptr(b.meta), a.n_out, a.k, a.n, a.m, _ptr(out),
                               _stream_ptr(stream))
     _check(st, "sbn_mask_flips")
+    return out
+
+
+def entropy_row_bytes(k: int, n: int, m: int) -> int:
+    return int(lib().sbn_entropy_row_bytes(k, n, m))
+
+
+def pack_entropy(w: PackedWeights, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """sbn_pack_entropy: the entropy-tight format [N_out, entropy_row_bytes] (uint8)."""
+    if out is None:
+        out = torch.empty((w.n_out, entropy_row_bytes(w.k, w.n, w.m)), dtype=torch.uint8,
+                          device=w.codes.device)
+    st = lib().sbn_pack_entropy(_ptr(w.codes), _ptr(w.meta), w.n_out, w.k, w.n, w.m, _ptr(out),
+                                _stream_ptr(stream))
+    _check(st, "sbn_pack_entropy")
+    return out
+
+
+def bitlinear_entropy(xq: torch.Tensor, s: torch.Tensor, ent: torch.Tensor, w: PackedWeights,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """sbn_bitlinear_entropy: decode contraction over entropy-tight weights
+    (shape, pattern and gamma from the PackedWeights they were packed from)."""
+    _need(xq, torch.int8, "xq")
+    _need(s, torch.float32, "s")
+    t, k = xq.shape
+    if out is None:
+        out = torch.empty((t, w.n_out), dtype=torch.bfloat16, device=xq.device)
+    st = lib().sbn_bitlinear_entropy(_ptr(xq), _ptr(s), t, k, w.n_out, w.n, w.m, _ptr(ent),
+                                     _ptr(w.gamma), _ptr(out), _stream_ptr(stream))
+    _check(st, "sbn_bitlinear_entropy")
+    return out
+
+
+def bitlinear_entropy_acc32(xq: torch.Tensor, ent: torch.Tensor, w: PackedWeights,
+                            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _need(xq, torch.int8, "xq")
+    t, k = xq.shape
+    if out is None:
+        out = torch.empty((t, w.n_out), dtype=torch.int32, device=xq.device)
+    st = lib().sbn_bitlinear_entropy_acc32(_ptr(xq), t, k, w.n_out, w.n, w.m, _ptr(ent), _ptr(out),
+                                           _stream_ptr(stream))
+    _check(st, "sbn_bitlinear_entropy_acc32")
     return out
 
 

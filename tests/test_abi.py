@@ -151,6 +151,23 @@ def test_mask_flips_validation(sbn_lib):
     assert lib.sbn_mask_flips(A, A, 8, 256, 2, 4, A + 4, None) == 4
 
 
+def test_entropy_validation(sbn_lib):
+    lib = sbn_lib
+    assert lib.sbn_pack_entropy(None, A, 8, 256, 2, 4, A, None) == 1
+    assert lib.sbn_pack_entropy(A, None, 8, 256, 2, 4, A, None) == 1
+    assert lib.sbn_pack_entropy(A, None, 8, 256, 4, 4, A, None) != 1     # dense: no meta
+    assert lib.sbn_pack_entropy(A, A, 8, 100, 2, 4, A, None) == 2
+    assert lib.sbn_pack_entropy(A, A, 8, 256, 2, 4, MIS, None) == 4
+    bl = lib.sbn_bitlinear_entropy
+    assert bl(None, A, 4, 256, 64, 2, 4, A, A, A, None) == 1
+    assert bl(A, A, 4, 256, 64, 8, 16, A, A, A, None) == 3                # m = 16: not decoded
+    assert bl(A, A, 4, 256, 64, 8, 8, A, A, A, None) == 3                 # dense
+    assert bl(A, A, 17, 256, 64, 2, 4, A, A, A, None) == 2                # decode only
+    assert bl(A, A, 4, 256, 64, 2, 4, MIS, A, A, None) == 4
+    assert lib.sbn_bitlinear_entropy_acc32(A, 4, 256, 64, 2, 4, A, None, None) == 1
+    assert lib.sbn_entropy_row_bytes(2560, 6, 8) == 608                   # 320 x 15 bits -> 600 B
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")
 def test_valid_arguments_without_gpu_fail_cleanly(sbn_lib):
     # every argument is valid, so the call reaches the device check and stops there

@@ -337,3 +337,51 @@ def test_mask_flips(nm, shape):
     got = int(sbn.mask_flips(p1, p2).cpu().item())
     assert got == oracle.mask_flips(oracle.nm_mask(w1, *nm), oracle.nm_mask(w2, *nm))
     assert int(sbn.mask_flips(p1, p1).cpu().item()) == 0
+
+
+ENT_DECODE = [(1, 4), (2, 4), (3, 4), (2, 8), (4, 8), (6, 8)]
+
+
+@pytest.mark.parametrize("nm", SUPPORTED)
+@pytest.mark.parametrize("shape", [(7, 128), (130, 1024), (257, 512)])
+def test_pack_entropy_matches_oracle(nm, shape):
+    n_out, k = shape
+    w = synth.latent_weights(n_out, k, seed=19, tag=f"entp{nm}{shape}")
+    from sparse_linear_layers_fwd_b200 import sbn
+    pw = run_quantize_weights(w, *nm)
+    got = sbn.pack_entropy(pw).cpu().numpy()
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, *nm)
+    assert np.array_equal(got, oracle.entropy_pack(mask, dense, *nm))
+
+
+def _entropy_decode_check(w, x, n, m):
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    pw = run_quantize_weights(w, n, m)
+    xq, s = sbn.quantize_acts(to_dev_bf16(x))
+    ent = sbn.pack_entropy(pw)
+    y_ent = sbn.bitlinear_entropy(xq, s, ent, pw)
+    acc_ent = sbn.bitlinear_entropy_acc32(xq, ent, pw)
+    y_can = sbn.bitlinear(xq, s, pw)
+    torch.cuda.synchronize()
+    assert sbn.get_device_error() == 0
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, n, m)
+    q, sc = oracle.quantize_acts(x)
+    acc = oracle.bitlinear_acc(q, dense)
+    assert np.array_equal(acc_ent.cpu().numpy(), acc)
+    assert np.array_equal(bf16_tensor_bits(y_ent), bf16_tensor_bits(y_can))
+    assert_y_close(bf16_tensor_bits(y_ent), oracle.dequant_bf16(acc, sc, gamma))
+
+
+@pytest.mark.parametrize("nm", ENT_DECODE)
+@pytest.mark.parametrize("shape", [(1, 128, 1), (5, 384, 7), (16, 1024, 130), (9, 512, 257)])
+def test_bitlinear_entropy(nm, shape):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=20, tag=f"entd{nm}{shape}")
+    x = synth.activations(t, k, seed=20, tag=f"entd{nm}{shape}", outlier_channels=2)
+    _entropy_decode_check(w, x, *nm)
+
+
+@pytest.mark.parametrize("t", synth.DECODE_TOKENS)
+def test_bitlinear_entropy_decode_full(t):
+    _entropy_decode_check(synth.decode_weights(), synth.decode_acts(t), 6, 8)
