@@ -46,11 +46,16 @@ constexpr int kEntThreads = 256;
 
 // Canonical packed weights (2-bit kept codes + keep bits) -> group words. One
 // thread per group; its word is OR-ed into the (zeroed) row stream, in at
-// most two 32-bit words.
+// most two 32-bit words. (i + 1 <= n <= 16 and pos < 16 keep the binomial
+// table index in range.)
 template <int M>
 __global__ void __launch_bounds__(kEntThreads)
 entropy_pack_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, int n_out,
                     int k, int n, int cstride, int mstride, uint32_t* __restrict__ ent, int estride) {
+  // binomials C(a, b), a, b <= 16, from a table instead of a division loop
+  __shared__ uint32_t s_binom[17 * 17];
+  for (int i = threadIdx.x; i < 17 * 17; i += kEntThreads) s_binom[i] = binom_u32(i / 17, i % 17);
+  __syncthreads();
   const int groups = k / M;
   const int bits = entropy_group_bits(n, M);
   const long long total = (long long)n_out * groups;
@@ -81,7 +86,7 @@ entropy_pack_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     int i = 0;
     for (int pos = 0; pos < M; ++pos) {
       if (!((keep >> pos) & 1u)) continue;
-      rank += binom_u32(pos, i + 1);
+      rank += s_binom[pos * 17 + i + 1];
       const uint32_t c2 = (uint32_t)(cw >> (2 * i)) & 3u;   // 00 -> 0, 01 -> +1, 11 -> -1
       const uint32_t digit = (c2 == 1u) ? 2u : (c2 == 3u ? 0u : 1u);
       v += digit * p3;
