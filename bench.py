@@ -13,7 +13,7 @@ is the decode GEMV sweep: W [6912, 2560] bf16 ~ N(0, 0.02), 6:8, activations
 of T = 1, 4 and 16 tokens. The prefill workload is T = 4096 through
 (K, N_out) = (2560, 6912) and (6912, 2560) at 2:4. decode_entropy is the
 decode sweep over the entropy-tight weight format (sbn_pack_entropy +
-sbn_bitlinear_entropy). The other shapes of the pages' workloads are
+sbn_bitlinear_entropy_x). The other shapes of the pages' workloads are
 covered by the parity tests.
 
 Timing: each step is a captured CUDA graph; steps rotate over enough
@@ -104,6 +104,12 @@ def ble_bytes(t, k, n_out, n, m):
     return entropy_bytes(n_out, k, n, m) + t * k + 4 * t + 4 + 2 * t * n_out
 
 
+def blex_bytes(t, k, n_out, n, m):
+    """sbn_bitlinear_entropy_x (act-quant fused): bf16 X + entropy-tight W +
+    gamma + bf16 Y."""
+    return 2 * t * k + entropy_bytes(n_out, k, n, m) + 4 + 2 * t * n_out
+
+
 def bl_ops(t, k, n_out, n, m):
     """Algorithmic ops (2 per kept multiply-add)."""
     return 2 * t * k * n_out * n // m
@@ -131,7 +137,7 @@ def act_bytes(t, k, n_out, n, m, mode):
     if mode is True or mode == "fused":
         return blx_bytes(t, k, n_out, n, m)
     if mode == "entropy":
-        return qa_bytes(t, k) + ble_bytes(t, k, n_out, n, m)
+        return blex_bytes(t, k, n_out, n, m)
     return qa_bytes(t, k) + bl_bytes(t, k, n_out, n, m)
 
 
@@ -212,6 +218,9 @@ TRAFFIC_FILES = {
     "bitlinear": ["bl_tc.cuh", "expand_dense.cuh", "expand.cuh", "async.cuh", "common.cuh"],
     "bitlinear_entropy": ["bl_decode_ent.cuh", "bl_decode_res.cuh", "bl_decode.cuh", "entropy.cuh",
                           "expand.cuh", "common.cuh"],
+    "bitlinear_entropy_x": ["bl_decode_ent.cuh", "bl_decode_res.cuh", "bl_decode.cuh", "entropy.cuh",
+                            "expand.cuh", "qa.cuh", "common.cuh"],
+    "pack_entropy": ["entropy_pack.cuh", "entropy.cuh", "common.cuh"],
 }
 
 
@@ -430,8 +439,7 @@ def run_ours(args, rank, world, local_rank):
             call_names.append(("pack_entropy", li, None))
         for t in ts:
             if mode == "entropy":
-                call_names.append(("quantize_acts", li, t))
-                call_names.append(("bitlinear_entropy", li, t))
+                call_names.append(("bitlinear_entropy_x", li, t))
             elif fused:
                 call_names.append(("bitlinear_x", li, t))
             else:
@@ -453,11 +461,7 @@ def run_ours(args, rank, world, local_rank):
             for x, (q, s), y in zip(L["xs"], L["qs"], L["ys"]):
                 if mode == "entropy":
                     if evs and evs[i]: evs[i][0].record(stream)
-                    sbn.quantize_acts(x, out_q=q, out_s=s, stream=stream)
-                    if evs and evs[i]: evs[i][1].record(stream)
-                    i += 1
-                    if evs and evs[i]: evs[i][0].record(stream)
-                    sbn.bitlinear_entropy(q, s, L["ent"], L["pw"], out=y, stream=stream)
+                    sbn.bitlinear_entropy_x(x, L["ent"], L["pw"], out=y, workspace=False, stream=stream)
                     if evs and evs[i]: evs[i][1].record(stream)
                     i += 1
                     continue
@@ -498,9 +502,9 @@ def run_ours(args, rank, world, local_rank):
     # our kernels per step: quantize_weights 1 per layer; quantize_acts 1 and
     # bitlinear 1 (+1 weight expansion when T > 16) per token set
     # (fused: one kernel per token set for T <= 16)
-    # (entropy: + 1 pack per layer, then quantize_acts + the entropy contraction)
+    # (entropy: + 1 pack per layer, then one fused entropy contraction per token set)
     launches_per_step = sum(1 + (1 if mode == "entropy" else 0)
-                            + sum((2 if mode == "entropy" else
+                            + sum((1 if mode == "entropy" else
                                    1 if fused and t <= 16 else 2 + (1 if t > 16 else 0))
                                   for t in ts)
                             for (_, _, _, _, ts) in layers)
@@ -595,6 +599,8 @@ def run_ours(args, rank, world, local_rank):
             dom_bytes = sum(blx_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
         elif dom == "bitlinear_entropy":
             dom_bytes = sum(ble_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
+        elif dom == "bitlinear_entropy_x":
+            dom_bytes = sum(blex_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
         elif dom == "pack_entropy":
             dom_bytes = sum(pe_bytes(n_out, k, n, m) for (n_out, k, n, m, ts) in layers)
         else:
@@ -620,14 +626,17 @@ def run_ours(args, rank, world, local_rank):
             b = blx_bytes(t, k, n_out, n, m)
         elif name == "bitlinear_entropy":
             b = ble_bytes(t, k, n_out, n, m)
+        elif name == "bitlinear_entropy_x":
+            b = blex_bytes(t, k, n_out, n, m)
         elif name == "pack_entropy":
             b = pe_bytes(n_out, k, n, m)
         else:
             b = bl_bytes(t, k, n_out, n, m)
         e = {"us": round(us, 3), "GB/s": round(b / (us * 1e-6) / 1e9, 1),
              "hbm_frac": round(b / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
-        if name in ("bitlinear", "bitlinear_x", "bitlinear_entropy"):
-            wb = entropy_bytes(n_out, k, n, m) if name == "bitlinear_entropy" else packed_bytes(n_out, k, n, m)
+        if name in ("bitlinear", "bitlinear_x", "bitlinear_entropy", "bitlinear_entropy_x"):
+            wb = (entropy_bytes(n_out, k, n, m) if name.startswith("bitlinear_entropy")
+                  else packed_bytes(n_out, k, n, m))
             e["weight_GB/s"] = round(wb / (us * 1e-6) / 1e9, 1)
             ops = bl_ops(t, k, n_out, n, m)
             e["TOPS"] = round(ops / (us * 1e-6) / 1e12, 3)
@@ -703,8 +712,7 @@ def run_e2e(args, data, layers, dev, stream, world):
             for j, hx in enumerate(hxs):
                 dxs[li][j].copy_(hx, non_blocking=True)
                 if mode == "entropy":
-                    q, s = sbn.quantize_acts(dxs[li][j], stream=stream)
-                    y = sbn.bitlinear_entropy(q, s, ent, pws[li], stream=stream)
+                    y = sbn.bitlinear_entropy_x(dxs[li][j], ent, pws[li], workspace=False, stream=stream)
                 elif fused:
                     y = sbn.bitlinear_x(dxs[li][j], pws[li], stream=stream)
                 else:

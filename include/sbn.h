@@ -311,6 +311,34 @@ sbn_status sbn_bitlinear_entropy_acc32(const int8_t* xq, int32_t t,
                                        int32_t* acc, void* stream);
 
 /*
+ * sbn_bitlinear_entropy_x -- sbn_quantize_acts fused into
+ * sbn_bitlinear_entropy: y from the bf16 activations x_bf16 [t, k]
+ * (device, 16-byte aligned), bit-identical to sbn_quantize_acts followed by
+ * sbn_bitlinear_entropy. Every CTA quantizes X itself (per-token absmax
+ * INT8, as sbn_quantize_acts) in its prologue.
+ *   xq, x_scale   optional (NULL for none) device outputs [t, k] int8 and
+ *                 [t] fp32: the INT8 activations and scales, bit-identical
+ *                 to sbn_quantize_acts.
+ *   workspace,    device scratch owned by the caller, 16-byte aligned, at
+ *   ws_bytes      least sbn_bitlinear_entropy_x_workspace_bytes(t, k) bytes;
+ *                 used only when the bf16 rows do not fit in shared memory
+ *                 and xq or x_scale is NULL (two-step route: quantize, then
+ *                 contract), else may be NULL. Contents unspecified after.
+ * Patterns and shapes as sbn_bitlinear_entropy. Errors: SBN_ERR_NULL,
+ * SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN, SBN_ERR_WORKSPACE (before
+ * anything is enqueued); SBN_ERR_CUDA.
+ */
+sbn_status sbn_bitlinear_entropy_x(const void* x_bf16, int32_t t, int32_t k,
+                                   int32_t n_out, int32_t n, int32_t m,
+                                   const uint8_t* ent, const float* gamma,
+                                   void* y_bf16, int8_t* xq, float* x_scale,
+                                   void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* Bytes of sbn_bitlinear_entropy_x's workspace (its two-step route). */
+size_t sbn_bitlinear_entropy_x_workspace_bytes(int32_t t, int32_t k);
+
+/*
  * sbn_get_device_error -- synchronizes `stream`, then reads and clears the
  * device error word of the current device. Returns SBN_OK, SBN_ERR_TIMEOUT
  * (a bounded device wait gave up; the affected outputs are unspecified) or

@@ -24,11 +24,12 @@ __host__ __device__ inline size_t ent_smem_bytes(const DresLayout& L) {
 }
 
 // MM: group size m; CB: code bytes per 16 positions (= 4n/m); NT: token
-// columns (8 or 16); DENSE: n == m (no keep bits); ACC: write int32 acc.
-template <int MM, int CB, int NT, bool ACC>
+// columns (8 or 16); ACC: write int32 acc; XBF: bf16 activations in, each
+// token row quantized in the prologue (as in bl_decode_res.cuh).
+template <int MM, int CB, int NT, bool ACC, bool XBF>
 __global__ void __launch_bounds__(kDresThreads, 1)
 bl_decode_ent_kernel(const DresParams p) {
-  constexpr bool DENSE = false, XBF = false;
+  constexpr bool DENSE = false;
   constexpr int kEntN = CB * MM / 4;                  // kept per group
   constexpr int kEntBits = entropy_group_bits(kEntN, MM);
   constexpr uint32_t kEntP3 = pow3_u32(kEntN);
@@ -39,7 +40,7 @@ bl_decode_ent_kernel(const DresParams p) {
   const int tiles = t_end - t_begin;
   // p.cstride is the entropy row stride; no keep-bit rows; the decode
   // tables follow the resident layout
-  const DresLayout L = dres_layout(p.tiles_per_cta, NT, p.K, p.cstride, 0, true, false);
+  const DresLayout L = dres_layout(p.tiles_per_cta, NT, p.K, p.cstride, 0, true, XBF);
   uint16_t* s_rank_mask = reinterpret_cast<uint16_t*>(dent_smem + ent_tables_offset(L));
   uint16_t* s_val_codes = s_rank_mask + kEntRankSlots;
   uint32_t* s_sel = reinterpret_cast<uint32_t*>(dent_smem + L.sel);

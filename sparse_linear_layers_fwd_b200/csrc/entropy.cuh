@@ -42,66 +42,6 @@ __host__ __device__ constexpr size_t entropy_row_bytes(int k, int n, int m) {
   return (((size_t)(k / m) * (size_t)entropy_group_bits(n, m) + 7u) / 8u + 15u) & ~(size_t)15;
 }
 
-constexpr int kEntThreads = 256;
-
-// Canonical packed weights (2-bit kept codes + keep bits) -> group words. One
-// thread per group; its word is OR-ed into the (zeroed) row stream, in at
-// most two 32-bit words. (i + 1 <= n <= 16 and pos < 16 keep the binomial
-// table index in range.)
-template <int M>
-__global__ void __launch_bounds__(kEntThreads)
-entropy_pack_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, int n_out,
-                    int k, int n, int cstride, int mstride, uint32_t* __restrict__ ent, int estride) {
-  // binomials C(a, b), a, b <= 16, from a table instead of a division loop
-  __shared__ uint32_t s_binom[17 * 17];
-  for (int i = threadIdx.x; i < 17 * 17; i += kEntThreads) s_binom[i] = binom_u32(i / 17, i % 17);
-  __syncthreads();
-  const int groups = k / M;
-  const int bits = entropy_group_bits(n, M);
-  const long long total = (long long)n_out * groups;
-  const uint32_t p3n = pow3_u32(n);
-  for (long long gidx = (long long)blockIdx.x * kEntThreads + threadIdx.x; gidx < total;
-       gidx += (long long)gridDim.x * kEntThreads) {
-    const int row = (int)(gidx / groups);
-    const int g = (int)(gidx - (long long)row * groups);
-    // keep bits of the group (all kept when n == M: no meta)
-    uint32_t keep = (1u << M) - 1u;
-    if (n != M) {
-      const uint8_t* mp = meta + (size_t)row * mstride;
-      const int bit = g * M;
-      keep = ((uint32_t)mp[bit >> 3] | ((M == 16) ? (uint32_t)mp[(bit >> 3) + 1] << 8 : 0u)) >> (bit & 7);
-      keep &= (1u << M) - 1u;
-    }
-    // the group's 2n code bits start at bit 2 n g of the row
-    const uint8_t* cp = codes + (size_t)row * cstride;
-    const int cbit = 2 * n * g;
-    uint64_t cw = 0ull;
-#pragma unroll
-    for (int b = 0; b < 5; ++b) {
-      const int byte = (cbit >> 3) + b;
-      if (byte < cstride) cw |= (uint64_t)cp[byte] << (8 * b);
-    }
-    cw >>= (cbit & 7);
-    uint32_t rank = 0u, v = 0u, p3 = 1u;
-    int i = 0;
-    for (int pos = 0; pos < M; ++pos) {
-      if (!((keep >> pos) & 1u)) continue;
-      rank += s_binom[pos * 17 + i + 1];
-      const uint32_t c2 = (uint32_t)(cw >> (2 * i)) & 3u;   // 00 -> 0, 01 -> +1, 11 -> -1
-      const uint32_t digit = (c2 == 1u) ? 2u : (c2 == 3u ? 0u : 1u);
-      v += digit * p3;
-      p3 *= 3u;
-      ++i;
-    }
-    const uint32_t word = rank * p3n + v;
-    const long long bo = (long long)g * bits;
-    uint32_t* rw = ent + (size_t)row * (estride / 4);
-    const int w0 = (int)(bo >> 5), sh = (int)(bo & 31);
-    atomicOr(rw + w0, word << sh);
-    if (sh + bits > 32) atomicOr(rw + w0 + 1, word >> (32 - sh));
-  }
-}
-
 constexpr int kEntRankSlots = 128;   // rank table entries (every word of M <= 8 has rank < 128)
 
 // Shared-memory tables for decoding group words of an n:M pattern (M <= 8):

@@ -5,10 +5,11 @@
 // scale preserved); per-token scale as on the promptingindex page, section
 // "How ternary quantization works during training".
 //
-// One CTA of 128 threads per token row. The row is held in registers
-// (MAXC 16-byte chunks per thread), so X is read from HBM exactly once:
-// max |x| (integer max of the 15 magnitude bits), one IEEE division for the
-// multiplier 127/s, then q = clamp(rint(x * mult), -127, 127).
+// One warp (K <= 3072) or one CTA of 128 threads (longer rows) per token
+// row. The row is held in registers (MAXC 16-byte chunks per thread), so X
+// is read from HBM exactly once: max |x| (integer max of the 15 magnitude
+// bits), one IEEE division for the multiplier 127/s, then
+// q = clamp(rint(x * mult), -127, 127).
 #pragma once
 
 #include "common.cuh"
@@ -71,6 +72,37 @@ qa_kernel(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __
 #pragma unroll
   for (int c = 0; c < MAXC; ++c) {
     const int idx = threadIdx.x + c * kQaThreads;
+    if (idx < kc) qr[idx] = quant8(v[c], mult);
+  }
+}
+
+// One warp per token row (rows of kc <= 32 * MAXC chunks, K <= 3072): the
+// row in registers, all its loads in flight at once, the maximum reduced in
+// the warp (no block barrier), and one wave of CTAs for thousands of rows.
+constexpr int kQawThreads = 128;   // small CTAs: 7 per SM at K = 2560
+template <int MAXC>
+__global__ void __launch_bounds__(kQawThreads)
+qa_warp_kernel(const uint4* __restrict__ x, int t, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+  const int row = blockIdx.x * (kQawThreads / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= t) return;   // whole warps only
+  const uint4* xr = x + (size_t)row * kc;
+  uint4 v[MAXC];
+  uint32_t amax = 0u;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int idx = lane + 32 * c;
+    v[c] = (idx < kc) ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
+    amax = max(amax, mag_max8(v[c]));
+  }
+  amax = __reduce_max_sync(0xffffffffu, amax);
+  const float s = fmaxf(__uint_as_float(amax << 16), 1e-5f);
+  const float mult = __fdiv_rn(127.0f, s);
+  if (lane == 0) scale[row] = s;
+  uint2* qr = xq + (size_t)row * kc;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int idx = lane + 32 * c;
     if (idx < kc) qr[idx] = quant8(v[c], mult);
   }
 }

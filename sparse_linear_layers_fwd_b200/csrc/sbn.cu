@@ -21,6 +21,7 @@
 #include "bl_decode_ent.cuh"
 #include "expand_dense.cuh"
 #include "entropy.cuh"
+#include "entropy_pack.cuh"
 #include "flip.cuh"
 #include "bl_tc.cuh"
 
@@ -216,7 +217,7 @@ sbn_status dispatch_decode_res(const DresParams& p, int n, int m, int grid, size
 }
 
 // Decode contraction over entropy-tight weights (patterns with m = 4 or 8).
-template <int MM, int CB, int NT, bool ACC>
+template <int MM, int CB, int NT, bool ACC, bool XBF>
 sbn_status launch_decode_ent(const DresParams& p, int grid, size_t smem, cudaStream_t st) {
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
@@ -224,7 +225,7 @@ sbn_status launch_decode_ent(const DresParams& p, int grid, size_t smem, cudaStr
     cudaGetLastError();
     return SBN_ERR_CUDA;
   }
-  auto kern = bl_decode_ent_kernel<MM, CB, NT, ACC>;
+  auto kern = bl_decode_ent_kernel<MM, CB, NT, ACC, XBF>;
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDresSmemMax) !=
         cudaSuccess) {
@@ -237,16 +238,16 @@ sbn_status launch_decode_ent(const DresParams& p, int grid, size_t smem, cudaStr
   return launch_status();
 }
 
-template <int NT, bool ACC>
+template <int NT, bool ACC, bool XBF>
 sbn_status dispatch_decode_ent(const DresParams& p, int n, int m, int grid, size_t smem,
                                cudaStream_t st) {
   switch (m * 8 + 4 * n / m) {
-    case 4 * 8 + 1: return launch_decode_ent<4, 1, NT, ACC>(p, grid, smem, st);
-    case 4 * 8 + 2: return launch_decode_ent<4, 2, NT, ACC>(p, grid, smem, st);
-    case 4 * 8 + 3: return launch_decode_ent<4, 3, NT, ACC>(p, grid, smem, st);
-    case 8 * 8 + 1: return launch_decode_ent<8, 1, NT, ACC>(p, grid, smem, st);
-    case 8 * 8 + 2: return launch_decode_ent<8, 2, NT, ACC>(p, grid, smem, st);
-    case 8 * 8 + 3: return launch_decode_ent<8, 3, NT, ACC>(p, grid, smem, st);
+    case 4 * 8 + 1: return launch_decode_ent<4, 1, NT, ACC, XBF>(p, grid, smem, st);
+    case 4 * 8 + 2: return launch_decode_ent<4, 2, NT, ACC, XBF>(p, grid, smem, st);
+    case 4 * 8 + 3: return launch_decode_ent<4, 3, NT, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 1: return launch_decode_ent<8, 1, NT, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 2: return launch_decode_ent<8, 2, NT, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 3: return launch_decode_ent<8, 3, NT, ACC, XBF>(p, grid, smem, st);
   }
   return SBN_ERR_PATTERN;
 }
@@ -467,12 +468,30 @@ size_t bitlinear_x_ws_bytes(int32_t t, int32_t k, int32_t n_out) {
   return round_up16((size_t)t * k) + round_up16((size_t)t * 4) + bitlinear_ws_bytes(t, k, n_out);
 }
 
-// One CTA per token row (qa.cuh); rows up to 16 * 128 * 8 positions stay in registers.
+// One warp per token row up to K = 3072, else one CTA per row (qa.cuh); rows
+// up to 16 * 128 * 8 positions stay in registers.
 sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, float* x_scale,
                                 cudaStream_t s) {
   const int kc = k / 8;
   const uint4* x = reinterpret_cast<const uint4*>(x_bf16);
   uint2* q = reinterpret_cast<uint2*>(xq);
+  const int wblocks = (t + kQawThreads / 32 - 1) / (kQawThreads / 32);
+  if (kc <= 32 * 4) {
+    qa_warp_kernel<4><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
+    return launch_status();
+  }
+  if (kc <= 32 * 8) {
+    qa_warp_kernel<8><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
+    return launch_status();
+  }
+  if (kc <= 32 * 10) {   // K <= 2560
+    qa_warp_kernel<10><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
+    return launch_status();
+  }
+  if (kc <= 32 * 12) {
+    qa_warp_kernel<12><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
+    return launch_status();
+  }
   const int need = (kc + kQaThreads - 1) / kQaThreads;
   if (need <= 1) qa_kernel<1><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
   else if (need <= 2) qa_kernel<2><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
@@ -484,33 +503,78 @@ sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, fl
   return launch_status();
 }
 
-template <bool ACC>
-sbn_status run_bitlinear_entropy(const int8_t* xq, const float* xs, int32_t t, int32_t k, int32_t n_out,
-                                 int32_t n, int32_t m, const uint8_t* ent, const float* gamma, uint16_t* y,
-                                 int32_t* acc, void* stream) {
+// Grid, CTA range and shared memory of the entropy decode; false when the
+// shape is outside it (t > 16, or rows that do not fit in shared memory).
+bool ent_decode_fits(int32_t t, int32_t k, int32_t n_out, int32_t n, int32_t m, int sms, bool xbf,
+                     int* grid, int* per_cta, size_t* smem) {
+  if (t < 1 || t > 16) return false;
+  const int estride = (int)entropy_row_bytes(k, n, m);
+  const int tiles = (n_out + 15) / 16;
+  *grid = std::min(sms, tiles);
+  *per_cta = (tiles + *grid - 1) / *grid;
+  const DresLayout L = dres_layout(*per_cta, t <= 8 ? 8 : 16, k, estride, 0, true, xbf);
+  *smem = ent_smem_bytes(L);
+  return *per_cta <= kDresMaxTiles && *smem <= kDresSmemMax;
+}
+
+sbn_status ent_decode_args(int32_t t, int32_t k, int32_t n_out, int32_t n, int32_t m) {
   if (!pattern_ok(n, m)) return SBN_ERR_PATTERN;
   if (n == m || (m != 4 && m != 8)) return SBN_ERR_PATTERN;
   if (t < 1 || t > 16 || n_out < 1 || k < 128 || (k % 128) != 0 || !prod_lt_2_31(n_out, k))
     return SBN_ERR_SHAPE;
+  return SBN_OK;
+}
+
+// One launch of the entropy decode. XBF: bf16 activations xbf, quantized in
+// the kernel (optional copies to xq_out, xs_out); else xq, xs.
+template <bool ACC, bool XBF>
+sbn_status launch_bitlinear_entropy(const int8_t* xq, const float* xs, const uint16_t* xbf, int8_t* xq_out,
+                                    float* xs_out, int32_t t, int32_t k, int32_t n_out, int32_t n,
+                                    int32_t m, const uint8_t* ent, const float* gamma, uint16_t* y,
+                                    int32_t* acc, int grid, int per_cta, size_t smem, cudaStream_t cs) {
+  DresParams q;
+  q.xq = xq; q.xs = xs; q.xbf = xbf; q.xq_out = xq_out; q.xs_out = xs_out;
+  q.codes = ent; q.meta = nullptr; q.gamma = gamma; q.y = y; q.acc_out = acc;
+  q.T = t; q.K = k; q.N = n_out; q.cstride = (int)entropy_row_bytes(k, n, m); q.mstride = 0;
+  q.tiles_per_cta = per_cta;
+  return t <= 8 ? dispatch_decode_ent<8, ACC, XBF>(q, n, m, grid, smem, cs)
+                : dispatch_decode_ent<16, ACC, XBF>(q, n, m, grid, smem, cs);
+}
+
+template <bool ACC>
+sbn_status run_bitlinear_entropy(const int8_t* xq, const float* xs, int32_t t, int32_t k, int32_t n_out,
+                                 int32_t n, int32_t m, const uint8_t* ent, const float* gamma, uint16_t* y,
+                                 int32_t* acc, void* stream) {
+  sbn_status st = ent_decode_args(t, k, n_out, n, m);
+  if (st != SBN_OK) return st;
   if (!aligned16(xq) || !aligned16(ent)) return SBN_ERR_ALIGN;
   int dev = 0, sms = 0;
-  sbn_status st = check_device(&dev, &sms);
-  if (st != SBN_OK) return st;
-  const int estride = (int)entropy_row_bytes(k, n, m);
-  const int tiles = (n_out + 15) / 16;
-  const int grid = std::min(sms, tiles);
-  const int per_cta = (tiles + grid - 1) / grid;
-  const int nt = t <= 8 ? 8 : 16;
-  const DresLayout L = dres_layout(per_cta, nt, k, estride, 0, true);
-  const size_t smem = ent_smem_bytes(L);
-  if (per_cta > kDresMaxTiles || smem > kDresSmemMax) return SBN_ERR_SHAPE;
-  DresParams q;
-  q.xq = xq; q.xs = xs; q.xbf = nullptr; q.xq_out = nullptr; q.xs_out = nullptr;
-  q.codes = ent; q.meta = nullptr; q.gamma = gamma; q.y = y; q.acc_out = acc;
-  q.T = t; q.K = k; q.N = n_out; q.cstride = estride; q.mstride = 0; q.tiles_per_cta = per_cta;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  return t <= 8 ? dispatch_decode_ent<8, ACC>(q, n, m, grid, smem, cs)
-                : dispatch_decode_ent<16, ACC>(q, n, m, grid, smem, cs);
+  if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
+  int grid = 0, per_cta = 0;
+  size_t smem = 0;
+  if (!ent_decode_fits(t, k, n_out, n, m, sms, false, &grid, &per_cta, &smem)) return SBN_ERR_SHAPE;
+  return launch_bitlinear_entropy<ACC, false>(xq, xs, nullptr, nullptr, nullptr, t, k, n_out, n, m, ent, gamma, y,
+                                       acc, grid, per_cta, smem, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Workspace of sbn_bitlinear_entropy_x when it runs as two steps (Xq and s).
+size_t bitlinear_entropy_x_ws_bytes(int32_t t, int32_t k) {
+  return round_up16((size_t)t * k) + round_up16((size_t)t * 4);
+}
+
+// Resident blocks per SM of the entropy packer (its grid fills the GPU once).
+int ent_pack_blocks_per_sm(int dev, int m) {
+  static int cached[kMaxDevices][3] = {};   // m = 4, 8, 16 (benign race: same value)
+  const int mi = m == 4 ? 0 : (m == 8 ? 1 : 2);
+  if (cached[dev][mi] == 0) {
+    int b = 0;
+    cudaError_t e = m == 4 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, entropy_pack_kernel<4>, kEpThreads, 0)
+                  : m == 8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, entropy_pack_kernel<8>, kEpThreads, 0)
+                           : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, entropy_pack_kernel<16>, kEpThreads, 0);
+    if (e != cudaSuccess) cudaGetLastError();
+    cached[dev][mi] = std::max(1, b);
+  }
+  return cached[dev][mi];
 }
 
 // Fixed scratch of sbn_quantize_weights_noalloc (see include/sbn.h).
@@ -645,21 +709,22 @@ sbn_status sbn_pack_entropy(const uint8_t* codes, const uint8_t* meta, int32_t n
   int dev = 0, sms = 0;
   if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const size_t ebytes = sbn_entropy_bytes(n_out, k, n, m);
-  if (cudaMemsetAsync(ent, 0, ebytes, cs) != cudaSuccess) {
-    cudaGetLastError();
-    return SBN_ERR_CUDA;
-  }
-  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
-  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
-  const int estride = (int)sbn_entropy_row_bytes(k, n, m);
-  const long long groups = (long long)n_out * (k / m);
-  const int grid = (int)std::max(1LL, std::min((groups + kEntThreads - 1) / kEntThreads, (long long)sms * 8));
+  const int cws = (int)(sbn_codes_row_bytes(k, n, m) / 4);
+  const int mws = (int)(sbn_meta_row_bytes(k, n, m) / 4);
+  const int ews = (int)(sbn_entropy_row_bytes(k, n, m) / 4);
+  EntPackParams prm;
+  fill_ent_pack_params(prm, n, m);
+  const long long segs = (k / m + 31) / 32;   // 32-group segments per row
+  const long long items = (long long)n_out * ((segs + kEpUnroll - 1) / kEpUnroll);
+  const int grid = (int)std::max(1LL, std::min((items + kEpWarps - 1) / kEpWarps,
+                                               (long long)sms * ent_pack_blocks_per_sm(dev, m)));
+  const uint32_t* c32 = reinterpret_cast<const uint32_t*>(codes);
+  const uint32_t* m32 = reinterpret_cast<const uint32_t*>(meta);
   uint32_t* e32 = reinterpret_cast<uint32_t*>(ent);
   switch (m) {
-    case 4: entropy_pack_kernel<4><<<grid, kEntThreads, 0, cs>>>(codes, meta, n_out, k, n, cstride, mstride, e32, estride); break;
-    case 8: entropy_pack_kernel<8><<<grid, kEntThreads, 0, cs>>>(codes, meta, n_out, k, n, cstride, mstride, e32, estride); break;
-    default: entropy_pack_kernel<16><<<grid, kEntThreads, 0, cs>>>(codes, meta, n_out, k, n, cstride, mstride, e32, estride); break;
+    case 4: entropy_pack_kernel<4><<<grid, kEpThreads, 0, cs>>>(c32, m32, n_out, k, n, cws, mws, e32, ews, prm); break;
+    case 8: entropy_pack_kernel<8><<<grid, kEpThreads, 0, cs>>>(c32, m32, n_out, k, n, cws, mws, e32, ews, prm); break;
+    default: entropy_pack_kernel<16><<<grid, kEpThreads, 0, cs>>>(c32, m32, n_out, k, n, cws, mws, e32, ews, prm); break;
   }
   return launch_status();
 }
@@ -678,6 +743,45 @@ sbn_status sbn_bitlinear_entropy_acc32(const int8_t* xq, int32_t t, int32_t k, i
   if (!xq || !ent || !acc) return SBN_ERR_NULL;
   if (!aligned16(acc)) return SBN_ERR_ALIGN;
   return run_bitlinear_entropy<true>(xq, nullptr, t, k, n_out, n, m, ent, nullptr, nullptr, acc, stream);
+}
+
+size_t sbn_bitlinear_entropy_x_workspace_bytes(int32_t t, int32_t k) {
+  if (t < 1 || k < 1) return 0;
+  return bitlinear_entropy_x_ws_bytes(t, k);
+}
+
+sbn_status sbn_bitlinear_entropy_x(const void* x_bf16, int32_t t, int32_t k, int32_t n_out, int32_t n,
+                                   int32_t m, const uint8_t* ent, const float* gamma, void* y_bf16,
+                                   int8_t* xq, float* x_scale, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  if (!x_bf16 || !ent || !gamma || !y_bf16) return SBN_ERR_NULL;
+  sbn_status st = ent_decode_args(t, k, n_out, n, m);
+  if (st != SBN_OK) return st;
+  if (!prod_lt_2_31(t, k) || !prod_lt_2_31(t, n_out)) return SBN_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(ent) || !aligned16(y_bf16) || (xq && !aligned16(xq)) ||
+      (reinterpret_cast<uintptr_t>(x_scale) & 3u) || (workspace && !aligned16(workspace)))
+    return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint16_t* y = reinterpret_cast<uint16_t*>(y_bf16);
+  int grid = 0, per_cta = 0;
+  size_t smem = 0;
+  if (ent_decode_fits(t, k, n_out, n, m, sms, true, &grid, &per_cta, &smem))
+    return launch_bitlinear_entropy<false, true>(nullptr, nullptr, reinterpret_cast<const uint16_t*>(x_bf16),
+                                                 xq, x_scale, t, k, n_out, n, m, ent, gamma, y, nullptr,
+                                                 grid, per_cta, smem, cs);
+  // two steps: quantize_acts into the given buffers or the workspace, then
+  // the contraction over int8 activations
+  if (!ent_decode_fits(t, k, n_out, n, m, sms, false, &grid, &per_cta, &smem)) return SBN_ERR_SHAPE;
+  if ((!xq || !x_scale) && (!workspace || ws_bytes < bitlinear_entropy_x_ws_bytes(t, k)))
+    return SBN_ERR_WORKSPACE;
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(workspace);
+  int8_t* q8 = xq ? xq : reinterpret_cast<int8_t*>(w8);
+  float* sc = x_scale ? x_scale : reinterpret_cast<float*>(w8 + round_up16((size_t)t * k));
+  if ((st = launch_quantize_acts(x_bf16, t, k, q8, sc, cs)) != SBN_OK) return st;
+  return launch_bitlinear_entropy<false, false>(q8, sc, nullptr, nullptr, nullptr, t, k, n_out, n, m, ent,
+                                                gamma, y, nullptr, grid, per_cta, smem, cs);
 }
 
 size_t sbn_bitlinear_x_workspace_bytes(int32_t t, int32_t k, int32_t n_out) {

@@ -59,6 +59,9 @@ PROTOTYPES = {
                                              _c_p, _c_p, _c_p, _c_p]),
     "sbn_bitlinear_entropy_acc32": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
                                                    _c_p, _c_p, _c_p]),
+    "sbn_bitlinear_entropy_x": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
+                                               _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "sbn_bitlinear_entropy_x_workspace_bytes": (_c_sz, [_c_i32, _c_i32]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
 
@@ -322,6 +325,30 @@ def bitlinear_entropy_acc32(xq: torch.Tensor, ent: torch.Tensor, w: PackedWeight
     st = lib().sbn_bitlinear_entropy_acc32(_ptr(xq), t, k, w.n_out, w.n, w.m, _ptr(ent), _ptr(out),
                                            _stream_ptr(stream))
     _check(st, "sbn_bitlinear_entropy_acc32")
+    return out
+
+
+def bitlinear_entropy_x(x: torch.Tensor, ent: torch.Tensor, w: PackedWeights,
+                        out: Optional[torch.Tensor] = None, out_q: Optional[torch.Tensor] = None,
+                        out_s: Optional[torch.Tensor] = None, workspace=None, stream=None) -> torch.Tensor:
+    """sbn_bitlinear_entropy_x: y = bitlinear_entropy(quantize_acts(x)) in one
+    call (one kernel when the bf16 rows fit in shared memory). out_q / out_s,
+    if given, receive Xq and s. workspace: None allocates the two-step route's
+    scratch, False passes none."""
+    _need(x, torch.bfloat16, "x")
+    t, k = x.shape
+    if k != w.k:
+        raise ValueError("K mismatch between activations and weights")
+    if out is None:
+        out = torch.empty((t, w.n_out), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((int(lib().sbn_bitlinear_entropy_x_workspace_bytes(t, k)),),
+                                dtype=torch.uint8, device=x.device)
+    ws_ptr, ws_n = (None, 0) if workspace is False else (_ptr(workspace), workspace.numel())
+    st = lib().sbn_bitlinear_entropy_x(_ptr(x), t, k, w.n_out, w.n, w.m, _ptr(ent), _ptr(w.gamma),
+                                       _ptr(out), _ptr(out_q), _ptr(out_s), ws_ptr, ws_n,
+                                       _stream_ptr(stream))
+    _check(st, "sbn_bitlinear_entropy_x")
     return out
 
 

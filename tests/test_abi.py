@@ -166,6 +166,17 @@ def test_entropy_validation(sbn_lib):
     assert bl(A, A, 4, 256, 64, 2, 4, MIS, A, A, None) == 4
     assert lib.sbn_bitlinear_entropy_acc32(A, 4, 256, 64, 2, 4, A, None, None) == 1
     assert lib.sbn_entropy_row_bytes(2560, 6, 8) == 608                   # 320 x 15 bits -> 600 B
+    bx = lib.sbn_bitlinear_entropy_x
+    assert bx(None, 4, 256, 64, 2, 4, A, A, A, None, None, None, 0, None) == 1
+    assert bx(A, 4, 256, 64, 2, 4, None, A, A, None, None, None, 0, None) == 1
+    assert bx(A, 4, 256, 64, 8, 16, A, A, A, None, None, None, 0, None) == 3     # m = 16: not decoded
+    assert bx(A, 17, 256, 64, 2, 4, A, A, A, None, None, None, 0, None) == 2     # decode only
+    assert bx(A, 4, 200, 64, 2, 4, A, A, A, None, None, None, 0, None) == 2
+    assert bx(MIS, 4, 256, 64, 2, 4, A, A, A, None, None, None, 0, None) == 4
+    assert bx(A, 4, 256, 64, 2, 4, A, A, A, MIS, None, None, 0, None) == 4       # xq copy
+    assert bx(A, 4, 256, 64, 2, 4, A, A, A, None, A + 2, None, 0, None) == 4     # x_scale copy
+    assert lib.sbn_bitlinear_entropy_x_workspace_bytes(4, 256) == 4 * 256 + 16
+    assert lib.sbn_bitlinear_entropy_x_workspace_bytes(0, 256) == 0
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")

@@ -343,13 +343,16 @@ ENT_DECODE = [(1, 4), (2, 4), (3, 4), (2, 8), (4, 8), (6, 8)]
 
 
 @pytest.mark.parametrize("nm", SUPPORTED)
-@pytest.mark.parametrize("shape", [(7, 128), (130, 1024), (257, 512)])
+@pytest.mark.parametrize("shape", [(7, 128), (130, 1024), (257, 512), (3, 1152)])
 def test_pack_entropy_matches_oracle(nm, shape):
     n_out, k = shape
     w = synth.latent_weights(n_out, k, seed=19, tag=f"entp{nm}{shape}")
     from sparse_linear_layers_fwd_b200 import sbn
+    import torch
     pw = run_quantize_weights(w, *nm)
-    got = sbn.pack_entropy(pw).cpu().numpy()
+    # every byte, row padding included, is written by the packer: start from 0xFF
+    out = torch.full((n_out, sbn.entropy_row_bytes(k, *nm)), 255, dtype=torch.uint8, device="cuda")
+    got = sbn.pack_entropy(pw, out=out).cpu().numpy()
     cb, mb, gamma, mask, dense = oracle.quantize_weights(w, *nm)
     assert np.array_equal(got, oracle.entropy_pack(mask, dense, *nm))
 
@@ -371,6 +374,25 @@ def _entropy_decode_check(w, x, n, m):
     assert np.array_equal(acc_ent.cpu().numpy(), acc)
     assert np.array_equal(bf16_tensor_bits(y_ent), bf16_tensor_bits(y_can))
     assert_y_close(bf16_tensor_bits(y_ent), oracle.dequant_bf16(acc, sc, gamma))
+    _entropy_fused_check(x, ent, pw, q, sc, y_ent)
+
+
+def _entropy_fused_check(x, ent, pw, q, sc, y_ent):
+    """sbn_bitlinear_entropy_x: Xq and s bit-exact against the oracle, y
+    bit-identical to sbn_quantize_acts followed by sbn_bitlinear_entropy."""
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    t, k = x.shape
+    xd = to_dev_bf16(x)
+    oq = torch.full((t, k), 99, dtype=torch.int8, device="cuda")
+    os_ = torch.full((t,), -1.0, dtype=torch.float32, device="cuda")
+    y_x = sbn.bitlinear_entropy_x(xd, ent, pw, out_q=oq, out_s=os_, workspace=False)
+    y_x2 = sbn.bitlinear_entropy_x(xd, ent, pw)
+    torch.cuda.synchronize()
+    assert sbn.get_device_error() == 0
+    assert np.array_equal(oq.cpu().numpy(), q) and np.array_equal(os_.cpu().numpy(), sc)
+    assert np.array_equal(bf16_tensor_bits(y_x), bf16_tensor_bits(y_ent))
+    assert np.array_equal(bf16_tensor_bits(y_x2), bf16_tensor_bits(y_ent))
 
 
 @pytest.mark.parametrize("nm", ENT_DECODE)
@@ -380,6 +402,23 @@ def test_bitlinear_entropy(nm, shape):
     w = synth.latent_weights(n_out, k, seed=20, tag=f"entd{nm}{shape}")
     x = synth.activations(t, k, seed=20, tag=f"entd{nm}{shape}", outlier_channels=2)
     _entropy_decode_check(w, x, *nm)
+
+
+def test_bitlinear_entropy_x_two_step_route():
+    # T = 16 bf16 rows of K = 6144 do not fit in shared memory beside the
+    # int8 rows: quantize_acts, then the contraction over int8 activations
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    t, k, n_out, n, m = 16, 6144, 40, 2, 8
+    w = synth.latent_weights(n_out, k, seed=21, tag="ent2step")
+    x = synth.activations(t, k, seed=21, tag="ent2step", outlier_channels=2)
+    _entropy_decode_check(w, x, n, m)
+    pw = run_quantize_weights(w, n, m)
+    ent = sbn.pack_entropy(pw)
+    with pytest.raises(sbn.SbnError) as e:   # no workspace and no Xq / s outputs to quantize into
+        sbn.bitlinear_entropy_x(to_dev_bf16(x), ent, pw, workspace=False)
+    assert e.value.status == 5
+    torch.cuda.synchronize()
 
 
 @pytest.mark.parametrize("t", synth.DECODE_TOKENS)
