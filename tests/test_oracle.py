@@ -172,7 +172,7 @@ def test_mask_index_bits_match_the_pages_accounting():
     assert oracle.entropy_group_bits(6, 8) == 15           # 28 * 729 = 20412 < 2^15
 
 
-def testcolex_rank_order_for_2of4():
+def test_colex_rank_order_for_2of4():
     order = [(0, 1), (0, 2), (1, 2), (0, 3), (1, 3), (2, 3)]
     for r, offs in enumerate(order):
         assert oracle.colex_rank(list(offs)) == r
