@@ -1,4 +1,5 @@
-"""Plain, slow CPU oracle of the Sparse-BitNet BitLinear forward.
+"""Plain, slow CPU oracle of the Sparse-BitNet BitLinear layer: the forward
+path and its straight-through backward.
 
 TEST INFRASTRUCTURE. This module is the yardstick the CUDA path is checked
 against. It shares no code with ``sparse_linear_layers_fwd_b200`` (no kernels,
@@ -25,6 +26,10 @@ What it computes (the BitLinear forward with a dynamic N:M mask):
    ("The BitLinear Layer", fourth operation: addition, subtraction, zero-skips).
 6. y      -- dequantization with the preserved scales ("The BitLinear Layer",
    fifth operation).
+7. dX, dW -- the backward of the layer under the straight-through estimator
+   ("Microsoft BitNet 1.58 ...", section "Training with the Straight-Through
+   Estimator": gradients cross the quantizer as the identity, the latent
+   weights take the update).
 
 Readings where the pages are silent (each is listed in the design doc):
 * gamma is taken over the whole dense latent tensor, before masking;
@@ -86,6 +91,8 @@ __all__ = [
     "entropy_row_bytes",
     "entropy_pack",
     "entropy_unpack",
+    "ste_grad_x",
+    "ste_grad_w",
 ]
 
 #: floor on gamma and on the per-token activation scale (not on the pages)
@@ -492,3 +499,35 @@ def entropy_unpack(packed: np.ndarray, k: int, n: int, m: int):
                 mask[r, g * m + j] = True
                 dense[r, g * m + j] = (v // 3 ** i) % 3 - 1
     return dense, mask
+
+
+# --------------------------------------------------------------------------
+# 7. backward through the layer (straight-through estimator)
+# --------------------------------------------------------------------------
+#
+# "Microsoft BitNet 1.58 ...", section "Training with the Straight-Through
+# Estimator": in the backward pass the gradients cross the quantizer as if it
+# were the identity function, and the full-precision latent weights receive
+# them. The forward multiplies Xd = Xq * s_t / 127 (the dequantized
+# activations) by Wd = gamma * C (C the dense masked codes): Y = Xd Wd^T.
+# With both quantizers (the N:M mask included) passed as the identity, the
+# gradients of a loss L with dL/dY = dY are
+#     dX = dY Wd      [T, K]     (to the activations X)
+#     dW = dY^T Xd    [N_out, K] (to the latent weights W, at every position)
+# Both are evaluated in fp64 and rounded once to bf16: gradients are kept in
+# bf16 ("BitNet b1.58: How Ternary Weights ...", section "How ternary
+# quantization works during training": the optimizer accumulates in FP16 or
+# BF16).
+
+def ste_grad_x(dy_bits: np.ndarray, dense_codes: np.ndarray, gamma: np.float32) -> np.ndarray:
+    """dX = bf16_rne(dY (gamma C)) for dY bf16 [T, N_out], C int8 [N_out, K]."""
+    dy = bf16_bits_to_f32(dy_bits).astype(np.float64)
+    wd = float(gamma) * np.asarray(dense_codes).astype(np.float64)
+    return bf16_bits_from_f64_rne(dy @ wd)
+
+
+def ste_grad_w(dy_bits: np.ndarray, xq: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """dW = bf16_rne(dY^T (Xq s_t / 127)) for dY bf16 [T, N_out], Xq int8 [T, K]."""
+    dy = bf16_bits_to_f32(dy_bits).astype(np.float64)
+    xd = np.asarray(xq).astype(np.float64) * (np.asarray(s).astype(np.float64)[:, None] / Q_ACT)
+    return bf16_bits_from_f64_rne(dy.T @ xd)

@@ -15,8 +15,9 @@ Pages cited:
   Accuracy" -- section "How ternary quantization works during training"
   (divide by mean |W|, round, clamp to [-1, 1]; INT8 per-token activations);
 * "Microsoft BitNet 1.58: The Era of 1-Bit Large Language Models" -- section
-  "The BitLinear Layer" (five operations) and "bitnet.cpp: Matrix-Free
-  Inference" (four 2-bit values per byte).
+  "The BitLinear Layer" (five operations), "bitnet.cpp: Matrix-Free
+  Inference" (four 2-bit values per byte) and "Training with the
+  Straight-Through Estimator" (the quantizer is the identity backward).
 """
 
 from __future__ import annotations
@@ -526,3 +527,130 @@ def check_entropy_bijection(impl, n=2, m=4):
             d2, m2 = impl.entropy_unpack(impl.entropy_pack(mask, dense, n, m), m, n, m)
             assert np.array_equal(d2, dense) and np.array_equal(m2, mask)
     assert len(seen) == math.comb(m, n) * 3 ** n
+
+
+# ---- backward (straight-through estimator) ----------------------------------
+#
+# "Microsoft BitNet 1.58 ...", section "Training with the Straight-Through
+# Estimator": the quantizer is the identity in the backward pass, so the
+# gradients are those of the bilinear map Y = Xd Wd^T of the dequantized
+# operands Xd = Xq s_t / 127 and Wd = gamma C that the forward multiplies.
+
+def _random_bf16_bits(rng, shape):
+    """Normal bf16 numbers of both signs, magnitudes 2**-7 .. 2**8."""
+    e = rng.integers(120, 136, size=shape)
+    mant = rng.integers(0, 128, size=shape)
+    sign = rng.integers(0, 2, size=shape) << 15
+    return (sign | (e << 7) | mant).astype(np.uint16)
+
+
+def _bf16_value(bits) -> Fraction:
+    return Fraction(float(bf16_to_f64(np.array([bits], np.uint16))[0]))
+
+
+def check_ste_grad_x_exact(impl, seed=41):
+    """dX[t, k] = sum_n dY[t, n] gamma C[n, k], exact rationals, then one
+    correct bf16 rounding; non-square so that a transposed operand fails."""
+    rng = np.random.default_rng(seed)
+    t, n_out, k = 3, 5, 12
+    dy = _random_bf16_bits(rng, (t, n_out))
+    c = rng.integers(-1, 2, size=(n_out, k)).astype(np.int8)
+    g = np.float32(0.0137)
+    got = np.asarray(impl.ste_grad_x(dy, c, g))
+    assert got.shape == (t, k)
+    for i in range(t):
+        for j in range(k):
+            exact = sum((_bf16_value(dy[i, nn]) * Fraction(float(g)) * int(c[nn, j]) for nn in range(n_out)),
+                        Fraction(0))
+            assert _bf16_value(got[i, j]) == fraction_to_bf16_value(exact), (i, j)
+
+
+def check_ste_grad_w_exact(impl, seed=42):
+    """dW[n, k] = sum_t dY[t, n] Xq[t, k] s_t / 127, exact rationals, then one
+    correct bf16 rounding."""
+    rng = np.random.default_rng(seed)
+    t, n_out, k = 4, 3, 7
+    dy = _random_bf16_bits(rng, (t, n_out))
+    q = rng.integers(-127, 128, size=(t, k)).astype(np.int8)
+    sc = np.array([0.5, 3.25, 17.0, 1e-5], dtype=np.float32)
+    got = np.asarray(impl.ste_grad_w(dy, q, sc))
+    assert got.shape == (n_out, k)
+    for nn in range(n_out):
+        for j in range(k):
+            exact = sum((_bf16_value(dy[i, nn]) * int(q[i, j]) * Fraction(float(sc[i])) / 127 for i in range(t)),
+                        Fraction(0))
+            assert _bf16_value(got[nn, j]) == fraction_to_bf16_value(exact), (nn, j)
+
+
+def check_ste_one_hot(impl):
+    """Closed forms: a one-hot dY at (t0, n0) gives dX[t0] = gamma C[n0] and
+    dW[n0] = Xq[t0] s_t0 / 127, every other row zero."""
+    t, n_out, k = 2, 3, 8
+    c = np.array([[1, 0, -1, 1, 0, 0, -1, 1], [0, 1, 1, 0, -1, 1, 0, 0], [-1, -1, 0, 0, 1, 1, 1, 0]], np.int8)
+    g = np.float32(0.25)
+    q = np.array([[3, -127, 0, 64, 5, -5, 100, 1], [1, 2, 3, 4, 5, 6, 7, 8]], np.int8)
+    sc = np.array([12.7, 0.127], dtype=np.float32)
+    dy = np.zeros((t, n_out), np.uint16)
+    dy[1, 2] = 0x3F80                                    # 1.0
+    dx = bf16_to_f64(np.asarray(impl.ste_grad_x(dy, c, g)))
+    assert np.all(dx[0] == 0) and np.array_equal(dx[1], 0.25 * c[2].astype(np.float64))
+    dw = np.asarray(impl.ste_grad_w(dy, q, sc))
+    assert np.all(bf16_to_f64(dw[:2]) == 0)
+    for j in range(k):
+        assert _bf16_value(dw[2, j]) == fraction_to_bf16_value(int(q[1, j]) * Fraction(float(sc[1])) / 127)
+
+
+def check_ste_finite_difference(impl, seed=43):
+    """The loss L = sum dY * (Xd Wd^T) is bilinear, so raising one entry of
+    Xd (or Wd) by 1 changes L by exactly the matching gradient entry."""
+    rng = np.random.default_rng(seed)
+    t, n_out, k = 3, 4, 16
+    dy = _random_bf16_bits(rng, (t, n_out))
+    c = rng.integers(-1, 2, size=(n_out, k)).astype(np.int8)
+    g = np.float32(0.021)
+    q = rng.integers(-127, 128, size=(t, k)).astype(np.int8)
+    sc = rng.uniform(0.5, 8.0, size=t).astype(np.float32)
+    G = bf16_to_f64(dy)
+    xd = q.astype(np.float64) * (sc.astype(np.float64)[:, None] / 127.0)
+    wd = float(g) * c.astype(np.float64)
+
+    def loss(a, b):
+        return float(np.einsum("tn,tk,nk->", G, a, b))
+
+    dx = bf16_to_f64(np.asarray(impl.ste_grad_x(dy, c, g)))
+    dw = bf16_to_f64(np.asarray(impl.ste_grad_w(dy, q, sc)))
+    base = loss(xd, wd)
+    tol = 1e-9 * (1.0 + abs(base))
+    for (i, j) in [(0, 0), (1, 7), (2, 15), (0, 9)]:
+        xp = xd.copy()
+        xp[i, j] += 1.0
+        fd = loss(xp, wd) - base
+        assert abs(dx[i, j] - fd) <= 2.0 ** -8 * abs(fd) + tol, (i, j)
+    for (nn, j) in [(0, 0), (3, 5), (2, 11), (1, 15)]:
+        wp = wd.copy()
+        wp[nn, j] += 1.0
+        fd = loss(xd, wp) - base
+        assert abs(dw[nn, j] - fd) <= 2.0 ** -8 * abs(fd) + tol, (nn, j)
+
+
+def check_ste_matches_forward(impl, w_bits, x_bits, n, m, seed=44):
+    """The backward linearizes the forward the oracle computes: for the
+    bilinear Y = Xd Wd^T, sum(Xd * dX) = sum(dY * Y) = sum(Wd * dW), with Y
+    from the forward's exact accumulators (acc gamma s_t / 127). Masked
+    codes, gamma and the dequantized activations must all be the forward's."""
+    rng = np.random.default_rng(seed)
+    cb, mb, g, mask, dense = _impl_quantize_weights(impl, w_bits, n, m)
+    q, sc = impl.quantize_acts(x_bits)
+    acc = np.asarray(impl.bitlinear_acc(q, dense)).astype(np.float64)
+    y = acc * float(g) * (np.asarray(sc, np.float64)[:, None] / 127.0)
+    dy = _random_bf16_bits(rng, y.shape)
+    G = bf16_to_f64(dy)
+    dx = bf16_to_f64(np.asarray(impl.ste_grad_x(dy, dense, g)))
+    dw = bf16_to_f64(np.asarray(impl.ste_grad_w(dy, q, sc)))
+    xd = np.asarray(q).astype(np.float64) * (np.asarray(sc, np.float64)[:, None] / 127.0)
+    wd = dense.astype(np.float64) * float(g)
+    gy = float(np.sum(G * y))
+    # each gradient entry is within 2**-8 of its exact value, so each sum is
+    # within 2**-8 of sum |operand| |gradient|
+    assert abs(float(np.sum(xd * dx)) - gy) <= 2.0 ** -8 * float(np.sum(np.abs(xd) * np.abs(dx))) + 1e-9 * (1 + abs(gy))
+    assert abs(float(np.sum(wd * dw)) - gy) <= 2.0 ** -8 * float(np.sum(np.abs(wd) * np.abs(dw))) + 1e-9 * (1 + abs(gy))

@@ -221,3 +221,27 @@ def test_entropy_round_trip_on_quantized_layers(nm):
     assert packed.shape == (9, oracle.entropy_row_bytes(256, n, m))
     d2, m2 = oracle.entropy_unpack(packed, 256, n, m)
     assert np.array_equal(d2, dense) and np.array_equal(m2, mask)
+
+
+# ---- backward: straight-through estimator ------------------------------------
+
+def test_ste_grad_x_exact_rationals():
+    pins.check_ste_grad_x_exact(oracle)
+
+
+def test_ste_grad_w_exact_rationals():
+    pins.check_ste_grad_w_exact(oracle)
+
+
+def test_ste_one_hot_closed_forms():
+    pins.check_ste_one_hot(oracle)
+
+
+def test_ste_finite_differences():
+    pins.check_ste_finite_difference(oracle)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8)])
+def test_ste_linearizes_the_forward(nm):
+    d = synth.layer_small()
+    pins.check_ste_matches_forward(oracle, d["w"], d["x"], *nm)

@@ -204,6 +204,33 @@ def _lex_rank(offs):
     return list(it.combinations(range(m), len(offs))).index(tuple(offs))
 
 
+def ste_dx_no_gamma(dy_bits, dense_codes, gamma):
+    return O.ste_grad_x(dy_bits, dense_codes, np.float32(1.0))       # mistake: gamma dropped
+
+
+def ste_dx_transposed(dy_bits, dense_codes, gamma):
+    dy = O.bf16_bits_to_f32(dy_bits).astype(np.float64)
+    return O.bf16_bits_from_f64_rne(dy @ (float(gamma) * dense_codes.astype(np.float64)).T)
+
+
+def ste_dx_sign_flip(dy_bits, dense_codes, gamma):
+    return O.ste_grad_x(dy_bits, -np.asarray(dense_codes), gamma)
+
+
+def ste_dw_no_127(dy_bits, xq, s):
+    return O.ste_grad_w(dy_bits, xq, np.asarray(s, np.float64) * 127.0)   # mistake: Xq s, not Xq s/127
+
+
+def ste_dw_unscaled(dy_bits, xq, s):
+    return O.ste_grad_w(dy_bits, xq, np.full(np.shape(s), 127.0))         # mistake: raw Xq
+
+
+def ste_dw_transposed_dy(dy_bits, xq, s):
+    dy = O.bf16_bits_to_f32(dy_bits).astype(np.float64)
+    xd = np.asarray(xq).astype(np.float64) * (np.asarray(s, np.float64)[:, None] / O.Q_ACT)
+    return O.bf16_bits_from_f64_rne(dy @ xd.T)
+
+
 MUTANTS = {
     "gamma_no_subnormal": dict(absmean_gamma=gamma_no_subnormal, gamma_bins=bins_no_subnormal),
     "gamma_exponent_off_by_one": dict(absmean_gamma=gamma_exponent_off_by_one),
@@ -231,6 +258,12 @@ MUTANTS = {
     "entropy_lex_rank": dict(entropy_pack=_entropy_pack_with(rank_fn=_lex_rank)),
     "entropy_digits_msb_first": dict(entropy_pack=_entropy_pack_with(digit_order=-1)),
     "entropy_bits_undersized": dict(entropy_group_bits=lambda n, m: O.entropy_group_bits(n, m) - 1),
+    "ste_dx_no_gamma": dict(ste_grad_x=ste_dx_no_gamma),
+    "ste_dx_transposed": dict(ste_grad_x=ste_dx_transposed),
+    "ste_dx_sign_flip": dict(ste_grad_x=ste_dx_sign_flip),
+    "ste_dw_no_127": dict(ste_grad_w=ste_dw_no_127),
+    "ste_dw_unscaled": dict(ste_grad_w=ste_dw_unscaled),
+    "ste_dw_transposed_dy": dict(ste_grad_w=ste_dw_transposed_dy),
 }
 
 
@@ -263,6 +296,11 @@ def all_pins(impl):
         ("entropy_accounting", lambda: pins.check_entropy_accounting(impl)),
         ("entropy_hand", lambda: pins.check_entropy_hand(impl)),
         ("entropy_bijection", lambda: pins.check_entropy_bijection(impl)),
+        ("ste_dx_exact", lambda: pins.check_ste_grad_x_exact(impl)),
+        ("ste_dw_exact", lambda: pins.check_ste_grad_w_exact(impl)),
+        ("ste_one_hot", lambda: pins.check_ste_one_hot(impl)),
+        ("ste_finite_difference", lambda: pins.check_ste_finite_difference(impl)),
+        ("ste_forward", lambda: pins.check_ste_matches_forward(impl, small["w"], small["x"], 2, 4)),
     ]
     failed = []
     for name, fn in checks:
