@@ -339,6 +339,37 @@ sbn_status sbn_bitlinear_entropy_x(const void* x_bf16, int32_t t, int32_t k,
 size_t sbn_bitlinear_entropy_x_workspace_bytes(int32_t t, int32_t k);
 
 /*
+ * Backward of the layer under the straight-through estimator ("Microsoft
+ * BitNet 1.58: The Era of 1-Bit Large Language Models", section "Training
+ * with the Straight-Through Estimator": gradients cross the quantizer as the
+ * identity; the latent weights take them). The forward multiplies the
+ * dequantized activations Xd = Xq * s_t / 127 by Wd = gamma * C (C the masked
+ * ternary codes), so with dY = dL/dY [t, n_out] (device, bf16, row-major,
+ * 16-byte aligned):
+ *
+ * sbn_bitlinear_grad_x -- dX = dY * (gamma C), [t, k] bf16 written to dx_bf16
+ *   (device, 16-byte aligned). codes, meta, gamma as written by
+ *   sbn_quantize_weights for (n_out, k, n, m). fp32 accumulation, one bf16
+ *   rounding.
+ * sbn_bitlinear_grad_w -- dW = dY^T * (Xq s / 127), [n_out, k] bf16 written
+ *   to dw_bf16 (device, 16-byte aligned): the gradient of every latent
+ *   weight, pruned positions included. xq [t, k] int8 and x_scale [t] fp32
+ *   as written by sbn_quantize_acts for the forward's X. fp32
+ *   accumulation, one bf16 rounding.
+ * Shapes as sbn_bitlinear (k a multiple of 128). Errors: SBN_ERR_NULL,
+ * SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN (before anything is
+ * enqueued); SBN_ERR_CUDA.
+ */
+sbn_status sbn_bitlinear_grad_x(const void* dy_bf16, int32_t t, int32_t k,
+                                int32_t n_out, int32_t n, int32_t m,
+                                const uint8_t* codes, const uint8_t* meta,
+                                const float* gamma, void* dx_bf16,
+                                void* stream);
+sbn_status sbn_bitlinear_grad_w(const void* dy_bf16, const int8_t* xq,
+                                const float* x_scale, int32_t t, int32_t k,
+                                int32_t n_out, void* dw_bf16, void* stream);
+
+/*
  * sbn_get_device_error -- synchronizes `stream`, then reads and clears the
  * device error word of the current device. Returns SBN_OK, SBN_ERR_TIMEOUT
  * (a bounded device wait gave up; the affected outputs are unspecified) or

@@ -22,6 +22,7 @@
 #include "expand_dense.cuh"
 #include "entropy.cuh"
 #include "entropy_pack.cuh"
+#include "bwd.cuh"
 #include "flip.cuh"
 #include "bl_tc.cuh"
 
@@ -562,6 +563,34 @@ size_t bitlinear_entropy_x_ws_bytes(int32_t t, int32_t k) {
   return round_up16((size_t)t * k) + round_up16((size_t)t * 4);
 }
 
+// Backward dX over the packed weights, per pattern.
+template <int MM, int CB, bool DENSE>
+sbn_status launch_bwd_dx(const uint16_t* dy, int t, int k, int n_out, const uint8_t* codes, const uint8_t* meta,
+                         int cstride, int mstride, const float* gamma, uint16_t* dx, cudaStream_t st) {
+  const dim3 grid(k / kBwTile, (t + kBwTile - 1) / kBwTile);
+  bwd_dx_kernel<MM, CB, DENSE><<<grid, kBwThreads, 0, st>>>(dy, t, k, n_out, codes, meta, cstride, mstride,
+                                                           gamma, dx);
+  return launch_status();
+}
+
+sbn_status dispatch_bwd_dx(const uint16_t* dy, int t, int k, int n_out, int n, int m, const uint8_t* codes,
+                           const uint8_t* meta, const float* gamma, uint16_t* dx, cudaStream_t st) {
+  const int cs = (int)sbn_codes_row_bytes(k, n, m), ms = (int)sbn_meta_row_bytes(k, n, m);
+  if (n == m) return launch_bwd_dx<8, 4, true>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+  switch (m * 8 + 4 * n / m) {
+    case 4 * 8 + 1: return launch_bwd_dx<4, 1, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 4 * 8 + 2: return launch_bwd_dx<4, 2, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 4 * 8 + 3: return launch_bwd_dx<4, 3, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 8 * 8 + 1: return launch_bwd_dx<8, 1, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 8 * 8 + 2: return launch_bwd_dx<8, 2, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 8 * 8 + 3: return launch_bwd_dx<8, 3, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 16 * 8 + 1: return launch_bwd_dx<16, 1, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 16 * 8 + 2: return launch_bwd_dx<16, 2, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+    case 16 * 8 + 3: return launch_bwd_dx<16, 3, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
+  }
+  return SBN_ERR_PATTERN;
+}
+
 // Resident blocks per SM of the entropy packer (its grid fills the GPU once).
 int ent_pack_blocks_per_sm(int dev, int m) {
   static int cached[kMaxDevices][3] = {};   // m = 4, 8, 16 (benign race: same value)
@@ -743,6 +772,41 @@ sbn_status sbn_bitlinear_entropy_acc32(const int8_t* xq, int32_t t, int32_t k, i
   if (!xq || !ent || !acc) return SBN_ERR_NULL;
   if (!aligned16(acc)) return SBN_ERR_ALIGN;
   return run_bitlinear_entropy<true>(xq, nullptr, t, k, n_out, n, m, ent, nullptr, nullptr, acc, stream);
+}
+
+sbn_status sbn_bitlinear_grad_x(const void* dy_bf16, int32_t t, int32_t k, int32_t n_out, int32_t n, int32_t m,
+                                const uint8_t* codes, const uint8_t* meta, const float* gamma, void* dx_bf16,
+                                void* stream) {
+  if (!dy_bf16 || !codes || !gamma || !dx_bf16 || (n != m && !meta)) return SBN_ERR_NULL;
+  if (!pattern_ok(n, m)) return SBN_ERR_PATTERN;
+  if (t < 1 || n_out < 1 || k < 128 || (k % 128) != 0) return SBN_ERR_SHAPE;
+  if (!prod_lt_2_31(t, k) || !prod_lt_2_31(n_out, k) || !prod_lt_2_31(t, n_out)) return SBN_ERR_SHAPE;
+  if ((t + kBwTile - 1) / kBwTile > 65535) return SBN_ERR_SHAPE;   // grid y
+  if (!aligned16(dy_bf16) || !aligned16(codes) || (meta && !aligned16(meta)) || !aligned16(dx_bf16) ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3u))
+    return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  return dispatch_bwd_dx(reinterpret_cast<const uint16_t*>(dy_bf16), t, k, n_out, n, m, codes, meta, gamma,
+                         reinterpret_cast<uint16_t*>(dx_bf16), reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_bitlinear_grad_w(const void* dy_bf16, const int8_t* xq, const float* x_scale, int32_t t,
+                                int32_t k, int32_t n_out, void* dw_bf16, void* stream) {
+  if (!dy_bf16 || !xq || !x_scale || !dw_bf16) return SBN_ERR_NULL;
+  if (t < 1 || n_out < 1 || k < 128 || (k % 128) != 0) return SBN_ERR_SHAPE;
+  if (!prod_lt_2_31(t, k) || !prod_lt_2_31(n_out, k) || !prod_lt_2_31(t, n_out)) return SBN_ERR_SHAPE;
+  if ((n_out + kBwTile - 1) / kBwTile > 65535) return SBN_ERR_SHAPE;   // grid y
+  if (!aligned16(dy_bf16) || !aligned16(xq) || !aligned16(dw_bf16) || (reinterpret_cast<uintptr_t>(x_scale) & 3u))
+    return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  const dim3 grid(k / kBwTile, (n_out + kBwTile - 1) / kBwTile);
+  bwd_dw_kernel<<<grid, kBwThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint16_t*>(dy_bf16), xq, x_scale, t, k, n_out, reinterpret_cast<uint16_t*>(dw_bf16));
+  return launch_status();
 }
 
 size_t sbn_bitlinear_entropy_x_workspace_bytes(int32_t t, int32_t k) {

@@ -62,6 +62,9 @@ PROTOTYPES = {
     "sbn_bitlinear_entropy_x": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
                                                _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "sbn_bitlinear_entropy_x_workspace_bytes": (_c_sz, [_c_i32, _c_i32]),
+    "sbn_bitlinear_grad_x": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p,
+                                            _c_p, _c_p]),
+    "sbn_bitlinear_grad_w": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
 
@@ -349,6 +352,38 @@ def bitlinear_entropy_x(x: torch.Tensor, ent: torch.Tensor, w: PackedWeights,
                                        _ptr(out), _ptr(out_q), _ptr(out_s), ws_ptr, ws_n,
                                        _stream_ptr(stream))
     _check(st, "sbn_bitlinear_entropy_x")
+    return out
+
+
+def grad_x(dy: torch.Tensor, w: PackedWeights, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """sbn_bitlinear_grad_x: dX = dY (gamma C) under the straight-through estimator."""
+    _need(dy, torch.bfloat16, "dy")
+    t, n_out = dy.shape
+    if n_out != w.n_out:
+        raise ValueError("N_out mismatch between dY and the weights")
+    if out is None:
+        out = torch.empty((t, w.k), dtype=torch.bfloat16, device=dy.device)
+    st = lib().sbn_bitlinear_grad_x(_ptr(dy), t, w.k, w.n_out, w.n, w.m, _ptr(w.codes), _ptr(w.meta),
+                                    _ptr(w.gamma), _ptr(out), _stream_ptr(stream))
+    _check(st, "sbn_bitlinear_grad_x")
+    return out
+
+
+def grad_w(dy: torch.Tensor, xq: torch.Tensor, s: torch.Tensor, out: Optional[torch.Tensor] = None,
+           stream=None) -> torch.Tensor:
+    """sbn_bitlinear_grad_w: dW = dY^T (Xq s / 127) under the straight-through
+    estimator (every latent weight, pruned ones included)."""
+    _need(dy, torch.bfloat16, "dy")
+    _need(xq, torch.int8, "xq")
+    _need(s, torch.float32, "s")
+    t, n_out = dy.shape
+    if xq.shape[0] != t:
+        raise ValueError("T mismatch between dY and Xq")
+    k = xq.shape[1]
+    if out is None:
+        out = torch.empty((n_out, k), dtype=torch.bfloat16, device=dy.device)
+    st = lib().sbn_bitlinear_grad_w(_ptr(dy), _ptr(xq), _ptr(s), t, k, n_out, _ptr(out), _stream_ptr(stream))
+    _check(st, "sbn_bitlinear_grad_w")
     return out
 
 

@@ -193,3 +193,23 @@ def test_product_path_does_not_import_oracle():
         assert "import oracle" not in text and "from oracle" not in text, f
     for f in list(pkg.rglob("*.cu")) + list(pkg.rglob("*.cuh")):
         assert "oracle" not in f.read_text(), f
+
+
+def test_backward_validation(sbn_lib):
+    lib = sbn_lib
+    gx = lib.sbn_bitlinear_grad_x
+    assert gx(None, 4, 256, 64, 2, 4, A, A, A, A, None) == 1
+    assert gx(A, 4, 256, 64, 2, 4, A, None, A, A, None) == 1                # 2:4 needs meta
+    assert gx(A, 4, 256, 64, 4, 4, A, None, A, A, None) not in (1, 2, 3, 4)  # dense: no meta
+    assert gx(A, 4, 256, 64, 3, 8, A, A, A, A, None) == 3
+    assert gx(A, 4, 200, 64, 2, 4, A, A, A, A, None) == 2
+    assert gx(A, 0, 256, 64, 2, 4, A, A, A, A, None) == 2
+    assert gx(MIS, 4, 256, 64, 2, 4, A, A, A, A, None) == 4
+    assert gx(A, 4, 256, 64, 2, 4, A, A, A, MIS, None) == 4
+    gw = lib.sbn_bitlinear_grad_w
+    assert gw(A, None, A, 4, 256, 64, A, None) == 1
+    assert gw(A, A, A, 4, 100, 64, A, None) == 2
+    assert gw(A, A, A, 4, 256, 0, A, None) == 2
+    assert gw(A, A, A + 2, 4, 256, 64, A, None) == 4
+    assert gw(A, A, A, 4, 256, 64, MIS, None) == 4
+

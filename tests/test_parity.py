@@ -424,3 +424,53 @@ def test_bitlinear_entropy_x_two_step_route():
 @pytest.mark.parametrize("t", synth.DECODE_TOKENS)
 def test_bitlinear_entropy_decode_full(t):
     _entropy_decode_check(synth.decode_weights(), synth.decode_acts(t), 6, 8)
+
+
+# ---- backward (straight-through estimator) ------------------------------------
+#
+# Tolerance from the arithmetic: the kernels accumulate L products in fp32
+# (error at most L * 2^-24 of the sum of |terms|) and both sides round once to
+# bf16 (2^-9 relative each): |got - ref| <= 2^-7 |ref| + L 2^-22 sum|terms|.
+
+def _grad_close(got_bits, ref_bits, abs_terms, length):
+    g = oracle.bf16_bits_to_f32(got_bits).astype(np.float64)
+    r = oracle.bf16_bits_to_f32(ref_bits).astype(np.float64)
+    bad = np.abs(g - r) > 2.0 ** -7 * np.abs(r) + length * 2.0 ** -22 * abs_terms
+    assert not bad.any(), f"{bad.sum()} of {bad.size} off; first {np.argwhere(bad)[:3]}"
+
+
+def _grad_check(w, x, dy, n, m):
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    pw = run_quantize_weights(w, n, m)
+    xq, s = sbn.quantize_acts(to_dev_bf16(x))
+    dyd = to_dev_bf16(dy)
+    dx = sbn.grad_x(dyd, pw)
+    dw = sbn.grad_w(dyd, xq, s)
+    torch.cuda.synchronize()
+    assert sbn.get_device_error() == 0
+    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, n, m)
+    q, sc = oracle.quantize_acts(x)
+    g = np.abs(oracle.bf16_bits_to_f32(dy).astype(np.float64))
+    _grad_close(bf16_tensor_bits(dx), oracle.ste_grad_x(dy, dense, gamma),
+                g @ (np.abs(dense.astype(np.float64)) * float(gamma)), dy.shape[1])
+    xd = np.abs(q.astype(np.float64)) * (sc.astype(np.float64)[:, None] / 127.0)
+    _grad_close(bf16_tensor_bits(dw), oracle.ste_grad_w(dy, q, sc), g.T @ xd, dy.shape[0])
+
+
+@pytest.mark.parametrize("nm", SUPPORTED)
+@pytest.mark.parametrize("shape", SHAPES)
+def test_backward_grads(nm, shape):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=23, tag=f"bw{nm}{shape}")
+    x = synth.activations(t, k, seed=23, tag=f"bw{nm}{shape}", outlier_channels=2)
+    dy = synth.activations(t, n_out, seed=24, tag=f"dy{nm}{shape}")
+    _grad_check(w, x, dy, *nm)
+
+
+def test_backward_grads_decode_layer():
+    # the decode layer's weights (6912 x 2560, 6:8) with 300 tokens
+    w = synth.decode_weights()
+    x = synth.activations(300, 2560, seed=25, tag="bwfull", outlier_channels=2)
+    dy = synth.activations(300, 6912, seed=26, tag="dyfull")
+    _grad_check(w, x, dy, 6, 8)
