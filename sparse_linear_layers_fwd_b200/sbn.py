@@ -355,7 +355,8 @@ def bitlinear_entropy_x(x: torch.Tensor, ent: torch.Tensor, w: PackedWeights,
     return out
 
 
-def grad_x(dy: torch.Tensor, w: PackedWeights, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+def bitlinear_grad_x(dy: torch.Tensor, w: PackedWeights, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
     """sbn_bitlinear_grad_x: dX = dY (gamma C) under the straight-through estimator."""
     _need(dy, torch.bfloat16, "dy")
     t, n_out = dy.shape
@@ -369,8 +370,8 @@ def grad_x(dy: torch.Tensor, w: PackedWeights, out: Optional[torch.Tensor] = Non
     return out
 
 
-def grad_w(dy: torch.Tensor, xq: torch.Tensor, s: torch.Tensor, out: Optional[torch.Tensor] = None,
-           stream=None) -> torch.Tensor:
+def bitlinear_grad_w(dy: torch.Tensor, xq: torch.Tensor, s: torch.Tensor,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """sbn_bitlinear_grad_w: dW = dY^T (Xq s / 127) under the straight-through
     estimator (every latent weight, pruned ones included)."""
     _need(dy, torch.bfloat16, "dy")

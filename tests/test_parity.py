@@ -445,8 +445,8 @@ def _grad_check(w, x, dy, n, m):
     pw = run_quantize_weights(w, n, m)
     xq, s = sbn.quantize_acts(to_dev_bf16(x))
     dyd = to_dev_bf16(dy)
-    dx = sbn.grad_x(dyd, pw)
-    dw = sbn.grad_w(dyd, xq, s)
+    dx = sbn.bitlinear_grad_x(dyd, pw)
+    dw = sbn.bitlinear_grad_w(dyd, xq, s)
     torch.cuda.synchronize()
     assert sbn.get_device_error() == 0
     cb, mb, gamma, mask, dense = oracle.quantize_weights(w, n, m)
