@@ -320,13 +320,18 @@ def cores_used():
 # CPU oracle legs (the only places bench.py runs oracle/)
 # ---------------------------------------------------------------------------
 
-def oracle_step(layers_data, rows):
+def oracle_step(layers_data, rows, mode="split"):
     """One step of the oracle on the first `rows` output features of every
-    layer: quantize_weights, then quantize_acts + contraction per token set."""
+    layer: quantize_weights, then quantize_acts + contraction per token set.
+    mode "entropy": the weights are packed into the entropy-tight format and
+    the contraction reads them back from it, as the GPU step does."""
     import oracle
     for (w, xs, n, m) in layers_data:
         ws = w[:rows]
         cb, mb, gamma, mask, dense = oracle.quantize_weights(ws, n, m)
+        if mode == "entropy":
+            ent = oracle.entropy_pack(mask, dense, n, m)
+            dense, _ = oracle.entropy_unpack(ent, ws.shape[1], n, m)
         for x in xs:
             q, s = oracle.quantize_acts(x)
             acc = oracle.bitlinear_acc(q, dense)
@@ -367,18 +372,18 @@ def make_layers_data(workload, rank=0):
     return out
 
 
-def run_oracle_timed(layers, data, target_s, max_frac=1.0):
+def run_oracle_timed(layers, data, target_s, max_frac=1.0, mode="split"):
     """Time the oracle on a row sample sized for about target_s seconds."""
     frac = min(max_frac, 0.02)
     rows_of = lambda f: [max(1, int(l[0] * f)) for l in layers]  # noqa: E731
     t0 = time.perf_counter()
     for (w, xs, n, m), r in zip(data, rows_of(frac)):
-        oracle_step([(w, xs, n, m)], r)
+        oracle_step([(w, xs, n, m)], r, mode)
     dt = time.perf_counter() - t0
     frac = min(max_frac, frac * max(1.0, target_s / max(dt, 1e-3)))
     t0 = time.perf_counter()
     for (w, xs, n, m), r in zip(data, rows_of(frac)):
-        oracle_step([(w, xs, n, m)], r)
+        oracle_step([(w, xs, n, m)], r, mode)
     dt = time.perf_counter() - t0
     return frac, dt
 
@@ -650,7 +655,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        frac, dt = run_oracle_timed(layers, data, target_s=args.cpu_seconds)
+        frac, dt = run_oracle_timed(layers, data, target_s=args.cpu_seconds, mode=workload_mode(args.workload))
         cpu = {"value": round(oracle_sample_metric(args.workload, layers, frac) / dt, 6),
                "unit": WORKLOADS[args.workload]["unit"], "cores": cores_used(),
                "kind": "oracle",
@@ -753,15 +758,16 @@ def run_reference(args, rank, world):
     data = make_layers_data(args.workload, 0)
     total_steps = args.steps + args.warmup
     per_step = max(0.01, args.reference_seconds / max(1, total_steps))
-    frac, _ = run_oracle_timed(layers, data, target_s=per_step)
+    mode = workload_mode(args.workload)
+    frac, _ = run_oracle_timed(layers, data, target_s=per_step, mode=mode)
     rows = [max(1, int(l[0] * frac)) for l in layers]
     for _ in range(args.warmup):
         for d, r in zip(data, rows):
-            oracle_step([d], r)
+            oracle_step([d], r, mode)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         for d, r in zip(data, rows):
-            oracle_step([d], r)
+            oracle_step([d], r, mode)
     dt = time.perf_counter() - t0
     value = oracle_sample_metric(args.workload, layers, frac) * args.steps / dt
     unit = WORKLOADS[args.workload]["unit"]
