@@ -5,7 +5,7 @@
 // scale preserved); per-token scale as on the promptingindex page, section
 // "How ternary quantization works during training".
 //
-// One warp (K <= 3072) or one CTA of 128 threads (longer rows) per token
+// One warp (K <= 2560) or one CTA of 128 threads (longer rows) per token
 // row. The row is held in registers (MAXC 16-byte chunks per thread), so X
 // is read from HBM exactly once: max |x| (integer max of the 15 magnitude
 // bits), one IEEE division for the multiplier 127/s, then
@@ -76,7 +76,7 @@ qa_kernel(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __
   }
 }
 
-// One warp per token row (rows of kc <= 32 * MAXC chunks, K <= 3072): the
+// One warp per token row (rows of kc <= 32 * MAXC chunks, K <= 2560): the
 // row in registers, all its loads in flight at once, the maximum reduced in
 // the warp (no block barrier), and one wave of CTAs for thousands of rows.
 constexpr int kQawThreads = 128;   // small CTAs: 7 per SM at K = 2560

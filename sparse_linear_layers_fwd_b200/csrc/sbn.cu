@@ -469,7 +469,7 @@ size_t bitlinear_x_ws_bytes(int32_t t, int32_t k, int32_t n_out) {
   return round_up16((size_t)t * k) + round_up16((size_t)t * 4) + bitlinear_ws_bytes(t, k, n_out);
 }
 
-// One warp per token row up to K = 3072, else one CTA per row (qa.cuh); rows
+// One warp per token row up to K = 2560, else one CTA per row (qa.cuh); rows
 // up to 16 * 128 * 8 positions stay in registers.
 sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, float* x_scale,
                                 cudaStream_t s) {
@@ -489,14 +489,8 @@ sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, fl
     qa_warp_kernel<10><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
     return launch_status();
   }
-  if (kc <= 32 * 12) {
-    qa_warp_kernel<12><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
-    return launch_status();
-  }
-  const int need = (kc + kQaThreads - 1) / kQaThreads;
-  if (need <= 1) qa_kernel<1><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 2) qa_kernel<2><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 4) qa_kernel<4><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
+  const int need = (kc + kQaThreads - 1) / kQaThreads;   // >= 3 here
+  if (need <= 4) qa_kernel<4><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
   else if (need <= 8) qa_kernel<8><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
   else if (need <= 12) qa_kernel<12><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
   else if (need <= 16) qa_kernel<16><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
