@@ -88,3 +88,24 @@ def test_reference_arm_other_ranks_do_nothing(capsys):
 
     b.run_reference(A(), rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+def test_entropy_workload_accounting():
+    # the bench's own size formulas against the oracle's format sizes, and
+    # the oracle step of the entropy workload on a small layer
+    import oracle
+    b = _bench()
+    for (n, m) in [(2, 4), (6, 8), (8, 16), (4, 4)]:
+        for k in (128, 2560):
+            assert b.entropy_bytes(3, k, n, m) == 3 * oracle.entropy_row_bytes(k, n, m)
+            assert b.packed_bytes(3, k, n, m) == 3 * (oracle.codes_row_bytes(k, n, m) + oracle.meta_row_bytes(k, n, m))
+    layers = b.WORKLOADS["decode_entropy"]["layers"]
+    assert b.workload_mode("decode_entropy") == "entropy"
+    (n_out, k, n, m, ts) = layers[0]
+    want = b.qw_bytes(n_out, k, n, m) + b.pe_bytes(n_out, k, n, m) + sum(
+        2 * t * k + b.entropy_bytes(n_out, k, n, m) + 4 + 2 * t * n_out for t in ts)
+    assert b.step_bytes(layers, "entropy") == want
+    from sparse_linear_layers_fwd_b200 import synth
+    w = synth.latent_weights(8, 256, seed=1, tag="ent_step")
+    x = synth.activations(2, 256, seed=1, tag="ent_step")
+    b.oracle_step([(w, [x], 6, 8)], 8, "entropy")
