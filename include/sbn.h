@@ -147,6 +147,46 @@ sbn_status sbn_quantize_weights_noalloc(const void* w_bf16, int32_t n_out, int32
                                         uint8_t* meta, float* gamma, void* stream);
 
 /*
+ * N_out-sharded (column-parallel) weight quantization.
+ *
+ * gamma is one scale for the whole tensor ("BitNet b1.58: How Ternary
+ * Weights Cut LLM Memory by 82% Without Losing Accuracy", section "How
+ * ternary quantization works during training": W is divided by the mean
+ * absolute value of the weight tensor). When the rows of a layer are split
+ * across devices, each shard computes the exact gamma bins of its rows, the
+ * caller sums the bins over the shards (for example with an NCCL all-reduce of
+ * SBN_GAMMA_BINS unsigned 64-bit integers: exact and independent of the order),
+ * and each shard quantizes its rows with sbn_quantize_weights_from_bins. The
+ * concatenated shards then equal sbn_quantize_weights on the whole tensor, byte
+ * for byte, gamma included.
+ *
+ * Bins: SBN_GAMMA_BINS uint64 values B[e] with sum_e B[e] * 2^(e - 134)
+ * equal to the exact sum of |w| over the rows. The split across e is not
+ * unique, but the bins of two shards add up to bins of their union.
+ */
+#define SBN_GAMMA_BINS 256
+
+/* Exact gamma bins of w_bf16 [n_out, k] (device, read only) into bins (device,
+ * SBN_GAMMA_BINS uint64, 16-byte aligned, overwritten; cleared on `stream`
+ * first). Errors: SBN_ERR_NULL, SBN_ERR_SHAPE (k a multiple of 128), SBN_ERR_ALIGN,
+ * SBN_ERR_CUDA. */
+sbn_status sbn_gamma_bins(const void* w_bf16, int32_t n_out, int32_t k,
+                          unsigned long long* bins, void* stream);
+
+/* Mask, codes and packing of w_bf16 [n_out, k] exactly as sbn_quantize_weights,
+ * with gamma = max(fl32(fl64(S) / total_elems), 1e-5) where S is the exact sum
+ * the bins (device, read only: the sum of every shard's bins) represent and
+ * total_elems the element count of the whole tensor (n_out * k <= total_elems
+ * <= 2^36). codes,
+ * meta and gamma as in sbn_quantize_weights; no workspace. Errors: SBN_ERR_NULL,
+ * SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN, SBN_ERR_CUDA. */
+sbn_status sbn_quantize_weights_from_bins(const void* w_bf16, int32_t n_out,
+                                          int32_t k, int32_t n, int32_t m,
+                                          const unsigned long long* bins,
+                                          int64_t total_elems, uint8_t* codes,
+                                          uint8_t* meta, float* gamma, void* stream);
+
+/*
  * sbn_quantize_acts -- per-token absmax INT8 activations.
  *
  * Defining passage: "The BitLinear Layer" (octagono page), second operation:

@@ -40,6 +40,31 @@ SBN_DEVFN uint2 quant8(const uint4& v, float mult) {
   return make_uint2(p0 | (p1 << 16), p2 | (p3 << 16));
 }
 
+// The same rounding as quant_pair without the float-to-integer conversion
+// unit, for values with |x| <= s (x from the row whose maximum magnitude is
+// s, mult = fl32(127 / s)): then |fl32(x * mult)| <= 127 * (1 + 2^-23), which
+// rounds to at most 127, so the clamp of quant_pair never acts and is left
+// out. fl32(p + 1.5 * 2^23) rounds p = fl32(x * mult) to the nearest integer
+// with ties to even (the sum lies in [2^23, 2^24), where the spacing of fp32
+// is 1, and 1.5 * 2^23 is even). The sum's bit pattern is
+// 0x4B400000 + rint(p), so its low byte is the two's-complement INT8 value;
+// four of them are gathered with byte permutes.
+SBN_DEVFN uint32_t quant4_magic(uint32_t wa, uint32_t wb, float mult) {
+  const float kMagic = 12582912.0f;
+  const float r0 = __fadd_rn(__fmul_rn(__uint_as_float(wa << 16), mult), kMagic);
+  const float r1 = __fadd_rn(__fmul_rn(__uint_as_float(wa & 0xFFFF0000u), mult), kMagic);
+  const float r2 = __fadd_rn(__fmul_rn(__uint_as_float(wb << 16), mult), kMagic);
+  const float r3 = __fadd_rn(__fmul_rn(__uint_as_float(wb & 0xFFFF0000u), mult), kMagic);
+  const uint32_t lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x0040u);
+  const uint32_t hi = __byte_perm(__float_as_uint(r2), __float_as_uint(r3), 0x0040u);
+  return __byte_perm(lo, hi, 0x5410u);
+}
+
+// Eight values of a row (16 bytes of bf16) with |x| <= s -> eight INT8 bytes.
+SBN_DEVFN uint2 quant8_magic(const uint4& v, float mult) {
+  return make_uint2(quant4_magic(v.x, v.y, mult), quant4_magic(v.z, v.w, mult));
+}
+
 SBN_DEVFN float block_absmax_scale(uint32_t amax) {
   __shared__ uint32_t s_red[kQaThreads / 32];
   amax = __reduce_max_sync(0xffffffffu, amax);

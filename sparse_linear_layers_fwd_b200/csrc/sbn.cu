@@ -16,8 +16,10 @@
 #include "qa.cuh"
 #include "qw.cuh"
 #include "qw_fused.cuh"
+#include "qw_shard.cuh"
 #include "bl_decode.cuh"
 #include "bl_decode_res.cuh"
+#include "bl_gemv.cuh"
 #include "bl_decode_ent.cuh"
 #include "expand_dense.cuh"
 #include "entropy.cuh"
@@ -217,6 +219,101 @@ sbn_status dispatch_decode_res(const DresParams& p, int n, int m, int grid, size
   return SBN_ERR_PATTERN;
 }
 
+// Decode GEMV (T <= 16): one CTA per SM, launched with programmatic
+// dependent launch so that its launch overlaps the tail of the previous
+// kernel on the stream (the kernel waits for that grid before it reads).
+template <int MM, int CB, int NT, bool DENSE, bool ACC, bool XBF>
+sbn_status launch_gemv(const GvParams& p, int grid, size_t smem, cudaStream_t st) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  auto kern = bl_gemv_kernel<MM, CB, NT, DENSE, ACC, XBF>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGvSmemMax) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  return SBN_OK;
+}
+
+template <int NT, bool ACC, bool XBF>
+sbn_status dispatch_gemv(const GvParams& p, int n, int m, int grid, size_t smem, cudaStream_t st) {
+  const int cb = 4 * n / m;
+  if (n == m) return launch_gemv<8, 4, NT, true, ACC, XBF>(p, grid, smem, st);
+  switch (m * 8 + cb) {
+    case 4 * 8 + 1: return launch_gemv<4, 1, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 4 * 8 + 2: return launch_gemv<4, 2, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 4 * 8 + 3: return launch_gemv<4, 3, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 1: return launch_gemv<8, 1, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 2: return launch_gemv<8, 2, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 8 * 8 + 3: return launch_gemv<8, 3, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 16 * 8 + 1: return launch_gemv<16, 1, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 16 * 8 + 2: return launch_gemv<16, 2, NT, false, ACC, XBF>(p, grid, smem, st);
+    case 16 * 8 + 3: return launch_gemv<16, 3, NT, false, ACC, XBF>(p, grid, smem, st);
+  }
+  return SBN_ERR_PATTERN;
+}
+
+// Grid, CTA range and shared memory of the decode GEMV; false when the shape
+// is outside it (t > 16, activation rows beyond the registers' reach, or
+// rows that do not fit in shared memory).
+bool gemv_fits(int32_t t, int32_t k, int32_t n_out, int32_t n, int32_t m, int sms, bool xbf, int* grid,
+               int* per_cta, size_t* smem) {
+  if (t < 1 || t > 16) return false;
+  // the consumer threads hold every activation chunk in registers
+  const long long chunks = (long long)t * (xbf ? k / 8 : k / 16);
+  if (chunks > (long long)kGvConsumers * kGvMaxChunks) return false;
+  const int cstride = (int)sbn_codes_row_bytes(k, n, m);
+  const int mstride = (int)sbn_meta_row_bytes(k, n, m);
+  const int tiles = (n_out + 15) / 16;
+  *grid = std::min(sms, tiles);
+  *per_cta = (tiles + *grid - 1) / *grid;
+  const GvLayout L = gv_layout(*per_cta, t <= 8 ? 8 : 16, t, k, cstride, mstride, n == m);
+  *smem = L.total;
+  return *per_cta <= kGvMaxTiles && L.total <= kGvSmemMax;
+}
+
+// One launch of the decode GEMV. XBF: bf16 activations xbf, quantized in the
+// kernel (optional copies to xq_out, xs_out); else xq, xs.
+template <bool ACC, bool XBF>
+sbn_status run_gemv(const int8_t* xq, const float* xs, const uint16_t* xbf, int8_t* xq_out, float* xs_out,
+                    int32_t t, int32_t k, int32_t n_out, int32_t n, int32_t m, const uint8_t* codes,
+                    const uint8_t* meta, const float* gamma, uint16_t* y, int32_t* acc, int grid, int per_cta,
+                    size_t smem, cudaStream_t cs) {
+  GvParams q;
+  q.xq = xq; q.xs = xs; q.xbf = xbf; q.xq_out = xq_out; q.xs_out = xs_out;
+  q.codes = codes; q.meta = meta; q.gamma = gamma; q.y = y; q.acc_out = acc;
+  q.T = t; q.K = k; q.N = n_out;
+  q.cstride = (int)sbn_codes_row_bytes(k, n, m); q.mstride = (int)sbn_meta_row_bytes(k, n, m);
+  q.tiles_per_cta = per_cta;
+  const int tiles = (n_out + 15) / 16;
+  q.tile_base = tiles / grid;
+  q.tile_rem = tiles % grid;
+  q.L = gv_layout(per_cta, t <= 8 ? 8 : 16, t, k, q.cstride, q.mstride, n == m);
+  return t <= 8 ? dispatch_gemv<8, ACC, XBF>(q, n, m, grid, smem, cs)
+                : dispatch_gemv<16, ACC, XBF>(q, n, m, grid, smem, cs);
+}
+
 // Decode contraction over entropy-tight weights (patterns with m = 4 or 8).
 template <int MM, int CB, int NT, bool ACC, bool XBF>
 sbn_status launch_decode_ent(const DresParams& p, int grid, size_t smem, cudaStream_t st) {
@@ -385,6 +482,11 @@ sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k
   const int cstride = (int)sbn_codes_row_bytes(k, n, m);
   const int mstride = (int)sbn_meta_row_bytes(k, n, m);
   if (t <= 16) {
+    int ggrid = 0, gper = 0;
+    size_t gsmem = 0;
+    if (gemv_fits(t, k, n_out, n, m, sms, false, &ggrid, &gper, &gsmem))
+      return run_gemv<ACC_OUT, false>(xq, xs, nullptr, nullptr, nullptr, t, k, n_out, n, m, codes, meta, gamma,
+                                      y, acc, ggrid, gper, gsmem, st);
     // resident kernel when the largest CTA's rows and Xq fit in shared memory
     const int tiles = (n_out + 15) / 16;
     const int grid = std::min(sms, tiles);
@@ -583,6 +685,23 @@ sbn_status dispatch_bwd_dx(const uint16_t* dy, int t, int k, int n_out, int n, i
     case 16 * 8 + 3: return launch_bwd_dx<16, 3, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
   }
   return SBN_ERR_PATTERN;
+}
+
+// Grid of the shard kernels: at most two waves of 512-thread CTAs.
+int shard_grid(long long work_items, int sms) {
+  const long long want = (work_items + kQbThreads - 1) / kQbThreads;
+  return (int)std::max(1LL, std::min(want, (long long)sms * 4));
+}
+
+template <int M>
+sbn_status launch_qw_from_bins(const uint16_t* w, int n_out, int k, int n, const unsigned long long* bins,
+                               long long n_elems, uint8_t* codes, uint8_t* meta, float* gamma, int sms,
+                               cudaStream_t st) {
+  const int cstride = (int)sbn_codes_row_bytes(k, n, M);
+  const int mstride = (int)sbn_meta_row_bytes(k, n, M);
+  qw_from_bins_kernel<M><<<shard_grid((long long)n_out * (k / 16), sms), kQbThreads, 0, st>>>(
+      w, n_out, k, n, bins, n_elems, codes, cstride, meta, mstride, gamma);
+  return launch_status();
 }
 
 // Resident blocks per SM of the entropy packer (its grid fills the GPU once).
@@ -865,6 +984,10 @@ sbn_status sbn_bitlinear_x(const void* x_bf16, int32_t t, int32_t k, int32_t n_o
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int grid = 0, per_cta = 0;
   size_t smem = 0;
+  if (gemv_fits(t, k, n_out, n, m, sms, true, &grid, &per_cta, &smem))
+    return run_gemv<false, true>(nullptr, nullptr, reinterpret_cast<const uint16_t*>(x_bf16), xq, x_scale, t, k,
+                                 n_out, n, m, codes, meta, gamma, reinterpret_cast<uint16_t*>(y_bf16), nullptr,
+                                 grid, per_cta, smem, cs);
   if (fused_decode_fits(t, k, n_out, n, m, sms, &grid, &per_cta, &smem)) {
     DresParams q;
     q.xq = nullptr; q.xs = nullptr; q.xbf = reinterpret_cast<const uint16_t*>(x_bf16);
@@ -952,6 +1075,46 @@ sbn_status sbn_quantize_weights_noalloc(const void* w_bf16, int32_t n_out, int32
   return launch_quantize_weights(reinterpret_cast<const uint16_t*>(w_bf16), n_out, k, n, m, codes,
                                  meta, gamma, reinterpret_cast<unsigned char*>(g_noalloc_ptr[dev]), sms,
                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_gamma_bins(const void* w_bf16, int32_t n_out, int32_t k, unsigned long long* bins,
+                          void* stream) {
+  if (!w_bf16 || !bins) return SBN_ERR_NULL;
+  if (n_out < 1 || k < 128 || (k % 128) != 0 || !prod_lt_2_31(n_out, k)) return SBN_ERR_SHAPE;
+  if (!aligned16(w_bf16) || !aligned16(bins)) return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(bins, 0, SBN_GAMMA_BINS * sizeof(unsigned long long), s) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  const long long chunks = (long long)n_out * k / 8;
+  gamma_bins_kernel<<<shard_grid(chunks, sms), kQbThreads, 0, s>>>(reinterpret_cast<const uint4*>(w_bf16), chunks,
+                                                                  bins);
+  return launch_status();
+}
+
+sbn_status sbn_quantize_weights_from_bins(const void* w_bf16, int32_t n_out, int32_t k, int32_t n, int32_t m,
+                                          const unsigned long long* bins, int64_t total_elems, uint8_t* codes,
+                                          uint8_t* meta, float* gamma, void* stream) {
+  if (!w_bf16 || !bins || !codes || !gamma || (n != m && !meta)) return SBN_ERR_NULL;
+  sbn_status st = validate_weights_shape(n_out, k, n, m);
+  if (st != SBN_OK) return st;
+  if (total_elems < (int64_t)n_out * k || total_elems > (1ll << 36)) return SBN_ERR_SHAPE;
+  if (!aligned16(w_bf16) || !aligned16(bins) || !aligned16(codes) || (meta && !aligned16(meta)) ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3u))
+    return SBN_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  if ((st = check_device(&dev, &sms)) != SBN_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t* w = reinterpret_cast<const uint16_t*>(w_bf16);
+  switch (m) {
+    case 4: return launch_qw_from_bins<4>(w, n_out, k, n, bins, total_elems, codes, meta, gamma, sms, s);
+    case 8: return launch_qw_from_bins<8>(w, n_out, k, n, bins, total_elems, codes, meta, gamma, sms, s);
+    default: return launch_qw_from_bins<16>(w, n_out, k, n, bins, total_elems, codes, meta, gamma, sms, s);
+  }
 }
 
 sbn_status sbn_get_device_error(void* stream) {

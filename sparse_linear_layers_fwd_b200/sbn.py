@@ -42,6 +42,9 @@ PROTOTYPES = {
                                             _c_p, _c_p, _c_sz, _c_p]),
     "sbn_quantize_weights_noalloc": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
                                                     _c_p, _c_p, _c_p]),
+    "sbn_gamma_bins": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_p, _c_p]),
+    "sbn_quantize_weights_from_bins": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
+                                                      ctypes.c_int64, _c_p, _c_p, _c_p, _c_p]),
     "sbn_quantize_acts": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p]),
     "sbn_bitlinear": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p,
                                      _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
@@ -184,6 +187,41 @@ def quantize_weights_noalloc(w: torch.Tensor, n: int, m: int, out: PackedWeights
     st = lib().sbn_quantize_weights_noalloc(_ptr(w), n_out, k, n, m, _ptr(out.codes),
                                             _ptr(out.meta), _ptr(out.gamma), _stream_ptr(stream))
     _check(st, "sbn_quantize_weights_noalloc")
+    return out
+
+
+GAMMA_BINS = 256   # SBN_GAMMA_BINS
+
+
+def gamma_bins(w: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """sbn_gamma_bins: the exact gamma bins of one shard of rows, as int64 [256]
+    (the bit patterns of the library's uint64 bins; every value stays below
+    2^63). Bins of several shards add up to the bins of their union, so a
+    column-parallel layer sums them with an all-reduce before quantizing."""
+    _need(w, torch.bfloat16, "w")
+    n_out, k = w.shape
+    if out is None:
+        out = torch.empty((GAMMA_BINS,), dtype=torch.int64, device=w.device)
+    _need(out, torch.int64, "bins")
+    st = lib().sbn_gamma_bins(_ptr(w), n_out, k, _ptr(out), _stream_ptr(stream))
+    _check(st, "sbn_gamma_bins")
+    return out
+
+
+def quantize_weights_from_bins(w: torch.Tensor, n: int, m: int, bins: torch.Tensor, total_elems: int,
+                               out: Optional[PackedWeights] = None, stream=None) -> PackedWeights:
+    """sbn_quantize_weights_from_bins: mask, codes and packing of one shard of
+    rows with the gamma of the whole tensor (bins summed over all shards,
+    total_elems the element count of the whole tensor)."""
+    _need(w, torch.bfloat16, "w")
+    _need(bins, torch.int64, "bins")
+    n_out, k = w.shape
+    if out is None:
+        out = alloc_packed(n_out, k, n, m, w.device)
+    st = lib().sbn_quantize_weights_from_bins(_ptr(w), n_out, k, n, m, _ptr(bins), int(total_elems),
+                                              _ptr(out.codes), _ptr(out.meta), _ptr(out.gamma),
+                                              _stream_ptr(stream))
+    _check(st, "sbn_quantize_weights_from_bins")
     return out
 
 

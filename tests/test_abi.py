@@ -82,6 +82,30 @@ def test_quantize_weights_validation(sbn_lib):
     assert qw(lib, wsb=100) == 5
 
 
+def test_sharded_quantization_validation(sbn_lib):
+    lib = sbn_lib
+    assert lib.sbn_gamma_bins(None, 64, 256, A, None) == 1
+    assert lib.sbn_gamma_bins(A, 64, 256, None, None) == 1
+    assert lib.sbn_gamma_bins(A, 64, 200, A, None) == 2
+    assert lib.sbn_gamma_bins(A, 0, 256, A, None) == 2
+    assert lib.sbn_gamma_bins(MIS, 64, 256, A, None) == 4
+    assert lib.sbn_gamma_bins(A, 64, 256, MIS, None) == 4
+
+    def fb(**kw):
+        a = dict(w=A, n_out=64, k=256, n=6, m=8, bins=A, total=64 * 256 * 4, codes=A, meta=A, g=A)
+        a.update(kw)
+        return lib.sbn_quantize_weights_from_bins(a["w"], a["n_out"], a["k"], a["n"], a["m"], a["bins"],
+                                                  a["total"], a["codes"], a["meta"], a["g"], None)
+    assert fb(bins=None) == 1
+    assert fb(meta=None) == 1
+    assert fb(n=5) == 3
+    assert fb(k=200) == 2
+    assert fb(total=64 * 256 - 1) == 2          # fewer elements than the shard itself
+    assert fb(total=(1 << 36) + 1) == 2
+    assert fb(bins=MIS) == 4
+    assert fb(codes=MIS) == 4
+
+
 def test_quantize_acts_validation(sbn_lib):
     lib = sbn_lib
     assert lib.sbn_quantize_acts(None, 4, 256, A, A, None) == 1

@@ -79,6 +79,7 @@ def _fused_check(w, x, n, m):
     y2 = sbn.bitlinear_x(xd, pw)
     torch.cuda.synchronize()
     assert np.array_equal(bf16_tensor_bits(y2), bf16_tensor_bits(y))
+    return bf16_tensor_bits(y)
 
 
 @pytest.mark.parametrize("nm", SUPPORTED)
@@ -88,6 +89,22 @@ def test_fused_act_quant_contraction(nm, shape):
     w = synth.latent_weights(n_out, k, seed=14, tag=f"fx{nm}{shape}")
     x = synth.activations(t, k, seed=14, tag=f"fx{nm}{shape}", outlier_channels=2)
     _fused_check(w, x, *nm)
+
+
+# decode GEMV: token counts on both sides of 8, ragged row tiles, K with a
+# half 256-position item at the end, and rows spread over many CTAs
+GEMV_SHAPES = [(9, 640, 50), (16, 1152, 33), (3, 2560, 200), (8, 256, 16), (12, 384, 4099)]
+
+
+@pytest.mark.parametrize("nm", SUPPORTED)
+@pytest.mark.parametrize("shape", GEMV_SHAPES)
+def test_gemv_shapes(nm, shape):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=21, tag=f"gv{nm}{shape}")
+    x = synth.activations(t, k, seed=21, tag=f"gv{nm}{shape}", outlier_channels=2)
+    g = full_parity(w, x, *nm)
+    # the fused route multiplies the same accumulators by the same scales
+    assert np.array_equal(_fused_check(w, x, *nm), g["y"])
 
 
 @pytest.mark.parametrize("t", synth.DECODE_TOKENS)
