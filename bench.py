@@ -2,30 +2,49 @@
 """Benchmark of the Sparse-BitNet BitLinear forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|decode_entropy]
+                    [--workload decode|decode_entropy|prefill|qwen05b|layer_small]
+                    [--only]
 
-One step is one pass of the whole path over one batch of synthetic input:
-sbn_quantize_weights on the latent weights (the dynamic N:M mask is
-recomputed every forward), then, for every token set, the activation
-quantization and the contraction: sbn_bitlinear_x (fused) for the decode
-workload, sbn_quantize_acts + sbn_bitlinear for prefill. The default workload
-is the decode GEMV sweep: W [6912, 2560] bf16 ~ N(0, 0.02), 6:8, activations
-of T = 1, 4 and 16 tokens. The prefill workload is T = 4096 through
-(K, N_out) = (2560, 6912) and (6912, 2560) at 2:4. decode_entropy is the
-decode sweep over the entropy-tight weight format (sbn_pack_entropy +
-sbn_bitlinear_entropy_x). The other shapes of the pages' workloads are
-covered by the parity tests.
+One step is one pass of the whole path over one batch of synthetic input.
+The headline workload (default: decode) is the decode GEMV sweep:
+sbn_quantize_weights on the latent weights W [6912, 2560] bf16 ~ N(0, 0.02)
+(the dynamic 6:8 mask is recomputed every forward), then sbn_bitlinear_x
+(activation quantization fused into the contraction) for T = 1, 4 and 16
+tokens. With N = 1 and without --only, the same JSON line also carries, under
+"workloads", every other configuration of the method's workloads, each with
+its own roofline, CPU baseline and end-to-end figure:
 
-Timing: each step is a captured CUDA graph; steps rotate over enough
-distinct copies of the inputs and outputs that their total exceeds 3x the
-L2 cache, so no step reads another step's data from L2. An untimed
-calibration replay with events around every call gives the per-call
-breakdown; the timed replays bracket only the dominant call. The timed region is
-K graph replays bracketed by barrier + synchronize, timed with CUDA events;
-for N > 1 the max over ranks is taken and every rank runs its own
-independent layer (weak scaling, no collective on the data path).
+* prefill      T = 4096 through (K, N_out) = (2560, 6912) and (6912, 2560) at
+               2:4: quantize_weights, then quantize_acts + bitlinear per layer;
+* qwen05b      the 24-layer Qwen2.5-0.5B-shaped stack (168 projections, hidden
+               896, intermediate 4864), T = 2048, 6:8, weights packed once,
+               quantize_acts + bitlinear per projection; tokens/s;
+* ffn3b        the 3B-scale FFN sweep: gate (K 2048, N_out 11008) and down
+               (K 11008, N_out 2048), T in {1, 64, 512, 8192} x n:m in
+               {2:4, 4:8, 6:8, 8:16, 8:8}; each entry's contraction and
+               activation quantization timed, and sbn_quantize_weights (the
+               per-step dynamic mask) timed separately per pattern;
+* layer_small  T = 16, K = N_out = 256, 2:4: latency of the three calls.
 
-Rank 0 prints one JSON line.
+Timing. Every step is a captured CUDA graph. Steps rotate over R copies of
+their inputs, with R such that the inputs of R steps exceed 3x the L2 cache
+(queried from the device), so no step finds another step's inputs in L2.
+The timed region is P passes of K graph replays, each pass bracketed by a
+barrier and a synchronize and timed with CUDA events on the graph's stream;
+the reported step time is the median pass (the max over ranks of each pass
+for N > 1). Per-call durations come from per-kind graphs that launch every
+call of one kind back to back over all R slots (events around the whole
+replay, not around each call: an event pair around a single launch costs
+several microseconds of its own); the kind with the largest time per step is
+the dominant kernel, whose algorithmic bytes or operations over its measured
+duration give the roofline line. The clocks are sampled during the timed
+region. `e2e` times the same step through the public binding from pinned
+host buffers (inputs copied in, outputs copied out, every step).
+
+The reference arm (--impl reference) is the CPU oracle, timed on the host
+cores with BLAS limited to one thread, on a bounded sample of the same
+workload. For N > 1 every rank runs its own independent layer (weak
+scaling, no collective on the data path); rank 0 prints one JSON line.
 """
 
 from __future__ import annotations
@@ -47,7 +66,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "BitLinear TOPS (prefill) and weight GB/s (decode) vs B200 roofline; tokens/s"
-L2_BYTES = 126 * 1024 * 1024
+L2_FALLBACK_BYTES = 126 * 1024 * 1024
+DATA_DESC = "synthetic (seeded: W ~ N(0,0.02) bf16, X ~ N(0,1) bf16)"
+DTYPE = "int8xternary->int32, bf16 io"
 
 
 # ---------------------------------------------------------------------------
@@ -115,25 +136,56 @@ def bl_ops(t, k, n_out, n, m):
     return 2 * t * k * n_out * n // m
 
 
+def _qwen_layers():
+    from sparse_linear_layers_fwd_b200 import synth
+    return [(n_out, k, 6, 8, [2048]) for _layer in range(24) for (_p, k, n_out) in synth.QWEN05B_PROJ]
+
+
 WORKLOADS = {
-    # name: list of layers (n_out, k, n, m, [token counts]) in one step
+    # name: list of layers (n_out, k, n, m, [token counts]) in one step; mode:
+    # "fused" (sbn_bitlinear_x), "split" (quantize_acts + bitlinear),
+    # "entropy" (pack_entropy + bitlinear_entropy_x); qw: the step quantizes
+    # the latent weights (else they are packed once, outside the step)
     "decode": dict(desc="decode GEMV sweep: K=2560, N_out=6912, 6:8, T in {1,4,16}; value = "
                         "algorithmic bytes of the step / step time; activation quantization "
                         "fused into the contraction (sbn_bitlinear_x)",
-                   unit="GB/s", fused=True, layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
+                   unit="GB/s", mode="fused", qw=True, layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
     "decode_entropy": dict(desc="decode GEMV sweep over entropy-tight weights: K=2560, N_out=6912, "
                                 "6:8, T in {1,4,16}; each step packs the quantized layer into the "
                                 "entropy-tight format (1.875 bit/weight) and contracts from it",
-                           unit="GB/s", mode="entropy", layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
+                           unit="GB/s", mode="entropy", qw=True, layers=[(6912, 2560, 6, 8, [1, 4, 16])]),
     "prefill": dict(desc="prefill GEMM: T=4096, (K,N_out)=(2560,6912) and (6912,2560), 2:4; value = "
                          "algorithmic ops (2 per kept multiply-add) of the step / step time",
-                    unit="TOPS", layers=[(6912, 2560, 2, 4, [4096]), (2560, 6912, 2, 4, [4096])]),
+                    unit="TOPS", mode="split", qw=True,
+                    layers=[(6912, 2560, 2, 4, [4096]), (2560, 6912, 2, 4, [4096])]),
+    "qwen05b": dict(desc="24-layer Qwen2.5-0.5B-shaped stack: 168 BitLinear projections (hidden 896, "
+                         "intermediate 4864), T=2048, 6:8, weights packed once; per projection "
+                         "quantize_acts + bitlinear; value = tokens / step time",
+                    unit="tokens/s", mode="split", qw=False, layers=None),
+    "layer_small": dict(desc="single BitLinear T=16, K=N_out=256, 2:4: latency of quantize_weights + "
+                             "quantize_acts + bitlinear",
+                        unit="us", mode="split", qw=True, layers=[(256, 256, 2, 4, [16])]),
 }
+EXTRA_WORKLOADS = ["prefill", "qwen05b", "ffn3b", "layer_small"]
+
+
+def workload_layers(workload):
+    layers = WORKLOADS[workload]["layers"]
+    return _qwen_layers() if layers is None else layers
+
+
+def is_fused(workload: str) -> bool:
+    """Whether the workload's steps use sbn_bitlinear_x (act-quant fused)."""
+    return WORKLOADS[workload]["mode"] == "fused"
+
+
+def workload_mode(workload: str):
+    """"fused", "entropy" or "split" (quantize_acts + bitlinear)."""
+    return WORKLOADS[workload]["mode"]
 
 
 def act_bytes(t, k, n_out, n, m, mode):
-    """Bytes of one token set after the weights are packed (mode: True or
-    "fused", False or "split", "entropy")."""
+    """Bytes of one token set after the weights are packed."""
     if mode is True or mode == "fused":
         return blx_bytes(t, k, n_out, n, m)
     if mode == "entropy":
@@ -141,10 +193,11 @@ def act_bytes(t, k, n_out, n, m, mode):
     return qa_bytes(t, k) + bl_bytes(t, k, n_out, n, m)
 
 
-def step_bytes(layers, mode=False):
+def step_bytes(layers, mode=False, qw=True):
     b = 0
     for (n_out, k, n, m, ts) in layers:
-        b += qw_bytes(n_out, k, n, m)
+        if qw:
+            b += qw_bytes(n_out, k, n, m)
         if mode == "entropy":
             b += pe_bytes(n_out, k, n, m)
         for t in ts:
@@ -160,19 +213,25 @@ def step_ops(layers):
     return sum(bl_ops(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
 
 
-# ---------------------------------------------------------------------------
-# across ranks (one process per GPU, each on its own independent layer)
-# ---------------------------------------------------------------------------
-
-def is_fused(workload: str) -> bool:
-    """Whether the workload's steps use sbn_bitlinear_x (act-quant fused)."""
-    return bool(WORKLOADS[workload].get("fused", False))
-
-
-def workload_mode(workload: str):
-    """"fused", "entropy" or "split" (quantize_acts + bitlinear)."""
+def step_units(workload, layers):
+    """Units of one step in the workload's unit (GB, T-ops, tokens or a step)."""
+    unit = WORKLOADS[workload]["unit"]
+    if unit == "TOPS":
+        return step_ops(layers) / 1e12
+    if unit == "tokens/s":
+        return layers[0][4][0]          # one pass of T tokens through the stack
+    if unit == "us":
+        return 1.0
     w = WORKLOADS[workload]
-    return w.get("mode", "fused" if w.get("fused") else "split")
+    return step_bytes(layers, w["mode"], w["qw"]) / 1e9
+
+
+def rate(workload, layers, steps, world, ms):
+    """Whole-job value: units of all ranks over the slowest rank's time (for
+    "us", the step latency instead)."""
+    if WORKLOADS[workload]["unit"] == "us":
+        return ms * 1e3 / steps
+    return step_units(workload, layers) * steps * world / (ms * 1e-3)
 
 
 def max_over_ranks(ms: float, world: int, device) -> float:
@@ -189,10 +248,52 @@ def max_over_ranks(ms: float, world: int, device) -> float:
 def whole_job_value(workload: str, steps: int, world: int, ms_max: float) -> float:
     """Units processed by all ranks (weak scaling: each rank runs a full step
     on its own layer) over the slowest rank's time, in the workload's unit."""
-    layers = WORKLOADS[workload]["layers"]
-    if WORKLOADS[workload]["unit"] == "TOPS":
-        return step_ops(layers) * steps * world / (ms_max * 1e-3) / 1e12
-    return step_bytes(layers, workload_mode(workload)) * steps * world / (ms_max * 1e-3) / 1e9
+    return rate(workload, workload_layers(workload), steps, world, ms_max)
+
+
+# the calls of one step, in order: (kind, layer, token count)
+def step_calls(workload, layers=None):
+    layers = layers if layers is not None else workload_layers(workload)
+    w = WORKLOADS[workload]
+    calls = []
+    for li, (n_out, k, n, m, ts) in enumerate(layers):
+        if w["qw"]:
+            calls.append(("quantize_weights", li, None))
+        if w["mode"] == "entropy":
+            calls.append(("pack_entropy", li, None))
+        for t in ts:
+            if w["mode"] == "entropy":
+                calls.append(("bitlinear_entropy_x", li, t))
+            elif w["mode"] == "fused":
+                calls.append(("bitlinear_x", li, t))
+            else:
+                calls.append(("quantize_acts", li, t))
+                calls.append(("bitlinear", li, t))
+    return calls
+
+
+def call_bytes(kind, layer, t):
+    n_out, k, n, m, _ = layer
+    return {"quantize_weights": lambda: qw_bytes(n_out, k, n, m),
+            "pack_entropy": lambda: pe_bytes(n_out, k, n, m),
+            "quantize_acts": lambda: qa_bytes(t, k),
+            "bitlinear": lambda: bl_bytes(t, k, n_out, n, m),
+            "bitlinear_x": lambda: blx_bytes(t, k, n_out, n, m),
+            "bitlinear_entropy_x": lambda: blex_bytes(t, k, n_out, n, m)}[kind]()
+
+
+def call_ops(kind, layer, t):
+    n_out, k, n, m, _ = layer
+    return bl_ops(t, k, n_out, n, m) if kind.startswith("bitlinear") else 0
+
+
+def call_launches(kind, t):
+    """Kernels of one call: the contraction over T > 16 tokens adds the weight expansion."""
+    return 2 if kind == "bitlinear" and t > 16 else 1
+
+
+def tensor_bound(kind, t):
+    return kind == "bitlinear" and t is not None and t > 16
 
 
 # ---------------------------------------------------------------------------
@@ -214,10 +315,9 @@ def load_peaks():
 # stays valid while these files are unchanged
 TRAFFIC_FILES = {
     "quantize_weights": ["qw_fused.cuh", "qw.cuh", "async.cuh", "common.cuh"],
-    "bitlinear_x": ["bl_decode_res.cuh", "bl_decode.cuh", "expand.cuh", "qa.cuh", "common.cuh"],
+    "quantize_acts": ["qa.cuh", "common.cuh"],
+    "bitlinear_x": ["bl_gemv.cuh", "bl_decode.cuh", "expand.cuh", "qa.cuh", "async.cuh", "common.cuh"],
     "bitlinear": ["bl_tc.cuh", "expand_dense.cuh", "expand.cuh", "async.cuh", "common.cuh"],
-    "bitlinear_entropy": ["bl_decode_ent.cuh", "bl_decode_res.cuh", "bl_decode.cuh", "entropy.cuh",
-                          "expand.cuh", "common.cuh"],
     "bitlinear_entropy_x": ["bl_decode_ent.cuh", "bl_decode_res.cuh", "bl_decode.cuh", "entropy.cuh",
                             "expand.cuh", "qa.cuh", "common.cuh"],
     "pack_entropy": ["entropy_pack.cuh", "entropy.cuh", "common.cuh"],
@@ -259,7 +359,6 @@ class ClockSampler:
         self.gpu = gpu_index
         self.period = period_ms
         self.proc = None
-        self.t0 = self.t1 = None
 
     def start(self):
         self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
@@ -271,9 +370,6 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
         time.sleep(0.3)
-
-    def mark(self, which):
-        setattr(self, which, time.time())
 
     def stop(self):
         if self.proc is None:
@@ -306,14 +402,16 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def cores_used():
+def oracle_threads_one():
+    """Context that limits BLAS to one thread (the oracle's numpy code is
+    otherwise single-threaded), so that the CPU baseline's core count is
+    exactly 1."""
     try:
         import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        blas = max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
-        return int(blas)
+        return threadpoolctl.threadpool_limits(limits=1)
     except Exception:  # noqa: BLE001
-        return 1
+        import contextlib
+        return contextlib.nullcontext()
 
 
 # ---------------------------------------------------------------------------
@@ -338,468 +436,638 @@ def oracle_step(layers_data, rows, mode="split"):
             oracle.dequant_bf16(acc, s, gamma)
 
 
-def oracle_sample_bytes(layers, rows_frac, fused=False):
-    tot = 0
-    for (n_out, k, n, m, ts) in layers:
-        r = max(1, int(n_out * rows_frac))
-        tot += qw_bytes(r, k, n, m)
-        for t in ts:
-            tot += act_bytes(t, k, r, n, m, fused)
-        if fused == "entropy":
-            tot += pe_bytes(r, k, n, m)
-    return tot
-
-
-def oracle_sample_metric(workload, layers, rows_frac):
-    """The sample's amount of work in the workload's unit (GB or T-ops)."""
-    if WORKLOADS[workload]["unit"] == "TOPS":
-        tot = 0
-        for (n_out, k, n, m, ts) in layers:
-            r = max(1, int(n_out * rows_frac))
-            tot += sum(bl_ops(t, k, r, n, m) for t in ts)
-        return tot / 1e12
-    return oracle_sample_bytes(layers, rows_frac, workload_mode(workload)) / 1e9
-
-
-def make_layers_data(workload, rank=0):
+def make_layers_data(workload, rank=0, layers=None, first=None):
+    """Seeded inputs of the workload's layers (the first `first` layers only
+    when given): (w bits, [x bits per token set], n, m)."""
     from sparse_linear_layers_fwd_b200 import synth
+    layers = layers if layers is not None else workload_layers(workload)
     out = []
-    for li, (n_out, k, n, m, ts) in enumerate(WORKLOADS[workload]["layers"]):
+    for li, (n_out, k, n, m, ts) in enumerate(layers[:first] if first else layers):
         tag = f"bench_{workload}_{li}_r{rank}"
         w = synth.latent_weights(n_out, k, seed=0, tag=tag)
-        xs = [synth.activations(t, k, seed=0, tag=f"{tag}_t{t}") for t in ts]
+        if workload == "qwen05b":
+            xs = [synth.activations(t, k, seed=0, tag=f"{tag}_t{t}",
+                                    heavy_tail_channels=synth.qwen_heavy_channels(k)) for t in ts]
+        elif workload == "layer_small":
+            xs = [synth.activations(t, k, seed=0, tag=f"{tag}_t{t}", outlier_channels=2) for t in ts]
+        else:
+            xs = [synth.activations(t, k, seed=0, tag=f"{tag}_t{t}") for t in ts]
         out.append((w, xs, n, m))
     return out
 
 
-def run_oracle_timed(layers, data, target_s, max_frac=1.0, mode="split"):
-    """Time the oracle on a row sample sized for about target_s seconds."""
-    frac = min(max_frac, 0.02)
-    rows_of = lambda f: [max(1, int(l[0] * f)) for l in layers]  # noqa: E731
-    t0 = time.perf_counter()
-    for (w, xs, n, m), r in zip(data, rows_of(frac)):
-        oracle_step([(w, xs, n, m)], r, mode)
-    dt = time.perf_counter() - t0
+def oracle_sample(workload, layers, data, target_s, max_frac=1.0):
+    """Time the oracle on a sample sized for about target_s seconds: a
+    fraction of the output rows of every layer in `data` (a prefix of the
+    workload's layers). Returns (seconds, fraction of one step's work done,
+    description)."""
+    mode = workload_mode(workload)
+    frac = min(max_frac, 0.01)
+
+    def run(f):
+        t0 = time.perf_counter()
+        for (w, xs, n, m), l in zip(data, layers):
+            oracle_step([(w, xs, n, m)], max(1, int(l[0] * f)), mode)
+        return time.perf_counter() - t0
+
+    dt = run(frac)
     frac = min(max_frac, frac * max(1.0, target_s / max(dt, 1e-3)))
-    t0 = time.perf_counter()
-    for (w, xs, n, m), r in zip(data, rows_of(frac)):
-        oracle_step([(w, xs, n, m)], r, mode)
-    dt = time.perf_counter() - t0
-    return frac, dt
+    dt = run(frac)
+    # work done relative to one full step: the contraction ops (or bytes) of
+    # the sampled rows of the sampled layers
+    def work(ls, f):
+        if WORKLOADS[workload]["unit"] in ("TOPS", "tokens/s"):
+            return sum(bl_ops(t, k, max(1, int(n_out * f)), n, m) for (n_out, k, n, m, ts) in ls for t in ts)
+        return step_bytes([(max(1, int(l[0] * f)),) + tuple(l[1:]) for l in ls], mode,
+                          WORKLOADS[workload]["qw"])
+    done = work(layers[:len(data)], frac) / work(workload_layers(workload), 1.0)
+    desc = (f"{frac:.3f} of the output features of {len(data)} of {len(workload_layers(workload))} "
+            f"layer(s), full K and all token sets; one pass, {dt:.1f} s")
+    return dt, done, desc
+
+
+def cpu_baseline(workload, target_s=10.0, first=None):
+    layers = workload_layers(workload)
+    data = make_layers_data(workload, 0, first=first)
+    with oracle_threads_one():
+        dt, done, desc = oracle_sample(workload, layers, data, target_s)
+    unit = WORKLOADS[workload]["unit"]
+    if unit == "us":
+        value = dt / done * 1e6
+    else:
+        value = step_units(workload, layers) * done / dt
+    return {"value": round(value, 6), "unit": unit, "cores": 1, "kind": "oracle", "sample": desc}
 
 
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args, rank, world, local_rank):
+def l2_bytes(dev):
+    import torch
+    try:
+        return int(torch.cuda.get_device_properties(dev).L2_cache_size) or L2_FALLBACK_BYTES
+    except Exception:  # noqa: BLE001
+        return L2_FALLBACK_BYTES
+
+
+def to_dev(bits, dev):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+class Engine:
+    """Slots of device buffers of one workload and the calls of its steps."""
+
+    def __init__(self, workload, layers, data, dev, stream, rotations):
+        import torch
+        from sparse_linear_layers_fwd_b200 import sbn
+        self.sbn = sbn
+        self.workload = workload
+        self.w = WORKLOADS[workload]
+        self.layers = layers
+        self.dev = dev
+        self.stream = stream
+        self.calls = step_calls(workload, layers)
+        base = []
+        for (w, xs, n, m), (n_out, k, _, _, ts) in zip(data, layers):
+            base.append((to_dev(w, dev), [to_dev(x, dev) for x in xs]))
+        self.slots = []
+        ws_of = {}
+        for r in range(rotations):
+            sl = []
+            for li, ((wd, xds), (n_out, k, n, m, ts)) in enumerate(zip(base, layers)):
+                L = dict(n=n, m=m)
+                L["w"] = wd if r == 0 else wd.clone()
+                L["xs"] = [x if r == 0 else x.clone() for x in xds]
+                L["pw"] = sbn.alloc_packed(n_out, k, n, m, dev)
+                L["ws"] = torch.empty(sbn.workspace_bytes(n_out, k), dtype=torch.uint8, device=dev)
+                L["qs"] = [(torch.empty((t, k), dtype=torch.int8, device=dev),
+                            torch.empty((t,), dtype=torch.float32, device=dev)) for t in ts]
+                L["ys"] = [torch.empty((t, n_out), dtype=torch.bfloat16, device=dev) for t in ts]
+                # the contraction's workspace is written and read within one
+                # call, so one per shape serves every slot
+                L["bws"] = ws_of.setdefault((n_out, k), torch.empty(
+                    (max(1, max(max(sbn.bitlinear_workspace_bytes(t, k, n_out),
+                                    sbn.bitlinear_x_workspace_bytes(t, k, n_out)) for t in ts)),),
+                    dtype=torch.uint8, device=dev))
+                L["ent"] = (torch.empty((n_out, sbn.entropy_row_bytes(k, n, m)), dtype=torch.uint8, device=dev)
+                            if self.w["mode"] == "entropy" else None)
+                sl.append(L)
+            self.slots.append(sl)
+        if not self.w["qw"]:
+            # weights packed once, outside the timed steps
+            with torch.cuda.stream(stream):
+                for sl in self.slots:
+                    for L in sl:
+                        sbn.quantize_weights(L["w"], L["n"], L["m"], out=L["pw"], workspace=L["ws"],
+                                             stream=stream)
+            stream.synchronize()
+
+    def enqueue(self, call, r):
+        kind, li, t = call
+        sbn, st = self.sbn, self.stream
+        L = self.slots[r][li]
+        ti = None if t is None else self.layers[li][4].index(t)
+        if kind == "quantize_weights":
+            sbn.quantize_weights(L["w"], L["n"], L["m"], out=L["pw"], workspace=L["ws"], stream=st)
+        elif kind == "pack_entropy":
+            sbn.pack_entropy(L["pw"], out=L["ent"], stream=st)
+        elif kind == "bitlinear_entropy_x":
+            sbn.bitlinear_entropy_x(L["xs"][ti], L["ent"], L["pw"], out=L["ys"][ti], workspace=False, stream=st)
+        elif kind == "bitlinear_x":
+            sbn.bitlinear_x(L["xs"][ti], L["pw"], out=L["ys"][ti], workspace=L["bws"], stream=st)
+        elif kind == "quantize_acts":
+            q, s = L["qs"][ti]
+            sbn.quantize_acts(L["xs"][ti], out_q=q, out_s=s, stream=st)
+        elif kind == "bitlinear":
+            q, s = L["qs"][ti]
+            sbn.bitlinear(q, s, L["pw"], out=L["ys"][ti], workspace=L["bws"], stream=st)
+        else:
+            raise ValueError(kind)
+
+    def graph(self, calls_of_slot):
+        """One CUDA graph over all slots: calls_of_slot(r) enqueued for r = 0..R-1."""
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for r in range(len(self.slots)):
+                for c in calls_of_slot(r):
+                    self.enqueue(c, r)
+        return g
+
+    def step_graphs(self):
+        import torch
+        gs = []
+        for r in range(len(self.slots)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                for c in self.calls:
+                    self.enqueue(c, r)
+            gs.append(g)
+        return gs
+
+
+def replay_ms(g, stream, reps, warmup=2):
+    """Mean milliseconds of one replay of graph g (events around reps replays)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def rotations_for(layers, workload, l2):
+    """Slots so that the inputs of R steps exceed 3x L2, at most 96."""
+    w = WORKLOADS[workload]
+    per_step = sum((2 * n_out * k if w["qw"] else packed_bytes(n_out, k, n, m)) + sum(2 * t * k for t in ts)
+                   for (n_out, k, n, m, ts) in layers)
+    return int(min(96, max(2, math.ceil(3 * l2 / per_step))))
+
+
+def kind_breakdown(eng, kinds, peaks, reps):
+    """Per kind: mean duration of one launch in back-to-back per-kind graphs
+    over all slots, its time per step and its achieved rate."""
+    out = {}
+    R = len(eng.slots)
+    for kind in kinds:
+        cs = [c for c in eng.calls if c[0] == kind]
+        g = eng.graph(lambda r: cs)
+        ms = replay_ms(g, eng.stream, reps)
+        del g
+        per_step_us = ms * 1e3 / R
+        nbytes = sum(call_bytes(c[0], eng.layers[c[1]], c[2]) for c in cs)
+        nops = sum(call_ops(c[0], eng.layers[c[1]], c[2]) for c in cs)
+        e = {"calls_per_step": len(cs), "us_per_step": round(per_step_us, 3),
+             "us_per_call": round(per_step_us / len(cs), 3),
+             "GB/s": round(nbytes / (per_step_us * 1e-6) / 1e9, 1),
+             "hbm_frac": round(nbytes / (per_step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+        if nops:
+            e["TOPS"] = round(nops / (per_step_us * 1e-6) / 1e12, 3)
+        out[kind] = e
+    return out
+
+
+def roofline_of(workload, eng, kind, per_kind, peaks, i8_peak):
+    cs = [c for c in eng.calls if c[0] == kind]
+    us = per_kind[kind]["us_per_step"]
+    tensor = all(tensor_bound(c[0], c[2]) for c in cs)
+    launches = sum(call_launches(c[0], c[2]) for c in cs)
+    if tensor:
+        ops = sum(call_ops(c[0], eng.layers[c[1]], c[2]) for c in cs)
+        dense = sum(2 * c[2] * eng.layers[c[1]][1] * eng.layers[c[1]][0] for c in cs)
+        achieved = ops / (us * 1e-6) / 1e12
+        peak, src = i8_peak
+        return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
+                "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kind, workload), "kernel": kind,
+                "ops_per_launch": ops // len(cs), "launch_us": round(us / len(cs), 3),
+                "launches_per_call": launches // len(cs), "peak_source": src,
+                "dense_equivalent_frac": round(dense / (us * 1e-6) / 1e12 / peak, 4)}
+    nbytes = sum(call_bytes(c[0], eng.layers[c[1]], c[2]) for c in cs)
+    achieved = nbytes / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": ncu_traffic(kind, workload),
+            "kernel": kind, "bytes_per_launch": nbytes // len(cs), "launch_us": round(us / len(cs), 3),
+            "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)"
+            if peaks["source"] == "measured" else "fallback 6650 GB/s"}
+
+
+def int8_peak(peaks):
+    """The INT8 dense tensor peak: the measured figure of the in-tree tcgen05
+    kind::i8 probe when it is recorded in MEASURED_PEAKS.json, else 2x the
+    measured bf16 figure (the nominal int8 : bf16 ratio), labelled as derived."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "i8_tops" in d:
+            return float(d["i8_tops"]), "measured i8_tops (in-tree tcgen05 kind::i8 probe, MEASURED_PEAKS.json)"
+    return 2.0 * peaks["bf16_tflops"], (f"derived: 2 x {peaks['source']} bf16_tflops {peaks['bf16_tflops']} "
+                                        f"(nominal int8 : bf16 ratio)")
+
+
+def run_workload(workload, args, rank, world, dev, stream, peaks, i8_peak_src, headline):
+    """Measure one workload on this rank; returns its JSON entry (rank 0)."""
     import torch
     import torch.distributed as dist
-    from sparse_linear_layers_fwd_b200 import sbn
-
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    sbn.lib()
-    layers = WORKLOADS[args.workload]["layers"]
-    data = make_layers_data(args.workload, rank)
-
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
-
-    in_bytes = sum(w.nbytes + sum(x.nbytes for x in xs) for (w, xs, _, _) in data)
-    R = max(2, math.ceil(3 * L2_BYTES / in_bytes))
-    stream = torch.cuda.Stream(device=dev)
-
-    # R rotation slots of inputs, packed weights, activations and outputs
-    slots = []
-    layer_bws = {}
-    for _ in range(R):
-        sl = []
-        for (w, xs, n, m), (n_out, k, _, _, ts) in zip(data, layers):
-            wd = to_dev(w)
-            xds = [to_dev(x) for x in xs]
-            pw = sbn.alloc_packed(n_out, k, n, m, dev)
-            ws = torch.empty(sbn.workspace_bytes(n_out, k), dtype=torch.uint8, device=dev)
-            qs = [(torch.empty((t, k), dtype=torch.int8, device=dev),
-                   torch.empty((t,), dtype=torch.float32, device=dev)) for t in ts]
-            ys = [torch.empty((t, n_out), dtype=torch.bfloat16, device=dev) for t in ts]
-            # the contraction's workspace (expanded weights, T > 16); written
-            # and read within one call, so one per layer serves every slot
-            bws = layer_bws.setdefault((n_out, k), torch.empty(
-                (max(1, max(max(sbn.bitlinear_workspace_bytes(t, k, n_out),
-                                sbn.bitlinear_x_workspace_bytes(t, k, n_out)) for t in ts)),),
-                dtype=torch.uint8, device=dev))
-            ent = (torch.empty((n_out, sbn.entropy_row_bytes(k, n, m)), dtype=torch.uint8, device=dev)
-                   if workload_mode(args.workload) == "entropy" else None)
-            sl.append(dict(w=wd, xs=xds, pw=pw, ws=ws, bws=bws, qs=qs, ys=ys, n=n, m=m, ent=ent))
-        slots.append(sl)
-
-    # per-call events inside each slot's graph: names of the calls in order
-    fused = is_fused(args.workload)
-    mode = workload_mode(args.workload)
-    call_names = []
-    for li, (n_out, k, n, m, ts) in enumerate(layers):
-        call_names.append(("quantize_weights", li, None))
-        if mode == "entropy":
-            call_names.append(("pack_entropy", li, None))
-        for t in ts:
-            if mode == "entropy":
-                call_names.append(("bitlinear_entropy_x", li, t))
-            elif fused:
-                call_names.append(("bitlinear_x", li, t))
-            else:
-                call_names.append(("quantize_acts", li, t))
-                call_names.append(("bitlinear", li, t))
-
-    def enqueue_step(sl, evs=None):
-        i = 0
-        for li, L in enumerate(sl):
-            if evs and evs[i]: evs[i][0].record(stream)
-            sbn.quantize_weights(L["w"], L["n"], L["m"], out=L["pw"], workspace=L["ws"], stream=stream)
-            if evs and evs[i]: evs[i][1].record(stream)
-            i += 1
-            if mode == "entropy":
-                if evs and evs[i]: evs[i][0].record(stream)
-                sbn.pack_entropy(L["pw"], out=L["ent"], stream=stream)
-                if evs and evs[i]: evs[i][1].record(stream)
-                i += 1
-            for x, (q, s), y in zip(L["xs"], L["qs"], L["ys"]):
-                if mode == "entropy":
-                    if evs and evs[i]: evs[i][0].record(stream)
-                    sbn.bitlinear_entropy_x(x, L["ent"], L["pw"], out=y, workspace=False, stream=stream)
-                    if evs and evs[i]: evs[i][1].record(stream)
-                    i += 1
-                    continue
-                if fused:
-                    if evs and evs[i]: evs[i][0].record(stream)
-                    sbn.bitlinear_x(x, L["pw"], out=y, workspace=L["bws"], stream=stream)
-                    if evs and evs[i]: evs[i][1].record(stream)
-                    i += 1
-                    continue
-                if evs and evs[i]: evs[i][0].record(stream)
-                sbn.quantize_acts(x, out_q=q, out_s=s, stream=stream)
-                if evs and evs[i]: evs[i][1].record(stream)
-                i += 1
-                if evs and evs[i]: evs[i][0].record(stream)
-                sbn.bitlinear(q, s, L["pw"], out=y, workspace=L["bws"], stream=stream)
-                if evs and evs[i]: evs[i][1].record(stream)
-                i += 1
-
-    def capture(which):
-        """One graph per slot; events around the calls `which` selects."""
-        gs, evss = [], []
-        for r in range(R):
-            evs = [(torch.cuda.Event(enable_timing=True, external=True),
-                    torch.cuda.Event(enable_timing=True, external=True)) if which(c) else None
-                   for c in call_names]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                enqueue_step(slots[r], evs)
-            gs.append(g)
-            evss.append(evs)
-        return gs, evss
-
+    layers = workload_layers(workload)
+    data = make_layers_data(workload, rank)
+    l2 = l2_bytes(dev)
+    R = rotations_for(layers, workload, l2)
+    eng = Engine(workload, layers, data, dev, stream, R)
     with torch.cuda.stream(stream):
-        enqueue_step(slots[0])  # load kernels before capture
+        for c in eng.calls:
+            eng.enqueue(c, 0)        # loads the kernels before capture
     stream.synchronize()
-    # calibration graphs: every call bracketed by events (per-call breakdown)
-    cal_graphs, cal_events = capture(lambda c: True)
-    # our kernels per step: quantize_weights 1 per layer; quantize_acts 1 and
-    # bitlinear 1 (+1 weight expansion when T > 16) per token set
-    # (fused: one kernel per token set for T <= 16)
-    # (entropy: + 1 pack per layer, then one fused entropy contraction per token set)
-    launches_per_step = sum(1 + (1 if mode == "entropy" else 0)
-                            + sum((1 if mode == "entropy" else
-                                   1 if fused and t <= 16 else 2 + (1 if t > 16 else 0))
-                                  for t in ts)
-                            for (_, _, _, _, ts) in layers)
+    graphs = eng.step_graphs()
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, R)):
+            graphs[i % R].replay()
+    stream.synchronize()
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    # warm-up, then one calibration replay per slot (untimed)
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            cal_graphs[i % R].replay()
-        for r in range(R):
-            cal_graphs[r].replay()
-    stream.synchronize()
-    per_call = {}
-    for r in range(R):
-        for (name, li, t), ab in zip(call_names, cal_events[r]):
-            per_call.setdefault((name, li, t), []).append(ab[0].elapsed_time(ab[1]))
-    cal_totals = {}
-    for (name, li, t), v in per_call.items():
-        cal_totals[name] = cal_totals.get(name, 0.0) + statistics.mean(v)
-    dom = max(cal_totals, key=cal_totals.get)
-    # timed graphs: events only around the dominant call (its live launch
-    # durations for the roofline), so the other calls run back to back
-    graphs, slot_events = capture(lambda c: c[0] == dom)
-    with torch.cuda.stream(stream):
-        for r in range(R):
-            graphs[r].replay()
-    stream.synchronize()
-
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    barrier()
-    torch.cuda.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for i in range(args.steps):
-            graphs[i % R].replay()
-        ev1.record(stream)
-    stream.synchronize()
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-
-    # the dominant call's durations in the last timed replay of every slot
-    used = min(R, args.steps)
-    dom_calls = {}
-    for r in range(used):
-        for (name, li, t), ab in zip(call_names, slot_events[r]):
-            if ab:
-                dom_calls.setdefault((name, li, t), []).append(ab[0].elapsed_time(ab[1]))
-
-    ms = max_over_ranks(ms, world, dev)
-
-    sb = step_bytes(layers, mode)
-    ms_per_step = ms / args.steps
-    value = whole_job_value(args.workload, args.steps, world, ms)
-
-    # dominant call (by total time in a calibration step): its time per step
-    # in the timed region
-    dom_ms = sum(statistics.mean(v) for v in dom_calls.values())
-    peaks = load_peaks()
-    n_dom_launches = len([c for c in call_names if c[0] == dom])
-    traffic = ncu_traffic(dom, args.workload)
-    tensor_bound = dom == "bitlinear" and min(t for (_, _, _, _, ts) in layers for t in ts) > 16
-    if tensor_bound:
-        # contraction on the tensor cores: algorithmic ops (2 per kept
-        # multiply-add) against the INT8 peak = measured bf16 peak x 2 (the
-        # nominal int8 : bf16 ratio of 4.5 : 2.25 POPS)
-        dom_ops = sum(bl_ops(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
-        achieved = dom_ops / (dom_ms * 1e-3) / 1e12
-        peak = 2.0 * peaks["bf16_tflops"]
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
-                    "unit": "TOPS", "frac": round(achieved / peak, 4), "traffic": traffic,
-                    "kernel": dom, "ops_per_launch": dom_ops // n_dom_launches,
-                    "launch_us": round(dom_ms * 1e3 / n_dom_launches, 3),
-                    "peak_source": f"2 x {peaks['source']} bf16_tflops {peaks['bf16_tflops']} "
-                                   f"(MEASURED_PEAKS.json; int8 = 2 x bf16 nominal)",
-                    "dense_equivalent_frac": round(
-                        sum(2 * t * k * n_out for (n_out, k, n, m, ts) in layers for t in ts)
-                        / (dom_ms * 1e-3) / 1e12 / peak, 4)}
-    else:
-        if dom == "quantize_weights":
-            dom_bytes = sum(qw_bytes(n_out, k, n, m) for (n_out, k, n, m, ts) in layers)
-        elif dom == "quantize_acts":
-            dom_bytes = sum(qa_bytes(t, k) for (n_out, k, n, m, ts) in layers for t in ts)
-        elif dom == "bitlinear_x":
-            dom_bytes = sum(blx_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
-        elif dom == "bitlinear_entropy":
-            dom_bytes = sum(ble_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
-        elif dom == "bitlinear_entropy_x":
-            dom_bytes = sum(blex_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
-        elif dom == "pack_entropy":
-            dom_bytes = sum(pe_bytes(n_out, k, n, m) for (n_out, k, n, m, ts) in layers)
-        else:
-            dom_bytes = sum(bl_bytes(t, k, n_out, n, m) for (n_out, k, n, m, ts) in layers for t in ts)
-        achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                    "traffic": traffic, "kernel": dom,
-                    "bytes_per_launch": dom_bytes // n_dom_launches,
-                    "launch_us": round(dom_ms * 1e3 / n_dom_launches, 3),
-                    "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)"
-                    if peaks["source"] == "measured" else "fallback 6650 GB/s"}
-    breakdown = {}
-    for (name, li, t), v in per_call.items():
-        key = f"{name}[L{li}]" + (f"[T={t}]" if t else "")
-        n_out, k, n, m, _ = layers[li]
-        us = statistics.mean(v) * 1e3
-        if name == "quantize_weights":
-            b = qw_bytes(n_out, k, n, m)
-        elif name == "quantize_acts":
-            b = qa_bytes(t, k)
-        elif name == "bitlinear_x":
-            b = blx_bytes(t, k, n_out, n, m)
-        elif name == "bitlinear_entropy":
-            b = ble_bytes(t, k, n_out, n, m)
-        elif name == "bitlinear_entropy_x":
-            b = blex_bytes(t, k, n_out, n, m)
-        elif name == "pack_entropy":
-            b = pe_bytes(n_out, k, n, m)
-        else:
-            b = bl_bytes(t, k, n_out, n, m)
-        e = {"us": round(us, 3), "GB/s": round(b / (us * 1e-6) / 1e9, 1),
-             "hbm_frac": round(b / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
-        if name in ("bitlinear", "bitlinear_x", "bitlinear_entropy", "bitlinear_entropy_x"):
-            wb = (entropy_bytes(n_out, k, n, m) if name.startswith("bitlinear_entropy")
-                  else packed_bytes(n_out, k, n, m))
-            e["weight_GB/s"] = round(wb / (us * 1e-6) / 1e9, 1)
-            ops = bl_ops(t, k, n_out, n, m)
-            e["TOPS"] = round(ops / (us * 1e-6) / 1e12, 3)
-            e["dense_eq_TOPS"] = round(2 * t * k * n_out / (us * 1e-6) / 1e12, 3)
-            e["tokens_per_s"] = round(t / (us * 1e-6), 1)
-        breakdown[key] = e
-
-    # ---- end to end through the public API with pinned host buffers ----
-    e2e = run_e2e(args, data, layers, dev, stream, world)
-
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only) ----
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        frac, dt = run_oracle_timed(layers, data, target_s=args.cpu_seconds, mode=workload_mode(args.workload))
-        cpu = {"value": round(oracle_sample_metric(args.workload, layers, frac) / dt, 6),
-               "unit": WORKLOADS[args.workload]["unit"], "cores": cores_used(),
-               "kind": "oracle",
-               "sample": f"{frac:.3f} of the output features of every layer, full K and all "
-                         f"token sets; one pass, {dt:.1f} s"}
-
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": WORKLOADS[args.workload]["unit"],
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, bf16 io",
-            "data": "synthetic (seeded: W ~ N(0,0.02) bf16, X ~ N(0,1) bf16)",
-            "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]["desc"],
-                       "bytes_per_step": sb, "tokens_per_step": step_tokens(layers),
-                       "ops_per_step": step_ops(layers),
-                       "l2": f"inputs rotated over {R} copies (> 3x L2) between steps",
-                       "parallelism": f"replicas x{world} (independent layers per rank)"},
-            "tokens_per_s": round(step_tokens(layers) * args.steps * world / (ms * 1e-3), 1),
-            "roofline": roofline, "breakdown": breakdown,
-            "breakdown_note": "per-call means from one untimed replay per rotation slot with "
-                              "events around every call; the timed replays bracket only the "
-                              "dominant call (roofline.launch_us)",
-            "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk, "cpu_baseline": cpu,
-        }
-        print(json.dumps(line), flush=True)
+    steps = args.steps
+    passes = args.passes
+    clocks = ClockSampler(dev.index if dev.index is not None else 0) if headline else None
+    if clocks:
+        clocks.start()
+    pass_ms = []
+    for _ in range(passes):
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(steps):
+                graphs[i % R].replay()
+            e1.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+        pass_ms.append(max_over_ranks(e0.elapsed_time(e1), world, dev))
+    clk = clocks.stop() if clocks else None
+    ms = statistics.median(pass_ms)
     graphs.clear()
 
+    kinds = list(dict.fromkeys(c[0] for c in eng.calls))
+    per_kind = kind_breakdown(eng, kinds, peaks, reps=max(3, args.kernel_reps))
+    dom = max(per_kind, key=lambda k: per_kind[k]["us_per_step"])
+    roof = roofline_of(workload, eng, dom, per_kind, peaks, i8_peak_src)
+    launches = sum(call_launches(c[0], c[2]) for c in eng.calls)
+    unit = WORKLOADS[workload]["unit"]
+    e2e = run_e2e(workload, eng, data, dev, stream, world, steps=max(3, min(steps, args.e2e_steps)))
+    entry = {
+        "metric": METRIC, "value": round(rate(workload, layers, steps, world, ms), 3), "unit": unit,
+        "higher_is_better": unit != "us", "ms_per_step": round(ms / steps, 5),
+        "passes_ms_per_step": [round(p / steps, 5) for p in pass_ms],
+        "config": {"workload": workload, "desc": WORKLOADS[workload]["desc"],
+                   "bytes_per_step": step_bytes(layers, WORKLOADS[workload]["mode"], WORKLOADS[workload]["qw"]),
+                   "tokens_per_step": step_tokens(layers), "ops_per_step": step_ops(layers),
+                   "l2": f"inputs rotated over {R} copies (> 3x the {l2 // (1 << 20)} MiB L2) between steps",
+                   "parallelism": f"replicas x{world} (independent layers per rank)"},
+        "tokens_per_s": round(step_tokens(layers) * steps * world / (ms * 1e-3), 1),
+        "roofline": roof, "breakdown": per_kind,
+        "breakdown_note": "per kind: back-to-back launches of every call of that kind over all rotation "
+                          "slots in one graph, events around the whole replay",
+        "e2e": e2e, "gpu_launches": launches * steps, "clocks": clk,
+    }
+    del eng
+    torch.cuda.empty_cache()
+    return entry
 
-def run_e2e(args, data, layers, dev, stream, world):
+
+def run_e2e(workload, eng, data, dev, stream, world, steps):
+    """The step through the public binding from pinned host buffers: H2D of the
+    step's inputs, the calls, D2H of its outputs, every step."""
     import torch
     import torch.distributed as dist
-    from sparse_linear_layers_fwd_b200 import sbn
-
+    sbn = eng.sbn
+    w = WORKLOADS[workload]
+    layers = eng.layers
     host = []
-    for (w, xs, n, m) in data:
-        hw = torch.from_numpy(np.ascontiguousarray(w).view(np.int16)).view(torch.bfloat16).pin_memory()
+    for (wb, xs, n, m) in data:
+        hw = (torch.from_numpy(np.ascontiguousarray(wb).view(np.int16)).view(torch.bfloat16).pin_memory()
+              if w["qw"] else torch.empty((wb.shape[0], 0), dtype=torch.bfloat16))
         hxs = [torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
                for x in xs]
         host.append((hw, hxs, n, m))
-    dw = [torch.empty(h[0].shape, dtype=torch.bfloat16, device=dev) for h in host]
-    dxs = [[torch.empty(x.shape, dtype=torch.bfloat16, device=dev) for x in h[1]] for h in host]
-    ys_host = [[torch.empty((x.shape[0], h[0].shape[0]), dtype=torch.bfloat16).pin_memory()
-                for x in h[1]] for h in host]
-    h2d = sum(h[0].numel() * 2 + sum(x.numel() * 2 for x in h[1]) for h in host)
+    ys_host = [[torch.empty((x.shape[0], h[0].shape[0]), dtype=torch.bfloat16).pin_memory() for x in h[1]]
+               for h in host]
+    L0 = eng.slots[0]
+    h2d = sum((h[0].numel() * 2 if w["qw"] else 0) + sum(x.numel() * 2 for x in h[1]) for h in host)
     d2h = sum(y.numel() * 2 for ys in ys_host for y in ys)
-    ws = [torch.empty(sbn.workspace_bytes(*h[0].shape), dtype=torch.uint8, device=dev) for h in host]
-    pws = [sbn.alloc_packed(h[0].shape[0], h[0].shape[1], h[2], h[3], dev) for h in host]
-
-    fused = is_fused(args.workload)
-    mode = workload_mode(args.workload)
 
     def step():
         for li, (hw, hxs, n, m) in enumerate(host):
-            dw[li].copy_(hw, non_blocking=True)
-            sbn.quantize_weights(dw[li], n, m, out=pws[li], workspace=ws[li], stream=stream)
-            ent = sbn.pack_entropy(pws[li], stream=stream) if mode == "entropy" else None
+            L = L0[li]
+            if w["qw"]:
+                L["w"].copy_(hw, non_blocking=True)
+                sbn.quantize_weights(L["w"], n, m, out=L["pw"], workspace=L["ws"], stream=stream)
+            ent = sbn.pack_entropy(L["pw"], out=L["ent"], stream=stream) if w["mode"] == "entropy" else None
             for j, hx in enumerate(hxs):
-                dxs[li][j].copy_(hx, non_blocking=True)
-                if mode == "entropy":
-                    y = sbn.bitlinear_entropy_x(dxs[li][j], ent, pws[li], workspace=False, stream=stream)
-                elif fused:
-                    y = sbn.bitlinear_x(dxs[li][j], pws[li], stream=stream)
+                L["xs"][j].copy_(hx, non_blocking=True)
+                if w["mode"] == "entropy":
+                    y = sbn.bitlinear_entropy_x(L["xs"][j], ent, L["pw"], out=L["ys"][j], workspace=False,
+                                                stream=stream)
+                elif w["mode"] == "fused":
+                    y = sbn.bitlinear_x(L["xs"][j], L["pw"], out=L["ys"][j], workspace=L["bws"], stream=stream)
                 else:
-                    q, s = sbn.quantize_acts(dxs[li][j], stream=stream)
-                    y = sbn.bitlinear(q, s, pws[li], stream=stream)
+                    q, s = L["qs"][j]
+                    sbn.quantize_acts(L["xs"][j], out_q=q, out_s=s, stream=stream)
+                    y = sbn.bitlinear(q, s, L["pw"], out=L["ys"][j], workspace=L["bws"], stream=stream)
                 ys_host[li][j].copy_(y, non_blocking=True)
 
-    steps = max(3, min(args.steps, args.e2e_steps))
     with torch.cuda.stream(stream):
-        for _ in range(max(3, min(args.warmup, 10))):
+        for _ in range(2):
             step()
     stream.synchronize()
     if world > 1:
         dist.barrier()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        ev0.record(stream)
+        e0.record(stream)
         for _ in range(steps):
             step()
-        ev1.record(stream)
+        e1.record(stream)
     stream.synchronize()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-    ev = whole_job_value(args.workload, steps, world, ms)
-    return {"value": round(ev, 3), "unit": WORKLOADS[args.workload]["unit"],
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(rate(workload, layers, steps, world, ms), 3), "unit": WORKLOADS[workload]["unit"],
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4)}
 
 
 # ---------------------------------------------------------------------------
-# reference arm: the CPU oracle as it stands
+# the 3B-scale pattern sweep
 # ---------------------------------------------------------------------------
 
+def run_ffn3b(args, dev, stream, peaks, i8_peak_src, with_cpu):
+    """Per pattern: sbn_quantize_weights of gate and down (the per-step dynamic
+    mask, timed separately); per (pattern, projection, T): quantize_acts and
+    bitlinear, each timed back to back over rotated copies of its inputs."""
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn, synth
+    l2 = l2_bytes(dev)
+    projs = [("gate", 2048, 11008), ("down", 11008, 2048)]
+    entries, qw_entries = [], []
+    tot_ops, tot_us = 0, 0.0
+    for (pn, k, n_out) in projs:
+        wbits = synth.latent_weights(n_out, k, seed=0, tag=f"bench_ffn3b_{pn}")
+        wd = to_dev(wbits, dev)
+        xs_dev = {t: to_dev(synth.activations(t, k, seed=0, tag=f"bench_ffn3b_{pn}_t{t}"), dev)
+                  for t in synth.FFN3B_TOKENS}
+        ws = torch.empty(sbn.workspace_bytes(n_out, k), dtype=torch.uint8, device=dev)
+        for (n, m) in synth.FFN3B_PATTERNS:
+            # quantize_weights: rotated latent copies
+            Rw = int(min(24, max(2, math.ceil(3 * l2 / (2 * n_out * k)))))
+            wcopies = [wd] + [wd.clone() for _ in range(Rw - 1)]
+            pws = [sbn.alloc_packed(n_out, k, n, m, dev) for _ in range(Rw)]
+            with torch.cuda.stream(stream):
+                for i in range(Rw):
+                    sbn.quantize_weights(wcopies[i], n, m, out=pws[i], workspace=ws, stream=stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(Rw):
+                    sbn.quantize_weights(wcopies[i], n, m, out=pws[i], workspace=ws, stream=stream)
+            us = replay_ms(g, stream, max(3, args.kernel_reps)) * 1e3 / Rw
+            del g
+            qb = qw_bytes(n_out, k, n, m)
+            qw_entries.append({"proj": pn, "pattern": f"{n}:{m}", "us": round(us, 3),
+                               "GB/s": round(qb / (us * 1e-6) / 1e9, 1),
+                               "hbm_frac": round(qb / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)})
+            del wcopies
+            for t in synth.FFN3B_TOKENS:
+                x = xs_dev[t]
+                per = bl_bytes(t, k, n_out, n, m)
+                R = int(min(48, max(1, math.ceil(3 * l2 / per))))
+                pw_r = [pws[i % Rw] for i in range(R)]
+                xq = [torch.empty((t, k), dtype=torch.int8, device=dev) for _ in range(R)]
+                xsc = [torch.empty((t,), dtype=torch.float32, device=dev) for _ in range(R)]
+                ys = [torch.empty((t, n_out), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+                xcopies = [x] + [x.clone() for _ in range(R - 1)]
+                bws = torch.empty((max(1, sbn.bitlinear_workspace_bytes(t, k, n_out)),), dtype=torch.uint8,
+                                  device=dev)
+                with torch.cuda.stream(stream):
+                    for i in range(R):
+                        sbn.quantize_acts(xcopies[i], out_q=xq[i], out_s=xsc[i], stream=stream)
+                        sbn.bitlinear(xq[i], xsc[i], pw_r[i], out=ys[i], workspace=bws, stream=stream)
+                stream.synchronize()
+                ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+                with torch.cuda.graph(ga, stream=stream):
+                    for i in range(R):
+                        sbn.quantize_acts(xcopies[i], out_q=xq[i], out_s=xsc[i], stream=stream)
+                with torch.cuda.graph(gb, stream=stream):
+                    for i in range(R):
+                        sbn.bitlinear(xq[i], xsc[i], pw_r[i], out=ys[i], workspace=bws, stream=stream)
+                reps = max(3, args.kernel_reps if t < 8192 else 3)
+                qa_us = replay_ms(ga, stream, reps) * 1e3 / R
+                bl_us = replay_ms(gb, stream, reps) * 1e3 / R
+                del ga, gb
+                ops = bl_ops(t, k, n_out, n, m)
+                tot_ops += ops
+                tot_us += bl_us
+                e = {"proj": pn, "pattern": f"{n}:{m}", "T": t, "bitlinear_us": round(bl_us, 3),
+                     "TOPS": round(ops / (bl_us * 1e-6) / 1e12, 3),
+                     "weight_GB/s": round(packed_bytes(n_out, k, n, m) / (bl_us * 1e-6) / 1e9, 1),
+                     "quantize_acts_us": round(qa_us, 3)}
+                if t > 16:
+                    peak, _src = i8_peak_src
+                    e["bound"] = "tensor"
+                    e["frac"] = round(ops / (bl_us * 1e-6) / 1e12 / peak, 4)
+                else:
+                    e["bound"] = "hbm"
+                    e["frac"] = round(per / (bl_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)
+                entries.append(e)
+                del xq, xsc, ys, xcopies, bws, pw_r
+            del pws
+        del wd, xs_dev
+        torch.cuda.empty_cache()
+    tops = tot_ops / (tot_us * 1e-6) / 1e12
+    peak, src = i8_peak_src
+    big = [e for e in entries if e["T"] >= 512]
+    dom = max(big, key=lambda e: e["bitlinear_us"])
+    out = {"metric": METRIC, "value": round(tops, 3), "unit": "TOPS", "higher_is_better": True,
+           "config": {"workload": "ffn3b",
+                      "desc": "3B-scale FFN sweep: gate (K=2048, N_out=11008) and down (K=11008, N_out=2048), "
+                              "T in {1,64,512,8192} x n:m in {2:4,4:8,6:8,8:16,8:8}; value = algorithmic ops "
+                              "of every contraction / their summed times; quantize_weights timed separately",
+                      "l2": "each entry rotated over enough input copies to exceed 3x L2"},
+           "roofline": {"bound": "tensor", "achieved": dom["TOPS"], "peak": round(peak, 1), "unit": "TOPS",
+                        "frac": dom["frac"], "traffic": None, "kernel": "bitlinear",
+                        "entry": f"{dom['proj']} {dom['pattern']} T={dom['T']}", "peak_source": src},
+           "sweep": entries, "quantize_weights": qw_entries}
+    if with_cpu:
+        out["cpu_baseline"] = ffn3b_cpu_baseline()
+    out["e2e"] = None
+    out["e2e_note"] = "per-entry kernel timings only; end-to-end figures are given for the other workloads"
+    return out
+
+
+def ffn3b_cpu_baseline(target_s=8.0):
+    """The oracle on a row sample of the 6:8 gate projection at T = 64 (TOPS)."""
+    import oracle
+    from sparse_linear_layers_fwd_b200 import synth
+    w = synth.latent_weights(11008, 2048, seed=0, tag="bench_ffn3b_gate")
+    x = synth.activations(64, 2048, seed=0, tag="bench_ffn3b_gate_t64")
+    with oracle_threads_one():
+        rows = 16
+        t0 = time.perf_counter()
+        oracle_step([(w, [x], 6, 8)], rows)
+        dt = time.perf_counter() - t0
+        rows = int(min(11008, max(16, rows * target_s / max(dt, 1e-3))))
+        t0 = time.perf_counter()
+        oracle_step([(w, [x], 6, 8)], rows)
+        dt = time.perf_counter() - t0
+    ops = bl_ops(64, 2048, rows, 6, 8)
+    return {"value": round(ops / dt / 1e12, 9), "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": f"gate projection 6:8, T=64, {rows} of 11008 output features; quantize_weights + "
+                      f"quantize_acts + contraction; one pass, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# driver
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    sbn.lib()
+    stream = torch.cuda.Stream(device=dev)
+    peaks = load_peaks()
+    i8 = int8_peak(peaks)
+    head = run_workload(args.workload, args, rank, world, dev, stream, peaks, i8, headline=True)
+    extras = {}
+    if world == 1 and not args.only:
+        for wl in EXTRA_WORKLOADS:
+            if wl == args.workload:
+                continue
+            try:
+                if wl == "ffn3b":
+                    extras[wl] = run_ffn3b(args, dev, stream, peaks, i8, with_cpu=not args.no_cpu_baseline)
+                else:
+                    e = run_workload(wl, args, rank, world, dev, stream, peaks, i8, headline=False)
+                    if not args.no_cpu_baseline:
+                        e["cpu_baseline"] = cpu_baseline(wl, target_s=args.cpu_seconds / 2,
+                                                         first=7 if wl == "qwen05b" else None)
+                    extras[wl] = e
+            except torch.cuda.OutOfMemoryError as ex:  # noqa: PERF203
+                extras[wl] = {"error": f"out of device memory: {ex}"[:200]}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, target_s=args.cpu_seconds)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": head["higher_is_better"], "scaling": "weak", "vs_baseline": None,
+            "dtype": DTYPE, "data": DATA_DESC, "config": head["config"],
+            "passes_ms_per_step": head["passes_ms_per_step"], "tokens_per_s": head["tokens_per_s"],
+            "roofline": head["roofline"], "breakdown": head["breakdown"],
+            "breakdown_note": head["breakdown_note"], "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"], "clocks": head["clocks"], "cpu_baseline": cpu,
+        }
+        if extras:
+            line["workloads"] = extras
+        print(json.dumps(line), flush=True)
+
+
 def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm, on the same config, metric and
+    unit: every step is the same bounded sample of the workload."""
     if rank != 0:
         return
-    layers = WORKLOADS[args.workload]["layers"]
-    data = make_layers_data(args.workload, 0)
-    total_steps = args.steps + args.warmup
-    per_step = max(0.01, args.reference_seconds / max(1, total_steps))
-    mode = workload_mode(args.workload)
-    frac, _ = run_oracle_timed(layers, data, target_s=per_step, mode=mode)
-    rows = [max(1, int(l[0] * frac)) for l in layers]
-    for _ in range(args.warmup):
-        for d, r in zip(data, rows):
-            oracle_step([d], r, mode)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        for d, r in zip(data, rows):
-            oracle_step([d], r, mode)
-    dt = time.perf_counter() - t0
-    value = oracle_sample_metric(args.workload, layers, frac) * args.steps / dt
-    unit = WORKLOADS[args.workload]["unit"]
+    workload = args.workload
+    layers = workload_layers(workload)
+    mode = workload_mode(workload)
+    data = make_layers_data(workload, 0, first=7 if workload == "qwen05b" else None)
+    per_step = max(0.01, args.reference_seconds / max(1, args.steps + args.warmup))
+    with oracle_threads_one():
+        _dt, done, desc = oracle_sample(workload, layers, data, per_step)   # sizes the sample
+        frac = desc_frac(desc)
+        for _ in range(args.warmup):
+            oracle_sample_step(workload, layers, data, frac)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_sample_step(workload, layers, data, frac)
+        dt = time.perf_counter() - t0
+    unit = WORKLOADS[workload]["unit"]
+    if unit == "us":
+        value = dt / args.steps / done * 1e6
+    else:
+        value = step_units(workload, layers) * done * args.steps / dt
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, bf16 io",
-        "data": "synthetic (seeded: W ~ N(0,0.02) bf16, X ~ N(0,1) bf16)",
-        "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]["desc"],
-                   "bytes_per_step": step_bytes(layers, workload_mode(args.workload)),
-                   "tokens_per_step": step_tokens(layers)},
-        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores_used(),
-                         "kind": "oracle",
-                         "sample": f"each step: {frac:.3f} of the output features of every "
-                                   f"layer, full K, all token sets"},
-        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": unit != "us",
+        "scaling": "weak", "vs_baseline": None, "dtype": DTYPE, "data": DATA_DESC,
+        "config": {"workload": workload, "desc": WORKLOADS[workload]["desc"],
+                   "bytes_per_step": step_bytes(layers, mode, WORKLOADS[workload]["qw"]),
+                   "tokens_per_step": step_tokens(layers), "ops_per_step": step_ops(layers),
+                   "l2": "host CPU (no GPU L2)", "parallelism": f"replicas x{world} (independent layers per rank)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": 1, "kind": "oracle",
+                         "sample": "each step: " + desc},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def desc_frac(desc):
+    return float(desc.split(" ", 1)[0])
+
+
+def oracle_sample_step(workload, layers, data, frac):
+    mode = workload_mode(workload)
+    for (w, xs, n, m), l in zip(data, layers):
+        oracle_step([(w, xs, n, m)], max(1, int(l[0] * frac)), mode)
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--passes", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--only", action="store_true", help="the headline workload only")
+    ap.add_argument("--kernel-reps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

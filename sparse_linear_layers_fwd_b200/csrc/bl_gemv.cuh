@@ -92,6 +92,9 @@ struct GvParams {
   int cstride, mstride;
   int tiles_per_cta;      // tiles of the largest CTA range
   int tile_base, tile_rem;  // CTA b owns tile_base (+1 if b < tile_rem) tiles
+  int kc;                 // 16-byte activation chunks per row (K/8 bf16 or K/16 INT8)
+  uint32_t kc_magic;      // ceil(2^32 / kc): q / kc == umulhi(q, kc_magic) for q < 2^16
+  int dr, drem;           // 992 = dr * kc + drem (the step of a thread's chunk index)
   GvLayout L;             // shared-memory layout (the host's gv_layout)
 };
 
@@ -100,6 +103,19 @@ struct GvParams {
 // on the stream start its launch.
 SBN_DEVFN void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 SBN_DEVFN void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// Elementwise max(|a|, |b|) of two bf16 pairs (the sign of each result is
+// the xor of the operands' signs; callers clear it).
+SBN_DEVFN uint32_t gv_absmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Largest magnitude of a 16-byte chunk (8 bf16) folded into a running pair.
+SBN_DEVFN uint32_t gv_chunk_absmax(const uint4& v, uint32_t run) {
+  return gv_absmax2(gv_absmax2(gv_absmax2(v.x, v.y), gv_absmax2(v.z, v.w)), run);
+}
 
 // Named barriers: 1 among the consumer warps; 2 from the producer's set-up
 // (it arrives) to the consumers (they wait).
@@ -159,6 +175,19 @@ SBN_DEVFN uint2 gv_selector_pair(uint32_t mask8) {
   return make_uint2(sel & 0xFFFFu, sel >> 16);
 }
 
+// The bits of the word array from bit OFF on, masked with MASK (compile-time
+// positions; MASK's highest bit below 32 - OFF % 32 + 32).
+template <int OFF, uint32_t MASK, int NW>
+SBN_DEVFN uint32_t gv_field(const uint32_t (&w)[NW]) {
+  constexpr int i = OFF / 32, s = OFF % 32;
+  constexpr int width = 32 - __builtin_clz(MASK);
+  if constexpr (s + width <= 32) {
+    return (w[i] >> s) & MASK;
+  } else {
+    return __funnelshift_r(w[i], w[i + 1], s) & MASK;
+  }
+}
+
 // Eight positions (group I of the thread's span) of one row -> int8 bytes
 // 0-3 (w0) and 4-7 (w1). cw: the span's code words; mw: its 8 keep bytes;
 // s_sel2: the selector pairs of the 256 keep masks.
@@ -174,9 +203,17 @@ SBN_DEVFN void gv_expand(const uint32_t (&cw)[CB], const uint32_t (&mw)[2], cons
     w1 = gv_prmt(ev, od, 0x7362u);
     return;
   } else if constexpr (MM != 16) {
-    // m = 4 or 8: every 8 positions keep 2*CB codes
+    // m = 4 or 8: every 8 positions keep 2*CB codes; the even- and
+    // odd-indexed codes are cut straight out of the code words
+    constexpr int kOff = 4 * CB * I;
+    constexpr uint32_t kMask = CB == 1 ? 0x3u : CB == 2 ? 0x33u : 0x333u;
     m8 = gv_prmt(mw[I / 4], 0u, 0x4440u | (I % 4));
-    v = gv_bits<4 * CB * I, 4 * CB, CB>(cw);
+    const uint32_t ev = gv_prmt(kCodeByteTable, 0u, gv_field<kOff, kMask, CB>(cw));
+    const uint32_t od = gv_prmt(kCodeByteTable, 0u, gv_field<kOff + 2, kMask, CB>(cw));
+    const uint2 sel = s_sel2[m8];
+    w0 = gv_prmt(ev, od, sel.x);
+    w1 = gv_prmt(ev, od, sel.y);
+    return;
   } else {
     // m = 16: a 16-position group keeps 4*CB codes, split unevenly between
     // its halves; the second half's codes follow the first half's
@@ -248,25 +285,21 @@ bl_gemv_kernel(const GvParams p) {
   // ---- consumers: activations global -> registers ----
   griddep_wait();
   const float gm = ACC ? 0.f : __ldg(p.gamma);
-  // chunk q of the T x kc chunks: row q / kc; this thread takes q = tid + 992 j
-  const int kc = XBF ? p.K / 8 : p.K / 16;   // 16-byte chunks per row (8 bf16 or 16 INT8)
+  // chunk q of the T x kc chunks (row q / kc): this thread takes
+  // q = tid + 992 j; warps past the last chunk skip the phase
+  const int kc = p.kc;
   const int nq = p.T * kc;
-  const int dr = kGvConsumers / kc, drem = kGvConsumers - dr * kc;
+  const bool xwarp = warp * 32 < nq;
+  const int q0r = (int)__umulhi((uint32_t)tid, p.kc_magic);
+  const int q0c = tid - q0r * kc;
+  const uint4* xsrc = reinterpret_cast<const uint4*>(XBF ? static_cast<const void*>(p.xbf)
+                                                         : static_cast<const void*>(p.xq));
   uint4 v[kGvMaxChunks];
-  int vrow[kGvMaxChunks], vcol[kGvMaxChunks];
-  {
-    int r = tid / kc, c = tid - (tid / kc) * kc;
+  if (xwarp) {
 #pragma unroll
     for (int j = 0; j < kGvMaxChunks; ++j) {
-      vrow[j] = r;
-      vcol[j] = c;
       const int q = tid + j * kGvConsumers;
-      if (q < nq)
-        v[j] = __ldg(reinterpret_cast<const uint4*>(XBF ? static_cast<const void*>(p.xbf)
-                                                       : static_cast<const void*>(p.xq)) + q);
-      r += dr;
-      c += drem;
-      if (c >= kc) { c -= kc; ++r; }
+      if (q < nq) v[j] = __ldg(xsrc + q);
     }
   }
   float xs_t = 0.f;
@@ -278,21 +311,29 @@ bl_gemv_kernel(const GvParams p) {
   gv_setup_wait();   // the producer's barriers and row maxima are initialized
 
   if (XBF) {
-    // per-row maxima: chunk maxima, reduced per row within the warp, then a
-    // shared atomic max per (warp, row)
+    if (xwarp) {
+      // per-row maxima: chunk maxima, reduced per row within the warp, then
+      // one shared atomic max per (warp, row)
+      int r = q0r, c = q0c;
 #pragma unroll
-    for (int j = 0; j < kGvMaxChunks; ++j) {
-      const bool ok = tid + j * kGvConsumers < nq;
-      const uint32_t m = ok ? mag_max8(v[j]) : 0u;
-      const int row = ok ? vrow[j] : -1;
-      uint32_t todo = __ballot_sync(0xffffffffu, ok);
-      while (todo) {
-        const int lead = __ffs(todo) - 1;
-        const int lr = __shfl_sync(0xffffffffu, row, lead);
-        const bool mine = row == lr;
-        const uint32_t rm = __reduce_max_sync(0xffffffffu, mine ? m : 0u);
-        if (lane == lead) atomicMax(&s_rmax[lr], rm);
-        todo &= ~__ballot_sync(0xffffffffu, mine);
+      for (int j = 0; j < kGvMaxChunks; ++j) {
+        if (j * kGvConsumers + warp * 32 >= nq) break;   // the whole warp is done
+        const bool ok = tid + j * kGvConsumers < nq;
+        const uint32_t m2 = ok ? gv_chunk_absmax(v[j], 0u) : 0u;
+        const uint32_t m = ok ? max(m2 & 0x7FFFu, (m2 >> 16) & 0x7FFFu) : 0u;
+        const int row = ok ? r : -1;
+        uint32_t todo = __ballot_sync(0xffffffffu, ok);
+        while (todo) {
+          const int lead = __ffs(todo) - 1;
+          const int lr = __shfl_sync(0xffffffffu, row, lead);
+          const bool mine = row == lr;
+          const uint32_t rm = __reduce_max_sync(0xffffffffu, mine ? m : 0u);
+          if (lane == lead) atomicMax(&s_rmax[lr], rm);
+          todo &= ~__ballot_sync(0xffffffffu, mine);
+        }
+        r += p.dr;
+        c += p.drem;
+        if (c >= kc) { c -= kc; ++r; }
       }
     }
     gv_consumer_sync();
@@ -303,21 +344,37 @@ bl_gemv_kernel(const GvParams p) {
       if (bid == 0 && p.xs_out) p.xs_out[tid] = sc;
     }
     gv_consumer_sync();
-    const bool out = bid == 0 && p.xq_out != nullptr;
+    if (xwarp) {
+      const bool out = bid == 0 && p.xq_out != nullptr;
+      int r = q0r, c = q0c;
 #pragma unroll
-    for (int j = 0; j < kGvMaxChunks; ++j) {
-      if (tid + j * kGvConsumers < nq) {
-        const uint2 q = quant8_magic(v[j], s_scale[vrow[j]]);
-        const int c = vcol[j];   // 8-position chunk of the row
-        *reinterpret_cast<uint2*>(s_x + (size_t)vrow[j] * L.xstride + gv_xchunk(c >> 1) + 8 * (c & 1)) = q;
-        if (out) *reinterpret_cast<uint2*>(p.xq_out + (size_t)vrow[j] * p.K + 8 * (size_t)c) = q;
+      for (int j = 0; j < kGvMaxChunks; ++j) {
+        if (j * kGvConsumers + warp * 32 >= nq) break;
+        if (tid + j * kGvConsumers < nq) {
+          const float mult = s_scale[r];
+          // scalar multiply and add: each rounds on its own (a fused
+          // multiply-add would round once and break ties of fl32(x * mult))
+          const uint2 q = quant8_magic(v[j], mult);
+          *reinterpret_cast<uint2*>(s_x + (size_t)r * L.xstride + gv_xchunk(c >> 1) + 8 * (c & 1)) = q;
+          if (out) *reinterpret_cast<uint2*>(p.xq_out + (size_t)r * p.K + 8 * (size_t)c) = q;
+        }
+        r += p.dr;
+        c += p.drem;
+        if (c >= kc) { c -= kc; ++r; }
       }
     }
   } else {
+    if (xwarp) {
+      int r = q0r, c = q0c;
 #pragma unroll
-    for (int j = 0; j < kGvMaxChunks; ++j)
-      if (tid + j * kGvConsumers < nq)
-        *reinterpret_cast<uint4*>(s_x + (size_t)vrow[j] * L.xstride + gv_xchunk(vcol[j])) = v[j];
+      for (int j = 0; j < kGvMaxChunks; ++j) {
+        if (j * kGvConsumers + warp * 32 >= nq) break;
+        if (tid + j * kGvConsumers < nq) *reinterpret_cast<uint4*>(s_x + (size_t)r * L.xstride + gv_xchunk(c)) = v[j];
+        r += p.dr;
+        c += p.drem;
+        if (c >= kc) { c -= kc; ++r; }
+      }
+    }
     if (!ACC && tid < p.T) s_ysc[tid] = __fdiv_rn(__fmul_rn(gm, xs_t), 127.0f);
   }
   gv_consumer_sync();
@@ -422,14 +479,15 @@ bl_gemv_kernel(const GvParams p) {
   gv_consumer_sync();
 
   const int rows = min(16 * tiles, p.N - row0);
-  for (int i = tid; i < rows * p.T; i += kGvConsumers) {
-    const int tok = i / rows, r = i - tok * rows;
-    const int a = s_acc[(size_t)(r >> 4) * 16 * NT + (r & 15) * NT + tok];
-    const int grow = row0 + r;
-    if (ACC) {
-      p.acc_out[(size_t)tok * p.N + grow] = a;
-    } else {
-      p.y[(size_t)tok * p.N + grow] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a, s_ysc[tok])));
+  for (int tok = 0; tok < p.T; ++tok) {
+    const float ysc = ACC ? 0.f : s_ysc[tok];
+    for (int r = tid; r < rows; r += kGvConsumers) {
+      const int a = s_acc[(size_t)(r >> 4) * 16 * NT + (r & 15) * NT + tok];
+      if (ACC) {
+        p.acc_out[(size_t)tok * p.N + row0 + r] = a;
+      } else {
+        p.y[(size_t)tok * p.N + row0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a, ysc)));
+      }
     }
   }
 }

@@ -310,6 +310,10 @@ sbn_status run_gemv(const int8_t* xq, const float* xs, const uint16_t* xbf, int8
   q.tile_base = tiles / grid;
   q.tile_rem = tiles % grid;
   q.L = gv_layout(per_cta, t <= 8 ? 8 : 16, t, k, q.cstride, q.mstride, n == m);
+  q.kc = XBF ? k / 8 : k / 16;
+  q.kc_magic = (uint32_t)(((1ull << 32) + (unsigned long long)q.kc - 1) / (unsigned long long)q.kc);
+  q.dr = kGvConsumers / q.kc;
+  q.drem = kGvConsumers % q.kc;
   return t <= 8 ? dispatch_gemv<8, ACC, XBF>(q, n, m, grid, smem, cs)
                 : dispatch_gemv<16, ACC, XBF>(q, n, m, grid, smem, cs);
 }

@@ -123,6 +123,56 @@ def test_fused_zero_rows_and_streaming_fallback():
     _fused_check(synth.latent_weights(64, 512, seed=16), x2, 2, 4)
 
 
+def _tie_scales():
+    """bf16 scales s in [1, 256) for which fl32(s/2 * fl32(127/s)) is exactly
+    63.5 although the exact product is not: rounding the product first (as
+    the definition does) gives the even 64, a fused multiply-add of the
+    product and the rounding constant would give 63 for half of them."""
+    out = []
+    for bits in range(0x3F80, 0x4380):
+        sv = np.uint32(bits << 16).view(np.float32)
+        p = np.float32(np.float32(sv / np.float32(2)) * np.float32(np.float32(127) / sv))
+        if p == np.float32(63.5):
+            out.append(bits)
+    return out
+
+
+def _tie_rows(scales, k, seed):
+    # row r: its maximum s_r first, then +-s_r/2 (exact in bf16) everywhere
+    rng = np.random.default_rng(seed)
+    x = np.empty((len(scales), k), dtype=np.uint16)
+    for r, sb in enumerate(scales):
+        row = np.full(k, sb - 0x80, dtype=np.uint16)
+        row[rng.random(k) < 0.5] |= np.uint16(0x8000)
+        row[0] = sb
+        x[r] = row
+    return x
+
+
+def test_activation_rounding_ties_quantize_acts():
+    from sparse_linear_layers_fwd_b200 import sbn
+    import torch
+    scales = _tie_scales()
+    assert len(scales) > 500
+    for k in (256, 2560, 4096):
+        x = _tie_rows(scales, k, seed=k)
+        q, sc = oracle.quantize_acts(x)
+        assert np.count_nonzero(np.abs(q.astype(np.int32)) == 64) > 0
+        xq, xs = sbn.quantize_acts(to_dev_bf16(x))
+        torch.cuda.synchronize()
+        assert np.array_equal(xs.cpu().numpy(), sc) and np.array_equal(xq.cpu().numpy(), q)
+
+
+@pytest.mark.parametrize("t,k", [(16, 2560), (9, 640), (1, 1152), (16, 384)])
+def test_activation_rounding_ties_fused(t, k):
+    # the fused decode path, 16 (or t) tie scales per call, all of them in turn
+    scales = _tie_scales()
+    w = synth.latent_weights(40, k, seed=23, tag="ties")
+    for i in range(0, len(scales), 16 * 9):
+        x = _tie_rows(scales[i:i + t], k, seed=i)
+        _fused_check(w, x, 6, 8)
+
+
 @pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (8, 8)])
 def test_all_zero_weights(nm):
     w = np.zeros((40, 256), np.uint16)
