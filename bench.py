@@ -679,16 +679,37 @@ def roofline_of(workload, eng, kind, per_kind, peaks, i8_peak):
             if peaks["source"] == "measured" else "fallback 6650 GB/s"}
 
 
-def int8_peak(peaks):
-    """The INT8 dense tensor peak: the measured figure of the in-tree tcgen05
-    kind::i8 probe when it is recorded in MEASURED_PEAKS.json, else 2x the
-    measured bf16 figure (the nominal int8 : bf16 ratio), labelled as derived."""
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        if "i8_tops" in d:
-            return float(d["i8_tops"]), "measured i8_tops (in-tree tcgen05 kind::i8 probe, MEASURED_PEAKS.json)"
+def measure_i8_peak(stream, iters=32768, reps=5):
+    """The INT8 dense rate of the tensor pipe, measured in this run: one CTA
+    per SM issuing back-to-back tcgen05.mma kind::i8 (128 x 256 x 32, the
+    prefill contraction's instruction and tile) with no loads, timed with CUDA
+    events; the best of `reps` launches. Returns TOP/s."""
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    with torch.cuda.stream(stream):
+        sbn.probe_i8_mma(iters, stream=stream)   # warm-up
+    stream.synchronize()
+    best = float("inf")
+    ctas = 0
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            ctas = sbn.probe_i8_mma(iters, stream=stream)
+            e1.record(stream)
+        stream.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    assert sbn.get_device_error() == 0
+    return ctas * iters * 2 * 128 * 256 * 32 / (best * 1e-3) / 1e12
+
+
+def int8_peak(peaks, measured=None):
+    """The INT8 dense tensor peak: the in-tree tcgen05 kind::i8 probe measured
+    in this run when given, else 2x the measured bf16 figure (the nominal
+    int8 : bf16 ratio), labelled as derived."""
+    if measured:
+        return measured, "measured in this run: in-tree tcgen05 kind::i8 probe (sbn_probe_i8_mma)"
     return 2.0 * peaks["bf16_tflops"], (f"derived: 2 x {peaks['source']} bf16_tflops {peaks['bf16_tflops']} "
                                         f"(nominal int8 : bf16 ratio)")
 
@@ -968,7 +989,12 @@ def run_ours(args, rank, world, local_rank):
     sbn.lib()
     stream = torch.cuda.Stream(device=dev)
     peaks = load_peaks()
-    i8 = int8_peak(peaks)
+    i8_measured = None
+    try:
+        i8_measured = measure_i8_peak(stream)
+    except Exception as ex:  # noqa: BLE001
+        print(f"i8 probe unavailable: {ex}", file=sys.stderr)
+    i8 = int8_peak(peaks, i8_measured)
     head = run_workload(args.workload, args, rank, world, dev, stream, peaks, i8, headline=True)
     extras = {}
     if world == 1 and not args.only:
@@ -999,6 +1025,8 @@ def run_ours(args, rank, world, local_rank):
             "roofline": head["roofline"], "breakdown": head["breakdown"],
             "breakdown_note": head["breakdown_note"], "e2e": head["e2e"],
             "gpu_launches": head["gpu_launches"], "clocks": head["clocks"], "cpu_baseline": cpu,
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                      "i8_tops": round(i8[0], 1), "i8_source": i8[1]},
         }
         if extras:
             line["workloads"] = extras

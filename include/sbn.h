@@ -410,6 +410,31 @@ sbn_status sbn_bitlinear_grad_w(const void* dy_bf16, const int8_t* xq,
                                 int32_t n_out, void* dw_bf16, void* stream);
 
 /*
+ * Measurement helper (no counterpart in the method): the INT8 rate of the
+ * tensor pipe. Launches one CTA per SM on `stream`, each issuing `iters`
+ * back-to-back tcgen05.mma kind::i8 instructions of M = 128, N = 256,
+ * K = 32 (2 * 128 * 256 * 32 operations each, int32 accumulation in tensor
+ * memory) on shared-memory operands -- the instruction and tile shape of the
+ * prefill contraction, with no loads in between. *ctas (host) receives the
+ * number of CTAs; the caller times the launch. Errors: SBN_ERR_NULL,
+ * SBN_ERR_SHAPE (iters outside 1..2^24), SBN_ERR_DEVICE, SBN_ERR_CUDA.
+ */
+sbn_status sbn_probe_i8_mma(int32_t iters, int32_t* ctas, void* stream);
+
+/*
+ * Test hook of the failure detection (no counterpart in the method): runs one
+ * of the library's bounded device waits on a condition that never comes, with
+ * a limit of limit_ns (1e3..1e8) nanoseconds, on `stream`. which = 0: an
+ * mbarrier wait (the kind every pipelined kernel uses); which = 1: the grid
+ * barrier of the weight quantizer. The wait gives up, records the timeout in
+ * the device error word and the kernel returns normally, so the next
+ * sbn_get_device_error returns SBN_ERR_TIMEOUT (and clears the word). No
+ * asynchronous copy or MMA is outstanding when the wait gives up. Errors:
+ * SBN_ERR_SHAPE (which or limit out of range), SBN_ERR_DEVICE, SBN_ERR_CUDA.
+ */
+sbn_status sbn_selftest_wait_timeout(int32_t which, int64_t limit_ns, void* stream);
+
+/*
  * sbn_get_device_error -- synchronizes `stream`, then reads and clears the
  * device error word of the current device. Returns SBN_OK, SBN_ERR_TIMEOUT
  * (a bounded device wait gave up; the affected outputs are unspecified) or

@@ -28,7 +28,7 @@ SBN_DEVFN void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
 // per warp) wait and the others meet it at a barrier: the phase completion
 // it observes, followed by the barrier, orders the arrived data before the
 // others' reads.
-SBN_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity) {
+SBN_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns = kMbarWaitNs) {
   const uint32_t a = smem_u32(bar);
   unsigned long long t0 = 0;
   for (uint32_t i = 0;; ++i) {
@@ -41,7 +41,7 @@ SBN_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (done) return true;
     const unsigned long long t = global_ns();
     if (i == 0u) t0 = t;
-    else if (t - t0 > kMbarWaitNs) break;
+    else if (t - t0 > limit_ns) break;
   }
   atomicOr(&g_dev_error, kDevErrTimeout);
   return false;

@@ -172,60 +172,167 @@ SBN_DEVFN uint32_t bmax2(uint32_t a, uint32_t b) { return as_u32(__hmax2(as_bf2(
 SBN_DEVFN uint32_t ble2(uint32_t a, uint32_t b) { return __hle2_mask(as_bf2(a), as_bf2(b)); }
 SBN_DEVFN uint32_t swap16(uint32_t a) { return __byte_perm(a, 0u, 0x1032u); }
 
+SBN_DEVFN uint32_t blt2(uint32_t a, uint32_t b) { return __hlt2_mask(as_bf2(a), as_bf2(b)); }
+
+// Bit j = element j of a group held as pairs (w0 = elements 0,1; ...), from
+// per-pair compare masks (0xFFFF per true half).
+SBN_DEVFN uint32_t pack_pair_masks(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
+  const uint32_t P = (m0 & 0x00010001u) | ((m1 & 0x00010001u) << 2) | ((m2 & 0x00010001u) << 4) |
+                     ((m3 & 0x00010001u) << 6);
+  return (P | (P >> 15)) & 0xFFu;
+}
+
+// The `need` (1 or 2) highest set bits of e.
+SBN_DEVFN uint32_t top_bits(uint32_t e, int need) {
+  const uint32_t h1 = 0x80000000u >> __clz(e);
+  return need == 1 ? h1 : h1 | (0x80000000u >> __clz(e ^ h1));
+}
+
 // Pruned positions (bit j = element j) of one group of 8 magnitudes held as
-// four pairs (w0 = elements 0,1; ...): the two smallest. The second
-// smallest a2 comes from a min/max network on the pairs; the elements with
-// magnitude <= a2 are exactly the two smallest unless the third smallest
-// equals a2 -- then false is returned and the caller ranks the group exactly.
-SBN_DEVFN bool prune_2of8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t& prune) {
+// four pairs (w0 = elements 0,1; ...): the two smallest, equal magnitudes
+// pruning the higher index first. The second smallest a2 comes from a
+// min/max network on the pairs; the elements with magnitude <= a2 are the
+// answer unless more than two share that bound -- then the ones below a2 are
+// pruned, and of those equal to a2 the highest-indexed fill up to two.
+SBN_DEVFN uint32_t prune_2of8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
   const uint32_t m01 = bmin2(w0, w1), M01 = bmax2(w0, w1);
   const uint32_t m23 = bmin2(w2, w3), M23 = bmax2(w2, w3);
   const uint32_t s1 = bmin2(m01, m23);                               // smallest per half
   const uint32_t s2 = bmin2(bmax2(m01, m23), bmin2(M01, M23));       // second per half
   const uint32_t a2 = bmin2(bmax2(s1, swap16(s1)), bmin2(s2, swap16(s2)));
-  const uint32_t P = (ble2(w0, a2) & 0x00010001u) | ((ble2(w1, a2) & 0x00010001u) << 2) |
-                     ((ble2(w2, a2) & 0x00010001u) << 4) | ((ble2(w3, a2) & 0x00010001u) << 6);
-  prune = (P | (P >> 15)) & 0xFFu;
-  return __popc(prune) == 2;
+  uint32_t le = pack_pair_masks(ble2(w0, a2), ble2(w1, a2), ble2(w2, a2), ble2(w3, a2));
+  if (__popc(le) != 2) {
+    const uint32_t lt = pack_pair_masks(blt2(w0, a2), blt2(w1, a2), blt2(w2, a2), blt2(w3, a2));
+    le = lt | top_bits(le & ~lt, 2 - __popc(lt));
+  }
+  return le;
 }
 
 // The same for one group of 4 magnitudes held as two pairs.
-SBN_DEVFN bool prune_2of4(uint32_t w0, uint32_t w1, uint32_t& prune) {
+SBN_DEVFN uint32_t prune_2of4(uint32_t w0, uint32_t w1) {
   const uint32_t m = bmin2(w0, w1), M = bmax2(w0, w1);
   const uint32_t a2 = bmin2(bmax2(m, swap16(m)), bmin2(M, swap16(M)));
-  const uint32_t P = (ble2(w0, a2) & 0x00010001u) | ((ble2(w1, a2) & 0x00010001u) << 2);
-  prune = (P | (P >> 15)) & 0xFu;
-  return __popc(prune) == 2;
+  uint32_t le = pack_pair_masks(ble2(w0, a2), ble2(w1, a2), 0u, 0u) & 0xFu;
+  if (__popc(le) != 2) {
+    const uint32_t lt = pack_pair_masks(blt2(w0, a2), blt2(w1, a2), 0u, 0u) & 0xFu;
+    le = lt | top_bits(le & ~lt, 2 - __popc(lt));
+  }
+  return le;
 }
 
-// Keep bits of one unit (16 magnitudes as 8 pairs) for 6:8 and 2:4 through
-// the networks above; other patterns, and groups where the boundary ties,
-// go through the exact rank selection.
+// Compare-exchange of two pairs, both lanes at once: a <- min, b <- max.
+SBN_DEVFN void ce2(uint32_t& a, uint32_t& b) {
+  const uint32_t lo = bmin2(a, b);
+  b = bmax2(a, b);
+  a = lo;
+}
+
+// Sorts the low halves of v[0..H) ascending and, independently, the high
+// halves (sorting networks of 1, 5 and 19 compare-exchanges).
+template <int H>
+SBN_DEVFN void sort_lanes(uint32_t (&v)[H]) {
+  if constexpr (H == 2) {
+    ce2(v[0], v[1]);
+  } else if constexpr (H == 4) {
+    ce2(v[0], v[1]); ce2(v[2], v[3]); ce2(v[0], v[2]); ce2(v[1], v[3]); ce2(v[1], v[2]);
+  } else if constexpr (H == 8) {
+    ce2(v[0], v[1]); ce2(v[2], v[3]); ce2(v[4], v[5]); ce2(v[6], v[7]);
+    ce2(v[0], v[2]); ce2(v[1], v[3]); ce2(v[4], v[6]); ce2(v[5], v[7]);
+    ce2(v[1], v[2]); ce2(v[5], v[6]);
+    ce2(v[0], v[4]); ce2(v[1], v[5]); ce2(v[2], v[6]); ce2(v[3], v[7]);
+    ce2(v[2], v[4]); ce2(v[3], v[5]);
+    ce2(v[1], v[2]); ce2(v[3], v[4]); ce2(v[5], v[6]);
+  }
+}
+
+// Bit j = element j of a group of 2H elements held as H pairs, from per-pair
+// compare masks (0xFFFF per true half).
+template <int H>
+SBN_DEVFN uint32_t pack_masks(const uint32_t (&m)[H]) {
+  uint32_t P = 0u;
+#pragma unroll
+  for (int j = 0; j < H; ++j) P |= (m[j] & 0x00010001u) << (2 * j);
+  return (P | (P >> 15)) & ((1u << (2 * H)) - 1u);
+}
+
+// Pruned positions (bit j = element j) of one group of M magnitudes held as
+// M/2 pairs w[0..M/2): the P smallest, equal magnitudes pruning the higher
+// index first. The even- and odd-indexed elements (low and high halves) are
+// sorted separately; the P-th smallest of the group is then the least of
+// max(A[i-1], B[P-1-i]) over the splits i of P between the two sorted lanes
+// A and B. Elements below it are pruned, and of those equal to it the
+// highest-indexed fill up to P.
+template <int M, int P>
+SBN_DEVFN uint32_t prune_group(const uint32_t* w) {
+  constexpr int H = M / 2;
+  constexpr int ilo = P > H ? P - H : 0, ihi = P < H ? P : H;
+  uint32_t v[H];
+#pragma unroll
+  for (int j = 0; j < H; ++j) v[j] = w[j];
+  sort_lanes<H>(v);
+  uint32_t T = 0u;
+#pragma unroll
+  for (int i = ilo; i <= ihi; ++i) {
+    uint32_t z;
+    if (i == 0) {
+      z = __byte_perm(v[P - 1], 0u, 0x3232u);            // B[P-1] in both halves
+    } else if (i == P) {
+      z = __byte_perm(v[P - 1], 0u, 0x1010u);            // A[P-1] in both halves
+    } else {
+      z = __byte_perm(v[i - 1], v[P - 1 - i], 0x7610u);  // (A[i-1], B[P-1-i])
+      z = bmax2(z, swap16(z));
+    }
+    T = (i == ilo) ? z : bmin2(T, z);
+  }
+  uint32_t m[H];
+#pragma unroll
+  for (int j = 0; j < H; ++j) m[j] = ble2(w[j], T);
+  uint32_t le = pack_masks<H>(m);
+  if (__popc(le) != P) {
+#pragma unroll
+    for (int j = 0; j < H; ++j) m[j] = blt2(w[j], T);
+    const uint32_t lt = pack_masks<H>(m);
+    uint32_t e = le & ~lt;
+    le = lt;
+    for (int need = P - __popc(lt); need > 0; --need) {
+      const uint32_t h = 0x80000000u >> __clz(e);
+      le |= h;
+      e ^= h;
+    }
+  }
+  return le;
+}
+
+// Keep bits of one unit (16 magnitudes as 8 pairs): 6:8 and 2:4 through the
+// specialized networks above, every other pattern through prune_group.
 template <int M>
 SBN_DEVFN uint32_t unit_keep_fast(const uint32_t (&mw)[8], int n) {
   if (M == 8 && n == 6) {
-    uint32_t p0, p1;
-    const bool a = prune_2of8(mw[0], mw[1], mw[2], mw[3], p0);
-    const bool b = prune_2of8(mw[4], mw[5], mw[6], mw[7], p1);
-    if (a && b) return (~(p0 | (p1 << 8))) & 0xFFFFu;
+    const uint32_t p0 = prune_2of8(mw[0], mw[1], mw[2], mw[3]);
+    const uint32_t p1 = prune_2of8(mw[4], mw[5], mw[6], mw[7]);
+    return (~(p0 | (p1 << 8))) & 0xFFFFu;
   } else if (M == 4 && n == 2) {
     uint32_t keep = 0u;
-    bool ok = true;
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      uint32_t pr;
-      ok &= prune_2of4(mw[2 * g], mw[2 * g + 1], pr);
-      keep |= ((~pr) & 0xFu) << (4 * g);
+    for (int g = 0; g < 4; ++g) keep |= ((~prune_2of4(mw[2 * g], mw[2 * g + 1])) & 0xFu) << (4 * g);
+    return keep;
+  }
+  uint32_t prune = 0u;
+#pragma unroll
+  for (int g = 0; g < 16 / M; ++g) {
+    const uint32_t* wg = mw + g * (M / 2);
+    uint32_t pg = 0u;
+    if (M == 4) {
+      pg = n == 1 ? prune_group<4, 3>(wg) : n == 3 ? prune_group<4, 1>(wg) : 0u;
+    } else if (M == 8) {
+      pg = n == 2 ? prune_group<8, 6>(wg) : n == 4 ? prune_group<8, 4>(wg) : 0u;
+    } else {
+      pg = n == 4 ? prune_group<16, 12>(wg) : n == 8 ? prune_group<16, 8>(wg)
+                  : n == 12 ? prune_group<16, 4>(wg) : 0u;
     }
-    if (ok) return keep;
+    prune |= pg << (g * M);
   }
-  uint32_t h[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    h[2 * i] = mw[i] & 0xFFFFu;
-    h[2 * i + 1] = mw[i] >> 16;
-  }
-  return unit_keep_bits<M>(h, n);
+  return (~prune) & 0xFFFFu;
 }
 
 // Four bytes with values in {0, 1, 3} -> their low two bits packed into 8

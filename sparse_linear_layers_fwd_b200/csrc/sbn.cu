@@ -16,6 +16,7 @@
 #include "qa.cuh"
 #include "qw.cuh"
 #include "qw_fused.cuh"
+#include "qw_stream.cuh"
 #include "qw_shard.cuh"
 #include "bl_decode.cuh"
 #include "bl_decode_res.cuh"
@@ -27,6 +28,7 @@
 #include "bwd.cuh"
 #include "flip.cuh"
 #include "bl_tc.cuh"
+#include "probe.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -81,38 +83,24 @@ sbn_status validate_weights_shape(int32_t n_out, int32_t k, int32_t n, int32_t m
 }
 
 
-// One cooperative launch of qw_fused_kernel: one CTA per SM, so that all
+// One cooperative launch of qw_stream_kernel: one CTA per SM, so that all
 // CTAs are resident for the grid barrier. The bins and the arrival counter
 // of the workspace are cleared first, on the same stream.
 template <int M>
-sbn_status launch_qw_fused(const uint16_t* w, int n_out, int k, int n, uint8_t* codes, int cstride,
-                           uint8_t* meta, int mstride, float* gamma, unsigned char* ws, int sms,
-                           cudaStream_t st) {
-  static bool attr_set[kMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    return SBN_ERR_CUDA;
-  }
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(qw_fused_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kQwSmemBytes) != cudaSuccess) {
-      cudaGetLastError();
-      return SBN_ERR_CUDA;
-    }
-    attr_set[dev] = true;
-  }
+sbn_status launch_qw_stream(const uint16_t* w, int n_out, int k, int n, uint8_t* codes, int cstride,
+                            uint8_t* meta, int mstride, float* gamma, unsigned char* ws, int sms,
+                            cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)std::min(sms, kQwMaxGrid));
-  cfg.blockDim = dim3(kQwThreads + 32);   // consumers + the producer warp
-  cfg.dynamicSmemBytes = kQwSmemBytes;
+  cfg.blockDim = dim3(kQsThreads);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, qw_fused_kernel<M>, w, n_out, k, n, codes, cstride, meta, mstride,
+  if (cudaLaunchKernelEx(&cfg, qw_stream_kernel<M>, w, n_out, k, n, codes, cstride, meta, mstride,
                          gamma, ws) != cudaSuccess) {
     cudaGetLastError();
     return SBN_ERR_CUDA;
@@ -133,9 +121,9 @@ sbn_status launch_quantize_weights(const uint16_t* w, int n_out, int k, int n, i
   const int cstride = (int)sbn_codes_row_bytes(k, n, m);
   const int mstride = (int)sbn_meta_row_bytes(k, n, m);
   switch (m) {
-    case 4: return launch_qw_fused<4>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
-    case 8: return launch_qw_fused<8>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
-    default: return launch_qw_fused<16>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
+    case 4: return launch_qw_stream<4>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
+    case 8: return launch_qw_stream<8>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
+    default: return launch_qw_stream<16>(w, n_out, k, n, codes, cstride, meta, mstride, gamma, ws, sms, st);
   }
 }
 
@@ -1119,6 +1107,36 @@ sbn_status sbn_quantize_weights_from_bins(const void* w_bf16, int32_t n_out, int
     case 8: return launch_qw_from_bins<8>(w, n_out, k, n, bins, total_elems, codes, meta, gamma, sms, s);
     default: return launch_qw_from_bins<16>(w, n_out, k, n, bins, total_elems, codes, meta, gamma, sms, s);
   }
+}
+
+sbn_status sbn_probe_i8_mma(int32_t iters, int32_t* ctas, void* stream) {
+  if (!ctas) return SBN_ERR_NULL;
+  if (iters < 1 || iters > (1 << 24)) return SBN_ERR_SHAPE;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(i8_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPkSmemBytes) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  i8_peak_kernel<<<sms, kPkThreads, kPkSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(iters);
+  *ctas = sms;
+  return launch_status();
+}
+
+sbn_status sbn_selftest_wait_timeout(int32_t which, int64_t limit_ns, void* stream) {
+  if (which != 0 && which != 1) return SBN_ERR_SHAPE;
+  if (limit_ns < 1000 || limit_ns > 100000000) return SBN_ERR_SHAPE;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(which, (unsigned long long)limit_ns);
+  return launch_status();
 }
 
 sbn_status sbn_get_device_error(void* stream) {

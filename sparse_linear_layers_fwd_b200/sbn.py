@@ -68,6 +68,8 @@ PROTOTYPES = {
     "sbn_bitlinear_grad_x": (ctypes.c_int, [_c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p,
                                             _c_p, _c_p]),
     "sbn_bitlinear_grad_w": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p]),
+    "sbn_probe_i8_mma": (ctypes.c_int, [_c_i32, ctypes.POINTER(ctypes.c_int32), _c_p]),
+    "sbn_selftest_wait_timeout": (ctypes.c_int, [_c_i32, ctypes.c_int64, _c_p]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
 
@@ -464,3 +466,17 @@ class BitLinear(torch.nn.Module):
         packed = self.pack()
         y = bitlinear_x(x2, packed)   # activation quantization fused for T <= 16
         return y.reshape(*lead, packed.n_out)
+
+
+def probe_i8_mma(iters: int, stream=None) -> int:
+    """sbn_probe_i8_mma: launches the tensor-pipe INT8 probe; returns the
+    number of CTAs (each issued `iters` MMAs of 2*128*256*32 operations)."""
+    ctas = ctypes.c_int32(0)
+    _check(lib().sbn_probe_i8_mma(int(iters), ctypes.byref(ctas), _stream_ptr(stream)), "sbn_probe_i8_mma")
+    return int(ctas.value)
+
+
+def selftest_wait_timeout(which: int, limit_ns: int, stream=None) -> None:
+    """sbn_selftest_wait_timeout: one bounded device wait that runs out (test hook)."""
+    _check(lib().sbn_selftest_wait_timeout(int(which), int(limit_ns), _stream_ptr(stream)),
+           "sbn_selftest_wait_timeout")
