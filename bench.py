@@ -314,10 +314,10 @@ def load_peaks():
 # device sources each call's kernels are built from: a recorded DRAM figure
 # stays valid while these files are unchanged
 TRAFFIC_FILES = {
-    "quantize_weights": ["qw_fused.cuh", "qw.cuh", "async.cuh", "common.cuh"],
+    "quantize_weights": ["qw_stream.cuh", "qw_fused.cuh", "qw.cuh", "async.cuh", "common.cuh"],
     "quantize_acts": ["qa.cuh", "common.cuh"],
     "bitlinear_x": ["bl_gemv.cuh", "bl_decode.cuh", "expand.cuh", "qa.cuh", "async.cuh", "common.cuh"],
-    "bitlinear": ["bl_tc.cuh", "expand_dense.cuh", "expand.cuh", "async.cuh", "common.cuh"],
+    "bitlinear": ["bl_tc_sp.cuh", "bl_tc.cuh", "expand_dense.cuh", "expand.cuh", "async.cuh", "common.cuh"],
     "bitlinear_entropy_x": ["bl_decode_ent.cuh", "bl_decode_res.cuh", "bl_decode.cuh", "entropy.cuh",
                             "expand.cuh", "qa.cuh", "common.cuh"],
     "pack_entropy": ["entropy_pack.cuh", "entropy.cuh", "common.cuh"],

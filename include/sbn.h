@@ -30,6 +30,14 @@
  *     Device-side failures (a bounded wait that ran out) are recorded in a
  *     device error word and reported by sbn_get_device_error.
  *   - Non-finite inputs (inf, NaN) give unspecified outputs.
+ *   - Per-device state: on its first call on a device the library caches,
+ *     for that device, the result of its capability check, the kernels'
+ *     shared-memory size attributes and the device address of the
+ *     sbn_quantize_weights_noalloc scratch array. These belong to the
+ *     device's primary context as it was then: after cudaDeviceReset (or any
+ *     other end of that context) they are stale, and the library must not be
+ *     called again on that device in the same process. Several host threads
+ *     may make first calls at the same time; they store the same values.
  *
  * Packed weight format (canonical; produced by sbn_quantize_weights and read
  * by sbn_bitlinear):
@@ -222,10 +230,18 @@ sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k,
  *                 inside the contraction kernel. Non-NULL (16-byte aligned,
  *                 ws_bytes >= sbn_bitlinear_workspace_bytes(t, k, n_out)):
  *                 for t > 16 the packed weights are first expanded once into
- *                 it as a dense int8 [n_out, k] matrix, which the tensor-core
- *                 kernel then loads by TMA like the activations. Ignored for
- *                 t <= 16. Its contents are unspecified afterwards. Both
- *                 routes give the same acc and y.
+ *                 it, and the tensor-core kernel then loads them by TMA like
+ *                 the activations: for 2:4 as the compressed operand of the
+ *                 sparse MMA (the kept int8 values [n_out, k/2] and their
+ *                 4-bit position metadata [n_out rounded up to 128, k/8]),
+ *                 for every other pattern as a dense int8 [n_out, k] matrix.
+ *                 Ignored for t <= 16. Its contents are unspecified
+ *                 afterwards. Both routes give the same acc and y.
+ * Tensor-core routes (t > 16): 2:4 runs the sparse INT8 MMA
+ * (tcgen05.mma.sp), which multiplies only the kept half of each group of
+ * four ("Sparse-BitNet ...", Abstract: the 2:4 pattern suits the sparse
+ * tensor cores); every other pattern runs the dense INT8 MMA on expanded
+ * weights.
  * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN,
  * SBN_ERR_WORKSPACE (before anything is enqueued); SBN_ERR_CUDA.
  */
@@ -235,7 +251,9 @@ sbn_status sbn_bitlinear(const int8_t* xq, const float* x_scale, int32_t t,
                          const float* gamma, void* y_bf16, void* workspace,
                          size_t ws_bytes, void* stream);
 
-/* Bytes of sbn_bitlinear's optional workspace: n_out * k when t > 16, else 0. */
+/* Bytes of sbn_bitlinear's optional workspace: when t > 16, the larger of
+ * n_out * k (dense expansion) and the compressed 2:4 form
+ * (round_up(n_out * k / 2, 128) + round_up(n_out, 128) * k / 8); else 0. */
 size_t sbn_bitlinear_workspace_bytes(int32_t t, int32_t k, int32_t n_out);
 
 /*

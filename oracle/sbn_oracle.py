@@ -31,7 +31,7 @@ What it computes (the BitLinear forward with a dynamic N:M mask):
    Estimator": gradients cross the quantizer as the identity, the latent
    weights take the update).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * gamma is taken over the whole dense latent tensor, before masking;
 * the exact sum of |w| is rounded once to fp64, divided by N_out*K in fp64,
   rounded to fp32 and floored at 1e-5 (the pages give no precision or epsilon);

@@ -1,6 +1,7 @@
 // Decode contraction (T <= 16 tokens), resident variant: every CTA copies
 // the packed weights of its output rows and the INT8 activations into shared
-// memory with a handful of bulk copies, then contracts them there.
+// memory with per-thread 16-byte asynchronous copies (cp.async), then
+// contracts them there.
 //
 // "Microsoft BitNet 1.58: The Era of 1-Bit Large Language Models", section
 // "bitnet.cpp: Matrix-Free Inference": 2-bit weights are moved on chip,

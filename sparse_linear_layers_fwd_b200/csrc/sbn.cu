@@ -23,6 +23,7 @@
 #include "bl_gemv.cuh"
 #include "bl_decode_ent.cuh"
 #include "expand_dense.cuh"
+#include "bl_tc_sp.cuh"
 #include "entropy.cuh"
 #include "entropy_pack.cuh"
 #include "bwd.cuh"
@@ -430,14 +431,14 @@ sbn_status dispatch_expand(const uint8_t* codes, const uint8_t* meta, int n_out,
   return SBN_ERR_PATTERN;
 }
 
-// TMA map of the INT8 activations [T, K]: boxes of 256 tokens x 128 bytes,
-// 128-byte swizzle (the layout the MMA descriptors describe).
-sbn_status make_act_tensor_map(CUtensorMap* tm, const int8_t* xq, int t, int k) {
+// TMA map of the INT8 activations [T, K]: boxes of box_rows tokens x 128
+// bytes, 128-byte swizzle (the layout the MMA descriptors describe).
+sbn_status make_act_tensor_map(CUtensorMap* tm, const int8_t* xq, int t, int k, int box_rows = kTcBN) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return SBN_ERR_CUDA;
   cuuint64_t gdim[2] = {(cuuint64_t)k, (cuuint64_t)t};
   cuuint64_t gstride[1] = {(cuuint64_t)k};
-  cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBN};
+  cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)box_rows};
   cuuint32_t estride[2] = {1, 1};
   const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(xq), gdim, gstride, box,
                          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -460,10 +461,88 @@ sbn_status make_weight_tensor_map(CUtensorMap* tm, const int8_t* wd, int n_out, 
   return r == CUDA_SUCCESS ? SBN_OK : SBN_ERR_CUDA;
 }
 
-// Bytes of the optional workspace of the contraction: the expanded weights
-// when t selects the tensor-core kernel, else none.
+// TMA maps of the compressed 2:4 workspace: kept values [N_out, K/2] in
+// boxes of 128 rows x 64 bytes (64-byte swizzle), metadata [N_pad, K/8] in
+// boxes of 128 rows x 16 bytes (no swizzle).
+sbn_status make_sp_weight_maps(CUtensorMap* tw, CUtensorMap* te, const int8_t* wsp, const uint8_t* esp,
+                               int n_out, int n_pad, int k) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return SBN_ERR_CUDA;
+  cuuint32_t estride[2] = {1, 1};
+  cuuint64_t wdim[2] = {(cuuint64_t)(k / 2), (cuuint64_t)n_out};
+  cuuint64_t wstr[1] = {(cuuint64_t)(k / 2)};
+  cuuint32_t wbox[2] = {(cuuint32_t)(kSpBK / 2), (cuuint32_t)kSpBM};
+  CUresult r = enc(tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(wsp), wdim, wstr, wbox, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return SBN_ERR_CUDA;
+  cuuint64_t edim[2] = {(cuuint64_t)(k / 8), (cuuint64_t)n_pad};
+  cuuint64_t estr[1] = {(cuuint64_t)(k / 8)};
+  cuuint32_t ebox[2] = {(cuuint32_t)(kSpBK / 8), (cuuint32_t)kSpBM};
+  r = enc(te, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(esp), edim, estr, ebox, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SBN_OK : SBN_ERR_CUDA;
+}
+
+// Compressed 2:4 workspace: kept values [N_out, K/2], then (at a 128-byte
+// boundary) the metadata [N_pad, K/8], N_pad = N_out rounded up to 128.
+size_t sp_values_bytes(int32_t k, int32_t n_out) {
+  return ((size_t)n_out * (size_t)(k / 2) + 127) & ~(size_t)127;
+}
+size_t sp_ws_bytes(int32_t k, int32_t n_out) {
+  const size_t n_pad = ((size_t)n_out + kSpBM - 1) / kSpBM * kSpBM;
+  return sp_values_bytes(k, n_out) + n_pad * (size_t)(k / 8);
+}
+
+// Bytes of the optional workspace of the contraction when t selects the
+// tensor-core kernel: room for the dense int8 expansion and for the
+// compressed 2:4 form, whichever is larger; else none.
 size_t bitlinear_ws_bytes(int32_t t, int32_t k, int32_t n_out) {
-  return t > 16 ? (size_t)n_out * (size_t)k : 0;
+  return t > 16 ? std::max((size_t)n_out * (size_t)k, sp_ws_bytes(k, n_out)) : 0;
+}
+
+template <bool ACC, bool TMA_A>
+sbn_status launch_tc_sp(const CUtensorMap& tm, const CUtensorMap& tw, const CUtensorMap& te, const TcParams& p,
+                        int sms, cudaStream_t st) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  auto kern = bl_tc_sp_kernel<ACC, TMA_A>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSpSmemBytes) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  const int tiles = ((p.N + kSpBM - 1) / kSpBM) * ((p.T + kSpBN - 1) / kSpBN);
+  kern<<<std::min(tiles, sms), kTcThreads, kSpSmemBytes, st>>>(tm, tw, te, p);
+  return launch_status();
+}
+
+// 2:4 weights on the sparse tensor-core MMA: expanded once into the
+// compressed workspace (ws non-NULL) or inside the kernel.
+template <bool ACC_OUT>
+sbn_status run_bitlinear_sp(const int8_t* xq, const TcParams& p, void* ws, int sms, cudaStream_t st) {
+  CUtensorMap tm;
+  sbn_status s2 = make_act_tensor_map(&tm, xq, p.T, p.K, kSpBN);
+  if (s2 != SBN_OK) return s2;
+  if (!ws) return launch_tc_sp<ACC_OUT, false>(tm, tm, tm, p, sms, st);
+  const int n_pad = (p.N + kSpBM - 1) / kSpBM * kSpBM;
+  int8_t* wsp = reinterpret_cast<int8_t*>(ws);
+  uint8_t* esp = reinterpret_cast<uint8_t*>(ws) + sp_values_bytes(p.K, p.N);
+  const long long units = (long long)n_pad * (p.K / 16);
+  const int grid = (int)std::max(1LL, std::min((units + 511) / 512, (long long)sms * 4));
+  expand_sparse24_kernel<<<grid, 512, 0, st>>>(p.codes, p.meta, p.N, n_pad, p.K, p.cstride, p.mstride, wsp, esp);
+  if ((s2 = launch_status()) != SBN_OK) return s2;
+  CUtensorMap tw, te;
+  if ((s2 = make_sp_weight_maps(&tw, &te, wsp, esp, p.N, n_pad, p.K)) != SBN_OK) return s2;
+  return launch_tc_sp<ACC_OUT, true>(tm, tw, te, p, sms, st);
 }
 
 template <bool ACC_OUT>
@@ -500,12 +579,13 @@ sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k
     return t <= 8 ? dispatch_decode<8, ACC_OUT>(p, n, m, sms, st)
                   : dispatch_decode<16, ACC_OUT>(p, n, m, sms, st);
   }
-  CUtensorMap tm;
-  const sbn_status st_map = make_act_tensor_map(&tm, xq, t, k);
-  if (st_map != SBN_OK) return st_map;
   TcParams p;
   p.codes = codes; p.meta = meta; p.xs = xs; p.gamma = gamma; p.y = y; p.acc_out = acc;
   p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
+  if (n == 2 && m == 4) return run_bitlinear_sp<ACC_OUT>(xq, p, ws, sms, st);
+  CUtensorMap tm;
+  const sbn_status st_map = make_act_tensor_map(&tm, xq, t, k);
+  if (st_map != SBN_OK) return st_map;
   if (ws) {
     // expand once into the workspace, then TMA both operands
     int8_t* wd = reinterpret_cast<int8_t*>(ws);

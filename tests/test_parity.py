@@ -50,12 +50,46 @@ def test_tensor_core_without_workspace(nm, shape):
 
 
 @pytest.mark.parametrize("which", ["up", "down"])
-def test_prefill_sampled_without_workspace(which):
+def test_prefill_full_without_workspace(which):
+    """Config-3 shapes (2:4, T=4096) with the weights expanded inside the
+    sparse tensor-core kernel: every accumulator and output compared."""
     d = synth.prefill(which)
-    g = run_layer(d["w"], d["x"], d["n"], d["m"], workspace=False)
-    cb, mb, gamma, mask, dense = oracle.quantize_weights(d["w"], d["n"], d["m"])
-    q, s = oracle.quantize_acts(d["x"])
-    _sampled_check(g, q, s, dense, gamma, d["x"].shape[0], d["w"].shape[0], seed=21)
+    full_parity(d["w"], d["x"], d["n"], d["m"], workspace=False)
+
+
+# 2:4 runs on the sparse tensor-core MMA: token tiles of 224, output-feature
+# tiles of 128, K stages of 128 positions; ragged tails on both tile axes
+SPARSE24_SHAPES = [(17, 128, 1), (224, 256, 128), (225, 384, 129), (449, 640, 300), (700, 128, 77),
+                   (300, 2560, 260)]
+
+
+@pytest.mark.parametrize("shape", SPARSE24_SHAPES)
+@pytest.mark.parametrize("ws", [None, False], ids=["workspace", "in_kernel"])
+def test_sparse24_tensor_core_tiles(shape, ws):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=5, tag=f"sp24{shape}")
+    x = synth.activations(t, k, seed=5, tag=f"sp24{shape}", outlier_channels=2)
+    full_parity(w, x, 2, 4, workspace=ws)
+
+
+@pytest.mark.parametrize("ws", [None, False], ids=["workspace", "in_kernel"])
+def test_sparse24_every_group_mask(ws):
+    """Rows whose 2:4 groups run through all six kept-position pairs (each
+    one a different metadata nibble), with kept zeros, ties and both signs."""
+    rng = np.random.default_rng(8)
+    pairs = [(0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3)]
+    n_out, k, t = 150, 768, 230
+    mag = np.full((n_out, k), 0.001, np.float32)
+    for r in range(n_out):
+        for g in range(k // 4):
+            a, b = pairs[(r + 7 * g) % 6]
+            mag[r, 4 * g + a] = rng.choice([0.03, 0.05, 0.0011])   # 0.0011: kept, codes to 0
+            mag[r, 4 * g + b] = rng.choice([0.03, 0.05])
+    mag[::5, :8] = 0.02                                            # four-way ties: keep positions 0, 1
+    sign = np.where(rng.random((n_out, k)) < 0.5, -1.0, 1.0).astype(np.float32)
+    w = ((mag * sign).view(np.uint32) >> 16).astype(np.uint16)
+    x = synth.activations(t, k, seed=8, outlier_channels=2)
+    full_parity(w, x, 2, 4, workspace=ws)
 
 
 def _fused_check(w, x, n, m):
@@ -294,15 +328,11 @@ def _sampled_check(g, q, s, dense, gamma, t, n_out, seed, nsamp=4096):
 
 
 @pytest.mark.parametrize("which", ["up", "down"])
-def test_prefill_sampled(which):
+def test_prefill_full(which):
+    """Config-3 shapes (2:4, T=4096, compressed workspace route): every
+    accumulator and output against the oracle's exact fp64 product."""
     d = synth.prefill(which)
-    w, x, n, m = d["w"], d["x"], d["n"], d["m"]
-    g = run_layer(w, x, n, m)
-    cb, mb, gamma, mask, dense = oracle.quantize_weights(w, n, m)
-    assert_weights_exact(g, cb, mb, gamma)
-    q, s = oracle.quantize_acts(x)
-    assert np.array_equal(g["xq"], q) and np.array_equal(g["s"], s)
-    _sampled_check(g, q, s, dense, gamma, x.shape[0], w.shape[0], seed=11)
+    full_parity(d["w"], d["x"], d["n"], d["m"])
 
 
 @pytest.mark.parametrize("proj", [p for p, _, _ in synth.QWEN05B_PROJ])
