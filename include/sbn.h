@@ -233,7 +233,7 @@ sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k,
  *                 it, and the tensor-core kernel then loads them by TMA like
  *                 the activations: for 2:4 as the compressed operand of the
  *                 sparse MMA (the kept int8 values [n_out, k/2] and their
- *                 4-bit position metadata [n_out rounded up to 128, k/8]),
+ *                 4-bit position metadata [n_out rounded up to 256, k/8]),
  *                 for every other pattern as a dense int8 [n_out, k] matrix.
  *                 Ignored for t <= 16. Its contents are unspecified
  *                 afterwards. Both routes give the same acc and y.
@@ -241,7 +241,9 @@ sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k,
  * (tcgen05.mma.sp), which multiplies only the kept half of each group of
  * four ("Sparse-BitNet ...", Abstract: the 2:4 pattern suits the sparse
  * tensor cores); every other pattern runs the dense INT8 MMA on expanded
- * weights.
+ * weights. With a workspace the MMAs run on CTA pairs (tcgen05 cta_group::2,
+ * 256 weight rows per tile, clusters of two CTAs) where the device can hold
+ * such clusters, else on single CTAs.
  * Errors: SBN_ERR_NULL, SBN_ERR_SHAPE, SBN_ERR_PATTERN, SBN_ERR_ALIGN,
  * SBN_ERR_WORKSPACE (before anything is enqueued); SBN_ERR_CUDA.
  */
@@ -253,7 +255,7 @@ sbn_status sbn_bitlinear(const int8_t* xq, const float* x_scale, int32_t t,
 
 /* Bytes of sbn_bitlinear's optional workspace: when t > 16, the larger of
  * n_out * k (dense expansion) and the compressed 2:4 form
- * (round_up(n_out * k / 2, 128) + round_up(n_out, 128) * k / 8); else 0. */
+ * (round_up(n_out * k / 2, 128) + round_up(n_out, 256) * k / 8); else 0. */
 size_t sbn_bitlinear_workspace_bytes(int32_t t, int32_t k, int32_t n_out);
 
 /*

@@ -47,6 +47,18 @@ SBN_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long limi
   return false;
 }
 
+// One non-blocking probe of the phase of the given parity (no suspension,
+// no time bound): true if it has completed. Callers fall back to mbar_wait.
+SBN_DEVFN bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Bulk copy (no tensor map) of `bytes` (a multiple of 16, both addresses
 // 16-byte aligned) from global to this CTA's shared memory, completing
 // `bytes` transactions on `bar`.

@@ -47,7 +47,6 @@ bl_decode_ent_kernel(const DresParams p) {
   int32_t* s_acc = reinterpret_cast<int32_t*>(dent_smem + L.acc);
   uint8_t* s_x = dent_smem + L.x;
   uint8_t* s_codes = dent_smem + L.codes;
-  uint8_t* s_meta = dent_smem + L.meta;
   uint16_t* s_xbf = reinterpret_cast<uint16_t*>(dent_smem + L.xbf);
   float* s_scale = reinterpret_cast<float*>(dent_smem + L.scale);
 

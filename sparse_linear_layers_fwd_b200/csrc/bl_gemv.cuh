@@ -194,7 +194,6 @@ SBN_DEVFN uint32_t gv_field(const uint32_t (&w)[NW]) {
 template <int MM, int CB, bool DENSE, int I>
 SBN_DEVFN void gv_expand(const uint32_t (&cw)[CB], const uint32_t (&mw)[2], const uint2* s_sel2, uint32_t& w0,
                          uint32_t& w1) {
-  uint32_t v, m8;
   if constexpr (DENSE) {
     // n == m: 8 codes per group, no keep bits; interleave even and odd
     uint32_t ev, od;
@@ -207,7 +206,7 @@ SBN_DEVFN void gv_expand(const uint32_t (&cw)[CB], const uint32_t (&mw)[2], cons
     // odd-indexed codes are cut straight out of the code words
     constexpr int kOff = 4 * CB * I;
     constexpr uint32_t kMask = CB == 1 ? 0x3u : CB == 2 ? 0x33u : 0x333u;
-    m8 = gv_prmt(mw[I / 4], 0u, 0x4440u | (I % 4));
+    const uint32_t m8 = gv_prmt(mw[I / 4], 0u, 0x4440u | (I % 4));
     const uint32_t ev = gv_prmt(kCodeByteTable, 0u, gv_field<kOff, kMask, CB>(cw));
     const uint32_t od = gv_prmt(kCodeByteTable, 0u, gv_field<kOff + 2, kMask, CB>(cw));
     const uint2 sel = s_sel2[m8];
@@ -220,18 +219,19 @@ SBN_DEVFN void gv_expand(const uint32_t (&cw)[CB], const uint32_t (&mw)[2], cons
     const uint32_t u = gv_bits<8 * CB * (I / 2), 8 * CB, CB>(cw);
     const uint32_t mlo = gv_prmt(mw[I / 4], 0u, 0x4440u | ((I & ~1) % 4));
     const int klo = __popc(mlo);
+    uint32_t v;
     if constexpr (I % 2 == 0) {
       v = u & ((1u << (2 * klo)) - 1u);   // klo <= 8
     } else {
       v = u >> (2 * klo);
     }
-    m8 = gv_prmt(mw[I / 4], 0u, 0x4440u | (I % 4));
+    const uint32_t m8 = gv_prmt(mw[I / 4], 0u, 0x4440u | (I % 4));
+    uint32_t ev, od;
+    gv_codes_eo(v, ev, od);
+    const uint2 sel = s_sel2[m8];
+    w0 = gv_prmt(ev, od, sel.x);
+    w1 = gv_prmt(ev, od, sel.y);
   }
-  uint32_t ev, od;
-  gv_codes_eo(v, ev, od);
-  const uint2 sel = s_sel2[m8];
-  w0 = gv_prmt(ev, od, sel.x);
-  w1 = gv_prmt(ev, od, sel.y);
 }
 
 // MM: group size m; CB: code bytes per 16 positions (= 4n/m); NT: token

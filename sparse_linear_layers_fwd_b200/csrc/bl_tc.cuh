@@ -1,4 +1,7 @@
-// Prefill contraction on the 5th-generation tensor cores (tcgen05, sm_100a).
+// Prefill contraction on the 5th-generation tensor cores (tcgen05, sm_100a),
+// without a workspace: the packed weights are expanded in shared memory by
+// producer warps (with a workspace the contraction runs on CTA pairs,
+// bl_tc2.cuh).
 //
 // "Microsoft BitNet 1.58: The Era of 1-Bit Large Language Models", section
 // "The BitLinear Layer", fourth and fifth operations; the Sparse-BitNet page
@@ -123,12 +126,9 @@ SBN_DEVFN uint32_t code_bits(const uint32_t (&cw)[NW], int bit) {
   return s ? ((lo >> s) | (hi << (32 - s))) : lo;
 }
 
-// TMA_A: the weights come expanded (dense int8 [N_out, K], expand_dense.cuh)
-// and warp 0 loads their tiles by TMA as well; the producer warps stay idle.
-template <int MM, int CB, bool DENSE, bool ACC, bool TMA_A>
+template <int MM, int CB, bool DENSE, bool ACC>
 __global__ void __launch_bounds__(kTcThreads, 1)
-bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-             const TcParams p) {
+bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kTcStages * kTcStageBytes);
@@ -145,13 +145,13 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
 
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      // one arrival per producer warp + the TMA thread's (or the TMA thread's alone)
-      mbar_init(&full[s], TMA_A ? 1 : kTcProducers / 32 + 1);
+      // one arrival per producer warp + the TMA thread's
+      mbar_init(&full[s], kTcProducers / 32 + 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], TMA_A ? 2 * kTcEpilogue / 32 : kTcEpilogue / 32);
+      mbar_init(&acc_empty[b], kTcEpilogue / 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -161,7 +161,7 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  if (!DENSE && !TMA_A) {
+  if (!DENSE) {
     for (int i = tid; i < 256 * kTcSelCopies; i += blockDim.x) s_sel[i] = expand_selector((uint32_t)(i / kTcSelCopies));
   }
   tc_fence_before();
@@ -175,14 +175,12 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
       int it = 0;
       for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         const int tok0 = (tile / row_tiles) * kTcBN;
-        const int row0 = (tile % row_tiles) * kTcBM;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kTcStages;
           const uint32_t ph = (it / kTcStages) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[s], TMA_A ? kTcABytes + kTcBBytes : kTcBBytes);
-          if (TMA_A) tma_load_2d(smem + (size_t)s * kTcStageBytes, &tmap_w, kb * kTcBK, row0, &full[s]);
+          mbar_arrive_expect_tx(&full[s], kTcBBytes);
           tma_load_2d(smem + (size_t)s * kTcStageBytes + kTcABytes, &tmap_x, kb * kTcBK, tok0, &full[s]);
         }
         if (!ok) break;
@@ -215,7 +213,7 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
         tc_commit(&acc_full[b]);  // arrives once every MMA of this tile has completed
       }
     }
-  } else if (!TMA_A && warp >= 4 && warp < 12) {
+  } else if (warp >= 4 && warp < 12) {
     // ---- producers: thread (i, h) expands units 4h..4h+3 of row i ----
     const int pi = tid - 128;
     const int i = pi & (kTcBM - 1), h = pi >> 7;
@@ -299,14 +297,12 @@ bl_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__
         if (lane == 0) mbar_arrive(&full[s]);
       }
     }
-  } else if (TMA_A ? (warp >= 4 && warp < 12) : warp >= 12) {
+  } else if (warp >= 12) {
     // ---- epilogue: TMEM -> registers -> y (or acc) ----
-    // warp w reads TMEM lane quadrant w % 4; with TMA_A the idle producer
-    // warps 4-11 drain the accumulator, two per quadrant, each half of the
-    // columns; otherwise warps 12-15 drain all of them
+    // warp w reads TMEM lane quadrant w % 4
     const int q = warp & 3;
-    const int c_first = TMA_A ? ((warp - 4) >> 2) * (kTcBN / 64) : 0;
-    const int c_count = TMA_A ? kTcBN / 64 : kTcBN / 32;
+    const int c_first = 0;
+    const int c_count = kTcBN / 32;
     const int row_in_tile = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const float g = ACC ? 0.f : __ldg(p.gamma);

@@ -28,10 +28,11 @@
 // in issue order, and a slot is rewritten only after the stage's `empty`
 // commit has come back through the load of the next round.
 //
-// Warp roles as in the dense kernel: warp 0 TMA, warp 1 TMEM + MMA thread,
-// and either (TMA_A) warps 4-11 draining the accumulators while A and E also
-// come by TMA from the compressed workspace, or (in-SMEM route) warps 4-11
-// expanding the packed rows into A and E and warps 12-15 draining.
+// This single-CTA kernel is the route without a workspace (the packed rows
+// are expanded in shared memory); with a workspace, 2:4 runs on CTA pairs
+// (bl_tc2.cuh). Warp roles as in the dense kernel: warp 0 TMA of the
+// activations, warp 1 TMEM + MMA thread, warps 4-11 expanding the packed
+// rows into A and E, warps 12-15 draining the accumulators.
 #pragma once
 
 #include <cuda.h>
@@ -127,10 +128,9 @@ SBN_DEVFN void tc_mma_sp_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uin
       : "memory");
 }
 
-template <bool ACC, bool TMA_A>
+template <bool ACC>
 __global__ void __launch_bounds__(kTcThreads, 1)
-bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                const __grid_constant__ CUtensorMap tmap_e, const TcParams p) {
+bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kSpStages * kSpStageBytes);
@@ -146,12 +146,12 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 
   if (tid == 0) {
     for (int s = 0; s < kSpStages; ++s) {
-      mbar_init(&full[s], TMA_A ? 1 : kTcProducers / 32 + 1);
+      mbar_init(&full[s], kTcProducers / 32 + 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], TMA_A ? 2 * kTcEpilogue / 32 : kTcEpilogue / 32);
+      mbar_init(&acc_empty[b], kTcEpilogue / 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -167,23 +167,18 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
   const uint32_t tmem = *s_tmem;
 
   if (warp == 0) {
-    // ---- TMA producer: activations, and with TMA_A the compressed weights + metadata ----
+    // ---- TMA producer of the activation tiles ----
     if (lane == 0) {
       int it = 0;
       for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         const int tok0 = (tile / row_tiles) * kSpBN;
-        const int row0 = (tile % row_tiles) * kSpBM;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kSpStages;
           const uint32_t ph = (it / kSpStages) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
           uint8_t* st = smem + (size_t)s * kSpStageBytes;
-          mbar_arrive_expect_tx(&full[s], TMA_A ? kSpStageBytes : kSpBBytes);
-          if (TMA_A) {
-            tma_load_2d(st, &tmap_w, kb * (kSpBK / 2), row0, &full[s]);
-            tma_load_2d(st + kSpABytes + kSpBBytes, &tmap_e, kb * (kSpBK / 8), row0, &full[s]);
-          }
+          mbar_arrive_expect_tx(&full[s], kSpBBytes);
           tma_load_2d(st + kSpABytes, &tmap_x, kb * kSpBK, tok0, &full[s]);
         }
         if (!ok) break;
@@ -221,7 +216,7 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         tc_commit(&acc_full[b]);
       }
     }
-  } else if (!TMA_A && warp >= 4 && warp < 12) {
+  } else if (warp >= 4 && warp < 12) {
     // ---- producers: thread (i, h) expands units 4h..4h+3 of row i ----
     const int pi = tid - 128;
     const int i = pi & (kSpBM - 1), h = pi >> 7;
@@ -281,14 +276,13 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         if (lane == 0) mbar_arrive(&full[s]);
       }
     }
-  } else if (TMA_A ? (warp >= 4 && warp < 12) : warp >= 12) {
-    // ---- epilogue: TMEM -> registers -> y (or acc) ----
-    // warp w reads TMEM lane quadrant w % 4; with TMA_A two warps share a
-    // quadrant, the first taking 32-column chunks 0-3 and the second 4-6
+  } else if (warp >= 12) {
+    // ---- epilogue: TMEM -> registers -> y (or acc); warp w reads TMEM
+    // lane quadrant w % 4 ----
     constexpr int kChunks = kSpBN / 32;
     const int q = warp & 3;
-    const int c_first = TMA_A ? ((warp - 4) >> 2) * ((kChunks + 1) / 2) : 0;
-    const int c_end = TMA_A ? (((warp - 4) >> 2) ? kChunks : (kChunks + 1) / 2) : kChunks;
+    const int c_first = 0;
+    const int c_end = kChunks;
     const int row_in_tile = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const float g = ACC ? 0.f : __ldg(p.gamma);
@@ -343,10 +337,11 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
   }
 }
 
-// Compressed 2:4 workspace: kept values int8 [N_out, K/2] (a unit's 8 kept
-// codes -> 8 bytes) and metadata [N_pad, K/8] (a unit's keep mask -> 16
-// metadata bits), N_pad = N_out rounded up to 128; pad rows get the
-// metadata of positions (0, 1), so every row the MMA reads is valid.
+// Compressed 2:4 workspace (the operands of the CTA-pair kernel): kept
+// values int8 [N_out, K/2] (a unit's 8 kept codes -> 8 bytes) and metadata
+// [N_pad, K/8] (a unit's keep mask -> 16 metadata bits), N_pad = N_out
+// rounded up to 256; pad rows get the metadata of positions (0, 1), so every
+// row the MMA reads is valid.
 // One thread per unit, grid-stride.
 __global__ void __launch_bounds__(512)
 expand_sparse24_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, int n_out, int n_pad,

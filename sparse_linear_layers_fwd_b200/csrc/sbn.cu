@@ -24,6 +24,7 @@
 #include "bl_decode_ent.cuh"
 #include "expand_dense.cuh"
 #include "bl_tc_sp.cuh"
+#include "bl_tc2.cuh"
 #include "entropy.cuh"
 #include "entropy_pack.cuh"
 #include "bwd.cuh"
@@ -359,16 +360,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-template <int MM, int CB, bool DENSE, bool ACC, bool TMA_A>
-sbn_status launch_tc(const CUtensorMap& tm, const CUtensorMap& tw, const TcParams& p, int sms,
-                     cudaStream_t st) {
+template <int MM, int CB, bool DENSE, bool ACC>
+sbn_status launch_tc(const CUtensorMap& tm, const TcParams& p, int sms, cudaStream_t st) {
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return SBN_ERR_CUDA;
   }
-  auto kern = bl_tc_kernel<MM, CB, DENSE, ACC, TMA_A>;
+  auto kern = bl_tc_kernel<MM, CB, DENSE, ACC>;
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes) !=
         cudaSuccess) {
@@ -378,7 +378,7 @@ sbn_status launch_tc(const CUtensorMap& tm, const CUtensorMap& tw, const TcParam
     attr_set[dev] = true;
   }
   const int tiles = ((p.N + kTcBM - 1) / kTcBM) * ((p.T + kTcBN - 1) / kTcBN);
-  kern<<<std::min(tiles, sms), kTcThreads, kTcSmemBytes, st>>>(tm, tw, p);
+  kern<<<std::min(tiles, sms), kTcThreads, kTcSmemBytes, st>>>(tm, p);
   return launch_status();
 }
 
@@ -386,18 +386,17 @@ sbn_status launch_tc(const CUtensorMap& tm, const CUtensorMap& tw, const TcParam
 template <bool ACC>
 sbn_status dispatch_tc(const CUtensorMap& tm, const TcParams& p, int n, int m, int sms, cudaStream_t st) {
   const int cb = 4 * n / m;
-  const CUtensorMap& unused = tm;
-  if (n == m) return launch_tc<8, 4, true, ACC, false>(tm, unused, p, sms, st);
+  if (n == m) return launch_tc<8, 4, true, ACC>(tm, p, sms, st);
   switch (m * 8 + cb) {
-    case 4 * 8 + 1: return launch_tc<4, 1, false, ACC, false>(tm, unused, p, sms, st);
-    case 4 * 8 + 2: return launch_tc<4, 2, false, ACC, false>(tm, unused, p, sms, st);
-    case 4 * 8 + 3: return launch_tc<4, 3, false, ACC, false>(tm, unused, p, sms, st);
-    case 8 * 8 + 1: return launch_tc<8, 1, false, ACC, false>(tm, unused, p, sms, st);
-    case 8 * 8 + 2: return launch_tc<8, 2, false, ACC, false>(tm, unused, p, sms, st);
-    case 8 * 8 + 3: return launch_tc<8, 3, false, ACC, false>(tm, unused, p, sms, st);
-    case 16 * 8 + 1: return launch_tc<16, 1, false, ACC, false>(tm, unused, p, sms, st);
-    case 16 * 8 + 2: return launch_tc<16, 2, false, ACC, false>(tm, unused, p, sms, st);
-    case 16 * 8 + 3: return launch_tc<16, 3, false, ACC, false>(tm, unused, p, sms, st);
+    case 4 * 8 + 1: return launch_tc<4, 1, false, ACC>(tm, p, sms, st);
+    case 4 * 8 + 2: return launch_tc<4, 2, false, ACC>(tm, p, sms, st);
+    case 4 * 8 + 3: return launch_tc<4, 3, false, ACC>(tm, p, sms, st);
+    case 8 * 8 + 1: return launch_tc<8, 1, false, ACC>(tm, p, sms, st);
+    case 8 * 8 + 2: return launch_tc<8, 2, false, ACC>(tm, p, sms, st);
+    case 8 * 8 + 3: return launch_tc<8, 3, false, ACC>(tm, p, sms, st);
+    case 16 * 8 + 1: return launch_tc<16, 1, false, ACC>(tm, p, sms, st);
+    case 16 * 8 + 2: return launch_tc<16, 2, false, ACC>(tm, p, sms, st);
+    case 16 * 8 + 3: return launch_tc<16, 3, false, ACC>(tm, p, sms, st);
   }
   return SBN_ERR_PATTERN;
 }
@@ -462,7 +461,7 @@ sbn_status make_weight_tensor_map(CUtensorMap* tm, const int8_t* wd, int n_out, 
 }
 
 // TMA maps of the compressed 2:4 workspace: kept values [N_out, K/2] in
-// boxes of 128 rows x 64 bytes (64-byte swizzle), metadata [N_pad, K/8] in
+// boxes of 128 rows x 128 bytes (128-byte swizzle), metadata [N_pad, K/8] in
 // boxes of 128 rows x 16 bytes (no swizzle).
 sbn_status make_sp_weight_maps(CUtensorMap* tw, CUtensorMap* te, const int8_t* wsp, const uint8_t* esp,
                                int n_out, int n_pad, int k) {
@@ -471,10 +470,10 @@ sbn_status make_sp_weight_maps(CUtensorMap* tw, CUtensorMap* te, const int8_t* w
   cuuint32_t estride[2] = {1, 1};
   cuuint64_t wdim[2] = {(cuuint64_t)(k / 2), (cuuint64_t)n_out};
   cuuint64_t wstr[1] = {(cuuint64_t)(k / 2)};
-  cuuint32_t wbox[2] = {(cuuint32_t)(kSpBK / 2), (cuuint32_t)kSpBM};
+  cuuint32_t wbox[2] = {128, (cuuint32_t)kSpBM};
   CUresult r = enc(tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(wsp), wdim, wstr, wbox, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return SBN_ERR_CUDA;
   cuuint64_t edim[2] = {(cuuint64_t)(k / 8), (cuuint64_t)n_pad};
   cuuint64_t estr[1] = {(cuuint64_t)(k / 8)};
@@ -486,13 +485,15 @@ sbn_status make_sp_weight_maps(CUtensorMap* tw, CUtensorMap* te, const int8_t* w
 }
 
 // Compressed 2:4 workspace: kept values [N_out, K/2], then (at a 128-byte
-// boundary) the metadata [N_pad, K/8], N_pad = N_out rounded up to 128.
+// boundary) the metadata [N_pad, K/8], N_pad = N_out rounded up to 256 (the
+// rows of a CTA pair's tile; pad rows carry valid metadata).
+constexpr int kSpRowPad = 256;
+int sp_rows_padded(int32_t n_out) { return (n_out + kSpRowPad - 1) / kSpRowPad * kSpRowPad; }
 size_t sp_values_bytes(int32_t k, int32_t n_out) {
   return ((size_t)n_out * (size_t)(k / 2) + 127) & ~(size_t)127;
 }
 size_t sp_ws_bytes(int32_t k, int32_t n_out) {
-  const size_t n_pad = ((size_t)n_out + kSpBM - 1) / kSpBM * kSpBM;
-  return sp_values_bytes(k, n_out) + n_pad * (size_t)(k / 8);
+  return sp_values_bytes(k, n_out) + (size_t)sp_rows_padded(n_out) * (size_t)(k / 8);
 }
 
 // Bytes of the optional workspace of the contraction when t selects the
@@ -502,16 +503,15 @@ size_t bitlinear_ws_bytes(int32_t t, int32_t k, int32_t n_out) {
   return t > 16 ? std::max((size_t)n_out * (size_t)k, sp_ws_bytes(k, n_out)) : 0;
 }
 
-template <bool ACC, bool TMA_A>
-sbn_status launch_tc_sp(const CUtensorMap& tm, const CUtensorMap& tw, const CUtensorMap& te, const TcParams& p,
-                        int sms, cudaStream_t st) {
+template <bool ACC>
+sbn_status launch_tc_sp(const CUtensorMap& tm, const TcParams& p, int sms, cudaStream_t st) {
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return SBN_ERR_CUDA;
   }
-  auto kern = bl_tc_sp_kernel<ACC, TMA_A>;
+  auto kern = bl_tc_sp_kernel<ACC>;
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSpSmemBytes) !=
         cudaSuccess) {
@@ -521,19 +521,99 @@ sbn_status launch_tc_sp(const CUtensorMap& tm, const CUtensorMap& tw, const CUte
     attr_set[dev] = true;
   }
   const int tiles = ((p.N + kSpBM - 1) / kSpBM) * ((p.T + kSpBN - 1) / kSpBN);
-  kern<<<std::min(tiles, sms), kTcThreads, kSpSmemBytes, st>>>(tm, tw, te, p);
+  kern<<<std::min(tiles, sms), kTcThreads, kSpSmemBytes, st>>>(tm, p);
+  return launch_status();
+}
+
+// CTA pairs of the pair kernel that can be resident at once on this device
+// (clusters of two need both SMs in one GPC); 0 if none.
+template <bool SPARSE, bool ACC>
+int tc2_max_pairs() {
+  static int cached[kMaxDevices];   // 0 unknown, else pairs + 1
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (cached[dev] == 0) {
+    using C = T2Cfg<SPARSE>;
+    auto kern = bl_tc2_kernel<SPARSE, ACC>;
+    int pairs = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2);
+      cfg.blockDim = dim3(kT2Threads);
+      cfg.dynamicSmemBytes = C::SMEM;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg) != cudaSuccess) pairs = 0;
+    }
+    cudaGetLastError();
+    cached[dev] = pairs + 1;
+  }
+  return cached[dev] - 1;
+}
+
+// TMA map of the bf16 output [T, N_out] for the pair kernel's tile stores:
+// boxes of 32 tokens x 32 rows.
+bool make_out_tensor_map(CUtensorMap* ty, const uint16_t* y, int t, int n_out) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)n_out, (cuuint64_t)t};
+  cuuint64_t gstride[1] = {(cuuint64_t)n_out * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estride[2] = {1, 1};
+  return enc(ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(y), gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool SPARSE, bool ACC>
+sbn_status launch_tc2(const CUtensorMap& tm, const CUtensorMap& tw, const CUtensorMap& te, const TcParams& p,
+                      int max_pairs, cudaStream_t st) {
+  using C = T2Cfg<SPARSE>;
+  // tile stores of the output where every row starts on a 16-byte boundary
+  const bool al = !ACC && p.y && (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
+  CUtensorMap ty = tm;   // unused unless y_tma
+  const int y_tma = (al && make_out_tensor_map(&ty, p.y, p.T, p.N)) ? 1 : 0;
+  const int tiles = ((p.N + 255) / 256) * ((p.T + C::BN - 1) / C::BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * std::min(tiles, max_pairs));
+  cfg.blockDim = dim3(kT2Threads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, bl_tc2_kernel<SPARSE, ACC>, tm, tw, te, ty, p, y_tma) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
   return launch_status();
 }
 
 // 2:4 weights on the sparse tensor-core MMA: expanded once into the
-// compressed workspace (ws non-NULL) or inside the kernel.
+// compressed workspace for the CTA-pair kernel (ws non-NULL and pairs can
+// be resident), else inside the single-CTA kernel.
 template <bool ACC_OUT>
 sbn_status run_bitlinear_sp(const int8_t* xq, const TcParams& p, void* ws, int sms, cudaStream_t st) {
   CUtensorMap tm;
-  sbn_status s2 = make_act_tensor_map(&tm, xq, p.T, p.K, kSpBN);
-  if (s2 != SBN_OK) return s2;
-  if (!ws) return launch_tc_sp<ACC_OUT, false>(tm, tm, tm, p, sms, st);
-  const int n_pad = (p.N + kSpBM - 1) / kSpBM * kSpBM;
+  sbn_status s2;
+  const int pairs = ws ? tc2_max_pairs<true, ACC_OUT>() : 0;
+  if (pairs <= 0) {
+    if ((s2 = make_act_tensor_map(&tm, xq, p.T, p.K, kSpBN)) != SBN_OK) return s2;
+    return launch_tc_sp<ACC_OUT>(tm, p, sms, st);
+  }
+  const int n_pad = sp_rows_padded(p.N);
   int8_t* wsp = reinterpret_cast<int8_t*>(ws);
   uint8_t* esp = reinterpret_cast<uint8_t*>(ws) + sp_values_bytes(p.K, p.N);
   const long long units = (long long)n_pad * (p.K / 16);
@@ -542,7 +622,8 @@ sbn_status run_bitlinear_sp(const int8_t* xq, const TcParams& p, void* ws, int s
   if ((s2 = launch_status()) != SBN_OK) return s2;
   CUtensorMap tw, te;
   if ((s2 = make_sp_weight_maps(&tw, &te, wsp, esp, p.N, n_pad, p.K)) != SBN_OK) return s2;
-  return launch_tc_sp<ACC_OUT, true>(tm, tw, te, p, sms, st);
+  if ((s2 = make_act_tensor_map(&tm, xq, p.T, p.K, T2Cfg<true>::HALF)) != SBN_OK) return s2;
+  return launch_tc2<true, ACC_OUT>(tm, tw, te, p, pairs, st);
 }
 
 template <bool ACC_OUT>
@@ -584,17 +665,19 @@ sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k
   p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
   if (n == 2 && m == 4) return run_bitlinear_sp<ACC_OUT>(xq, p, ws, sms, st);
   CUtensorMap tm;
-  const sbn_status st_map = make_act_tensor_map(&tm, xq, t, k);
-  if (st_map != SBN_OK) return st_map;
-  if (ws) {
-    // expand once into the workspace, then TMA both operands
+  const int pairs = ws ? tc2_max_pairs<false, ACC_OUT>() : 0;
+  if (pairs > 0) {
+    // expand once into the workspace, then TMA both operands on CTA pairs
     int8_t* wd = reinterpret_cast<int8_t*>(ws);
     sbn_status s2 = dispatch_expand(codes, meta, n_out, k, n, m, cstride, mstride, wd, sms, st);
     if (s2 != SBN_OK) return s2;
     CUtensorMap tw;
     if ((s2 = make_weight_tensor_map(&tw, wd, n_out, k)) != SBN_OK) return s2;
-    return launch_tc<8, 4, true, ACC_OUT, true>(tm, tw, p, sms, st);
+    if ((s2 = make_act_tensor_map(&tm, xq, t, k, T2Cfg<false>::HALF)) != SBN_OK) return s2;
+    return launch_tc2<false, ACC_OUT>(tm, tw, tw, p, pairs, st);
   }
+  const sbn_status st_map = make_act_tensor_map(&tm, xq, t, k);
+  if (st_map != SBN_OK) return st_map;
   return dispatch_tc<ACC_OUT>(tm, p, n, m, sms, st);
 }
 

@@ -146,8 +146,8 @@ def test_bitlinear_validation(sbn_lib):
     # the optional workspace: used (and checked) only when T > 16
     need = lib.sbn_bitlinear_workspace_bytes(64, 256, 64)
     assert need == 64 * 256
-    # small n_out: the compressed 2:4 form (kept values + metadata of 128 rows) is larger
-    assert lib.sbn_bitlinear_workspace_bytes(17, 256, 16) == 16 * 128 + 128 * 32
+    # small n_out: the compressed 2:4 form (kept values + metadata of 256 rows) is larger
+    assert lib.sbn_bitlinear_workspace_bytes(17, 256, 16) == 16 * 128 + 256 * 32
     assert lib.sbn_bitlinear_workspace_bytes(17, 6912, 2560) == 2560 * 6912
     assert lib.sbn_bitlinear_workspace_bytes(16, 256, 64) == 0
     assert bl(t=64, ws=MIS, ws_bytes=need) == 4
