@@ -664,12 +664,13 @@ def roofline_of(workload, eng, kind, per_kind, peaks, i8_peak):
         ops = sum(call_ops(c[0], eng.layers[c[1]], c[2]) for c in cs)
         dense = sum(2 * c[2] * eng.layers[c[1]][1] * eng.layers[c[1]][0] for c in cs)
         achieved = ops / (us * 1e-6) / 1e12
-        peak, src = i8_peak
+        patterns = {(eng.layers[c[1]][2], eng.layers[c[1]][3]) for c in cs}
+        peak, src, logical = i8_peak.for_patterns(patterns)
         return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
                 "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kind, workload), "kernel": kind,
                 "ops_per_launch": ops // len(cs), "launch_us": round(us / len(cs), 3),
                 "launches_per_call": launches // len(cs), "peak_source": src,
-                "dense_equivalent_frac": round(dense / (us * 1e-6) / 1e12 / peak, 4)}
+                "dense_equivalent_frac": round(dense / (us * 1e-6) / 1e12 / logical, 4)}
     nbytes = sum(call_bytes(c[0], eng.layers[c[1]], c[2]) for c in cs)
     achieved = nbytes / (us * 1e-6) / 1e9
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -704,14 +705,60 @@ def measure_i8_peak(stream, iters=32768, reps=5):
     return ctas * iters * 2 * 128 * 256 * 32 / (best * 1e-3) / 1e12
 
 
-def int8_peak(peaks, measured=None):
-    """The INT8 dense tensor peak: the in-tree tcgen05 kind::i8 probe measured
-    in this run when given, else 2x the measured bf16 figure (the nominal
-    int8 : bf16 ratio), labelled as derived."""
-    if measured:
-        return measured, "measured in this run: in-tree tcgen05 kind::i8 probe (sbn_probe_i8_mma)"
-    return 2.0 * peaks["bf16_tflops"], (f"derived: 2 x {peaks['source']} bf16_tflops {peaks['bf16_tflops']} "
-                                        f"(nominal int8 : bf16 ratio)")
+def measure_i8_sparse_peak(stream, iters=32768, reps=5):
+    """The sparse INT8 rate of the tensor pipe, measured in this run: CTA pairs
+    issuing back-to-back tcgen05.mma.sp.cta_group::2 kind::i8 (256 x 224 x 64
+    logical positions, the 2:4 prefill contraction's instruction and tile)
+    with no loads; the best of `reps` launches. Returns logical TOP/s (2 per
+    multiply-add of all positions; half of them are products of kept
+    weights)."""
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn
+    with torch.cuda.stream(stream):
+        sbn.probe_i8_sparse_mma(iters, stream=stream)   # warm-up
+    stream.synchronize()
+    best = float("inf")
+    pairs = 0
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            pairs = sbn.probe_i8_sparse_mma(iters, stream=stream)
+            e1.record(stream)
+        stream.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    assert sbn.get_device_error() == 0
+    return pairs * iters * 2 * 256 * 224 * 64 / (best * 1e-3) / 1e12
+
+
+class I8Peaks:
+    """The tensor peaks a prefill contraction is measured against, in
+    algorithmic operations (2 per multiply-add of a kept weight):
+    - dense patterns run the dense INT8 MMA on expanded weights: the dense
+      probe's rate (else 2x the measured bf16 figure, labelled derived);
+    - 2:4 runs the sparse MMA, which multiplies only the kept half: half the
+      sparse probe's logical rate (else the dense figure, labelled so)."""
+
+    def __init__(self, peaks, dense_measured=None, sparse_logical=None):
+        if dense_measured:
+            self.dense = (dense_measured, "measured in this run: in-tree tcgen05 kind::i8 probe (sbn_probe_i8_mma)")
+        else:
+            self.dense = (2.0 * peaks["bf16_tflops"], f"derived: 2 x {peaks['source']} bf16_tflops "
+                          f"{peaks['bf16_tflops']} (nominal int8 : bf16 ratio)")
+        self.sparse_logical = sparse_logical
+        if sparse_logical:
+            self.sparse = (sparse_logical / 2.0, "measured in this run: half the logical rate of the in-tree "
+                           "tcgen05.mma.sp kind::i8 probe on CTA pairs (sbn_probe_i8_sparse_mma); 2:4 "
+                           "multiplies only the kept half")
+        else:
+            self.sparse = (self.dense[0], "sparse probe unavailable: dense figure " + self.dense[1])
+
+    def for_patterns(self, patterns):
+        """(peak, source, logical peak) for contractions of these (n, m)."""
+        if patterns and all(nm == (2, 4) for nm in patterns):
+            return self.sparse[0], self.sparse[1], 2.0 * self.sparse[0]
+        return self.dense[0], self.dense[1], self.dense[0]
 
 
 def run_workload(workload, args, rank, world, dev, stream, peaks, i8_peak_src, headline):
@@ -924,7 +971,7 @@ def run_ffn3b(args, dev, stream, peaks, i8_peak_src, with_cpu):
                      "weight_GB/s": round(packed_bytes(n_out, k, n, m) / (bl_us * 1e-6) / 1e9, 1),
                      "quantize_acts_us": round(qa_us, 3)}
                 if t > 16:
-                    peak, _src = i8_peak_src
+                    peak, _src, _lg = i8_peak_src.for_patterns({(n, m)})
                     e["bound"] = "tensor"
                     e["frac"] = round(ops / (bl_us * 1e-6) / 1e12 / peak, 4)
                 else:
@@ -936,9 +983,9 @@ def run_ffn3b(args, dev, stream, peaks, i8_peak_src, with_cpu):
         del wd, xs_dev
         torch.cuda.empty_cache()
     tops = tot_ops / (tot_us * 1e-6) / 1e12
-    peak, src = i8_peak_src
     big = [e for e in entries if e["T"] >= 512]
     dom = max(big, key=lambda e: e["bitlinear_us"])
+    peak, src, _lg = i8_peak_src.for_patterns({tuple(int(v) for v in dom["pattern"].split(":"))})
     out = {"metric": METRIC, "value": round(tops, 3), "unit": "TOPS", "higher_is_better": True,
            "config": {"workload": "ffn3b",
                       "desc": "3B-scale FFN sweep: gate (K=2048, N_out=11008) and down (K=11008, N_out=2048), "
@@ -989,12 +1036,16 @@ def run_ours(args, rank, world, local_rank):
     sbn.lib()
     stream = torch.cuda.Stream(device=dev)
     peaks = load_peaks()
-    i8_measured = None
+    i8_measured = sp_measured = None
     try:
         i8_measured = measure_i8_peak(stream)
     except Exception as ex:  # noqa: BLE001
         print(f"i8 probe unavailable: {ex}", file=sys.stderr)
-    i8 = int8_peak(peaks, i8_measured)
+    try:
+        sp_measured = measure_i8_sparse_peak(stream)
+    except Exception as ex:  # noqa: BLE001
+        print(f"sparse i8 probe unavailable: {ex}", file=sys.stderr)
+    i8 = I8Peaks(peaks, i8_measured, sp_measured)
     head = run_workload(args.workload, args, rank, world, dev, stream, peaks, i8, headline=True)
     extras = {}
     if world == 1 and not args.only:
@@ -1026,7 +1077,9 @@ def run_ours(args, rank, world, local_rank):
             "breakdown_note": head["breakdown_note"], "e2e": head["e2e"],
             "gpu_launches": head["gpu_launches"], "clocks": head["clocks"], "cpu_baseline": cpu,
             "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
-                      "i8_tops": round(i8[0], 1), "i8_source": i8[1]},
+                      "i8_tops": round(i8.dense[0], 1), "i8_source": i8.dense[1],
+                      "i8_sparse_tops_logical": round(i8.sparse_logical, 1) if i8.sparse_logical else None,
+                      "i8_sparse_tops_algorithmic": round(i8.sparse[0], 1), "i8_sparse_source": i8.sparse[1]},
         }
         if extras:
             line["workloads"] = extras

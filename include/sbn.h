@@ -442,6 +442,21 @@ sbn_status sbn_bitlinear_grad_w(const void* dy_bf16, const int8_t* xq,
 sbn_status sbn_probe_i8_mma(int32_t iters, int32_t* ctas, void* stream);
 
 /*
+ * Measurement helper (no counterpart in the method): the sparse INT8 rate of
+ * the tensor pipe on CTA pairs. Launches clusters of two CTAs (one per SM)
+ * on `stream`; in each pair one thread issues `iters` back-to-back
+ * tcgen05.mma.sp.cta_group::2.kind::i8 instructions of M = 256, N = 224,
+ * K = 64 logical positions (2 * 256 * 224 * 64 logical operations each, half
+ * of them products of kept weights; int32 accumulation in tensor memory) on
+ * shared-memory operands with valid 2:4 metadata -- the instruction and tile
+ * shape of the 2:4 prefill contraction, with no loads in between. *pairs
+ * (host) receives the number of pairs; the caller times the launch. Errors:
+ * SBN_ERR_NULL, SBN_ERR_SHAPE (iters outside 1..2^24), SBN_ERR_DEVICE (no
+ * pair can be resident), SBN_ERR_CUDA.
+ */
+sbn_status sbn_probe_i8_sparse_mma(int32_t iters, int32_t* pairs, void* stream);
+
+/*
  * Test hook of the failure detection (no counterpart in the method): runs one
  * of the library's bounded device waits on a condition that never comes, with
  * a limit of limit_ns (1e3..1e8) nanoseconds, on `stream`. which = 0: an

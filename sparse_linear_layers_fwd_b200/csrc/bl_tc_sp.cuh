@@ -341,27 +341,38 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
 // values int8 [N_out, K/2] (a unit's 8 kept codes -> 8 bytes) and metadata
 // [N_pad, K/8] (a unit's keep mask -> 16 metadata bits), N_pad = N_out
 // rounded up to 256; pad rows get the metadata of positions (0, 1), so every
-// row the MMA reads is valid.
-// One thread per unit, grid-stride.
+// row the MMA reads is valid. One thread takes 8 consecutive units of a row
+// (K is a multiple of 128): 16-byte loads of their codes and keep masks,
+// 16-byte stores of 64 value bytes and 16 metadata bytes; grid-stride.
 __global__ void __launch_bounds__(512)
 expand_sparse24_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, int n_out, int n_pad,
                        int k, int cstride, int mstride, int8_t* __restrict__ wsp, uint8_t* __restrict__ esp) {
-  const int upr = k >> 4;
-  const long long total = (long long)n_pad * upr;
+  const int gpr = k >> 7;   // groups of 8 units per row
+  const long long total = (long long)n_pad * gpr;
   for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
        g += (long long)gridDim.x * blockDim.x) {
-    const int row = (int)(g / upr);
-    const int u = (int)(g - (long long)row * upr);
-    uint16_t e = 0x4444u;
+    const int row = (int)(g / gpr);
+    const int gu = (int)(g - (long long)row * gpr);
+    uint4 e = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
     if (row < n_out) {
-      const uint32_t cw = *reinterpret_cast<const uint16_t*>(codes + (size_t)row * cstride + (size_t)u * 2);
-      const uint32_t m16 = *reinterpret_cast<const uint16_t*>(meta + (size_t)row * mstride + (size_t)u * 2);
-      uint32_t q0, q1;
-      codes8_to_s8(cw, q0, q1);
-      *reinterpret_cast<uint2*>(wsp + (size_t)row * (k / 2) + (size_t)u * 8) = make_uint2(q0, q1);
-      e = (uint16_t)sp_meta16(m16);
+      const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + (size_t)row * cstride + (size_t)gu * 16));
+      const uint4 mw = __ldg(reinterpret_cast<const uint4*>(meta + (size_t)row * mstride + (size_t)gu * 16));
+      const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
+      uint4* dst = reinterpret_cast<uint4*>(wsp + (size_t)row * (k / 2) + (size_t)gu * 64);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // two units per 32-bit word of codes: 16 kept values -> 16 bytes
+        uint32_t q0, q1, q2, q3;
+        codes8_to_s8(c4[i] & 0xFFFFu, q0, q1);
+        codes8_to_s8(c4[i] >> 16, q2, q3);
+        dst[i] = make_uint4(q0, q1, q2, q3);
+      }
+      e.x = sp_meta16(mw.x & 0xFFFFu) | (sp_meta16(mw.x >> 16) << 16);
+      e.y = sp_meta16(mw.y & 0xFFFFu) | (sp_meta16(mw.y >> 16) << 16);
+      e.z = sp_meta16(mw.z & 0xFFFFu) | (sp_meta16(mw.z >> 16) << 16);
+      e.w = sp_meta16(mw.w & 0xFFFFu) | (sp_meta16(mw.w >> 16) << 16);
     }
-    *reinterpret_cast<uint16_t*>(esp + (size_t)row * (k / 8) + (size_t)u * 2) = e;
+    *reinterpret_cast<uint4*>(esp + (size_t)row * (k / 8) + (size_t)gu * 16) = e;
   }
 }
 

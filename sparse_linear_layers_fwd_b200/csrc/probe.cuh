@@ -1,4 +1,4 @@
-// Two small kernels that serve measurement and testing, not the method:
+// Small kernels that serve measurement and testing, not the method:
 //
 // * i8_peak_kernel: the tensor pipe's INT8 rate on this part. Every CTA (one
 //   per SM) issues a long run of `tcgen05.mma.cta_group::1.kind::i8` (M = 128,
@@ -15,6 +15,7 @@
 
 #include "async.cuh"
 #include "bl_tc.cuh"
+#include "bl_tc2.cuh"
 #include "common.cuh"
 #include "qw_stream.cuh"
 
@@ -64,6 +65,64 @@ __global__ void __launch_bounds__(kPkThreads, 1) i8_peak_kernel(int iters) {
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kPkTmemCols) : "memory");
+  }
+}
+
+// The sparse INT8 rate on CTA pairs: clusters of two CTAs (one per SM: the
+// shared memory asked for leaves no room for a second CTA, so no CTA waits
+// for another's tensor memory), the leader issuing back-to-back
+// `tcgen05.mma.sp.cta_group::2.kind::i8` of M = 256, N = 224, K = 64 logical
+// positions (the prefill pair kernel's 2:4 instruction), with valid
+// metadata (positions 0 and 1 of every group) copied into tensor memory once.
+// 2 * 256 * 224 * 64 logical operations per instruction, half of them
+// products of kept weights.
+constexpr size_t kPsSmemBytes = 120 * 1024;
+constexpr uint32_t kPsTmemCols = 256;
+__global__ void __launch_bounds__(kPkThreads, 1) i8_sparse_peak_kernel(int iters) {
+  extern __shared__ uint8_t ps_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ps_raw) + 1023) & ~uintptr_t(1023));
+  // A 128 x 128 bytes | B 112 x 128 bytes | metadata 128 x 16 bytes | barrier, TMEM slot
+  constexpr int kA = 128 * 128, kB = 112 * 128, kE = 128 * 16;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kA + kB + kE);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < (kA + kB + kE) / 4; i += kPkThreads) reinterpret_cast<uint32_t*>(smem)[i] = 0x44444444u;
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(s_tmem)),
+                 "r"(kPsTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  if (warp == 1 && lane == 0 && cluster_rank() == 0) {
+    const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem));
+    const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + kA));
+    const uint32_t e = tmem + 224;
+    tc_cp_meta_pair(e, meta_block_desc(smem_u32(smem + kA + kB)));
+    for (int i = 0; i < iters; ++i) {
+      // 32-byte steps of A and 64-byte steps of B inside the swizzled rows
+      tc_mma_pair<true>(tmem, adesc + (uint64_t)(2 * (i & 3)), bdesc + (uint64_t)(4 * (i & 1)),
+                        e + 2u * (uint32_t)(i & 1), i > 0 ? 1u : 0u);
+    }
+    tc_commit_pair(bar);   // arrives in both CTAs once every MMA has completed
+  }
+  if (lane == 0) mbar_wait(bar, 0u);
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kPsTmemCols) : "memory");
   }
 }
 

@@ -616,8 +616,8 @@ sbn_status run_bitlinear_sp(const int8_t* xq, const TcParams& p, void* ws, int s
   const int n_pad = sp_rows_padded(p.N);
   int8_t* wsp = reinterpret_cast<int8_t*>(ws);
   uint8_t* esp = reinterpret_cast<uint8_t*>(ws) + sp_values_bytes(p.K, p.N);
-  const long long units = (long long)n_pad * (p.K / 16);
-  const int grid = (int)std::max(1LL, std::min((units + 511) / 512, (long long)sms * 4));
+  const long long groups = (long long)n_pad * (p.K / 128);
+  const int grid = (int)std::max(1LL, std::min((groups + 511) / 512, (long long)sms * 4));
   expand_sparse24_kernel<<<grid, 512, 0, st>>>(p.codes, p.meta, p.N, n_pad, p.K, p.cstride, p.mstride, wsp, esp);
   if ((s2 = launch_status()) != SBN_OK) return s2;
   CUtensorMap tw, te;
@@ -1289,6 +1289,55 @@ sbn_status sbn_probe_i8_mma(int32_t iters, int32_t* ctas, void* stream) {
   }
   i8_peak_kernel<<<sms, kPkThreads, kPkSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(iters);
   *ctas = sms;
+  return launch_status();
+}
+
+sbn_status sbn_probe_i8_sparse_mma(int32_t iters, int32_t* pairs, void* stream) {
+  if (!pairs) return SBN_ERR_NULL;
+  if (iters < 1 || iters > (1 << 24)) return SBN_ERR_SHAPE;
+  int dev = 0, sms = 0;
+  sbn_status st = check_device(&dev, &sms);
+  if (st != SBN_OK) return st;
+  static int cached[kMaxDevices];   // 0 unknown, else resident pairs + 1
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaFuncSetAttribute(i8_sparse_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPsSmemBytes) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2);
+      cfg.blockDim = dim3(kPkThreads);
+      cfg.dynamicSmemBytes = kPsSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, i8_sparse_peak_kernel, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    cached[dev] = n + 1;
+  }
+  const int np = std::min(cached[dev] - 1, sms / 2);
+  if (np <= 0) return SBN_ERR_DEVICE;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * np);
+  cfg.blockDim = dim3(kPkThreads);
+  cfg.dynamicSmemBytes = kPsSmemBytes;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, i8_sparse_peak_kernel, (int)iters) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  *pairs = np;
   return launch_status();
 }
 

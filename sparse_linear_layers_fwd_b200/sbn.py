@@ -69,6 +69,7 @@ PROTOTYPES = {
                                             _c_p, _c_p]),
     "sbn_bitlinear_grad_w": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p]),
     "sbn_probe_i8_mma": (ctypes.c_int, [_c_i32, ctypes.POINTER(ctypes.c_int32), _c_p]),
+    "sbn_probe_i8_sparse_mma": (ctypes.c_int, [_c_i32, ctypes.POINTER(ctypes.c_int32), _c_p]),
     "sbn_selftest_wait_timeout": (ctypes.c_int, [_c_i32, ctypes.c_int64, _c_p]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
@@ -474,6 +475,16 @@ def probe_i8_mma(iters: int, stream=None) -> int:
     ctas = ctypes.c_int32(0)
     _check(lib().sbn_probe_i8_mma(int(iters), ctypes.byref(ctas), _stream_ptr(stream)), "sbn_probe_i8_mma")
     return int(ctas.value)
+
+
+def probe_i8_sparse_mma(iters: int, stream=None) -> int:
+    """sbn_probe_i8_sparse_mma: launches the sparse INT8 probe on CTA pairs;
+    returns the number of pairs (each issued `iters` MMAs of 2*256*224*64
+    logical operations)."""
+    pairs = ctypes.c_int32(0)
+    _check(lib().sbn_probe_i8_sparse_mma(int(iters), ctypes.byref(pairs), _stream_ptr(stream)),
+           "sbn_probe_i8_sparse_mma")
+    return int(pairs.value)
 
 
 def selftest_wait_timeout(which: int, limit_ns: int, stream=None) -> None:

@@ -113,6 +113,9 @@ def test_probe_and_selftest_validation(sbn_lib):
     assert lib.sbn_probe_i8_mma(10, None, None) == 1
     assert lib.sbn_probe_i8_mma(0, ctypes.byref(ctas), None) == 2
     assert lib.sbn_probe_i8_mma((1 << 24) + 1, ctypes.byref(ctas), None) == 2
+    assert lib.sbn_probe_i8_sparse_mma(10, None, None) == 1
+    assert lib.sbn_probe_i8_sparse_mma(0, ctypes.byref(ctas), None) == 2
+    assert lib.sbn_probe_i8_sparse_mma((1 << 24) + 1, ctypes.byref(ctas), None) == 2
     assert lib.sbn_selftest_wait_timeout(2, 1000000, None) == 2
     assert lib.sbn_selftest_wait_timeout(0, 10, None) == 2
     assert lib.sbn_selftest_wait_timeout(1, 10 ** 9, None) == 2
