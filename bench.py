@@ -166,7 +166,7 @@ WORKLOADS = {
                              "quantize_acts + bitlinear",
                         unit="us", mode="split", qw=True, layers=[(256, 256, 2, 4, [16])]),
 }
-EXTRA_WORKLOADS = ["prefill", "qwen05b", "ffn3b", "layer_small"]
+EXTRA_WORKLOADS = ["prefill", "qwen05b", "ffn3b", "layer_small", "backward"]
 
 
 def workload_layers(workload):
@@ -317,7 +317,8 @@ TRAFFIC_FILES = {
     "quantize_weights": ["qw_stream.cuh", "qw_fused.cuh", "qw.cuh", "async.cuh", "common.cuh"],
     "quantize_acts": ["qa.cuh", "common.cuh"],
     "bitlinear_x": ["bl_gemv.cuh", "bl_decode.cuh", "expand.cuh", "qa.cuh", "async.cuh", "common.cuh"],
-    "bitlinear": ["bl_tc_sp.cuh", "bl_tc.cuh", "expand_dense.cuh", "expand.cuh", "async.cuh", "common.cuh"],
+    "bitlinear": ["bl_tc2.cuh", "bl_tc_sp.cuh", "bl_tc.cuh", "expand_dense.cuh", "expand.cuh", "async.cuh",
+                  "common.cuh"],
     "bitlinear_entropy_x": ["bl_decode_ent.cuh", "bl_decode_res.cuh", "bl_decode.cuh", "entropy.cuh",
                             "expand.cuh", "qa.cuh", "common.cuh"],
     "pack_entropy": ["entropy_pack.cuh", "entropy.cuh", "common.cuh"],
@@ -900,6 +901,62 @@ def run_e2e(workload, eng, data, dev, stream, world, steps):
 # the 3B-scale pattern sweep
 # ---------------------------------------------------------------------------
 
+def run_backward(args, dev, stream, peaks):
+    """The straight-through backward of the prefill up-projection (T = 4096,
+    K = 2560, N_out = 6912, 2:4): sbn_bitlinear_grad_x and sbn_bitlinear_grad_w,
+    each timed back to back over rotated copies of its inputs (more than 3x L2)
+    in one graph. value = 2 * T * K * N_out flops per call, both calls, over
+    their summed time; the roofline divides by the measured bf16 tensor peak."""
+    import torch
+    from sparse_linear_layers_fwd_b200 import sbn, synth
+    l2 = l2_bytes(dev)
+    t, k, n_out, n, m = 4096, 2560, 6912, 2, 4
+    w = to_dev(synth.latent_weights(n_out, k, seed=0, tag="bench_bwd"), dev)
+    x = to_dev(synth.activations(t, k, seed=0, tag="bench_bwd_x"), dev)
+    dy0 = to_dev(synth.activations(t, n_out, seed=0, tag="bench_bwd_dy"), dev)
+    pw = sbn.quantize_weights(w, n, m)
+    xq, xs = sbn.quantize_acts(x)
+    R = int(min(16, max(2, math.ceil(3 * l2 / (2 * t * n_out)))))
+    dys = [dy0] + [dy0.clone() for _ in range(R - 1)]
+    dxs = [torch.empty((t, k), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    dws = [torch.empty((n_out, k), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    with torch.cuda.stream(stream):
+        for i in range(R):
+            sbn.bitlinear_grad_x(dys[i], pw, out=dxs[i], stream=stream)
+            sbn.bitlinear_grad_w(dys[i], xq, xs, out=dws[i], stream=stream)
+    stream.synchronize()
+    gx, gw = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gx, stream=stream):
+        for i in range(R):
+            sbn.bitlinear_grad_x(dys[i], pw, out=dxs[i], stream=stream)
+    with torch.cuda.graph(gw, stream=stream):
+        for i in range(R):
+            sbn.bitlinear_grad_w(dys[i], xq, xs, out=dws[i], stream=stream)
+    reps = max(3, args.kernel_reps)
+    dx_us = replay_ms(gx, stream, reps) * 1e3 / R
+    dw_us = replay_ms(gw, stream, reps) * 1e3 / R
+    del gx, gw
+    assert sbn.get_device_error() == 0
+    flops = 2 * t * k * n_out
+    peak = peaks["bf16_tflops"]
+    tf_x, tf_w = flops / (dx_us * 1e-6) / 1e12, flops / (dw_us * 1e-6) / 1e12
+    value = 2 * flops / ((dx_us + dw_us) * 1e-6) / 1e12
+    dom, dom_us, dom_tf = ("grad_w", dw_us, tf_w) if dw_us >= dx_us else ("grad_x", dx_us, tf_x)
+    return {"metric": "straight-through backward TFLOP/s (dX and dW of one layer)", "value": round(value, 2),
+            "unit": "TFLOP/s", "higher_is_better": True,
+            "config": {"workload": "backward",
+                       "desc": "dX = gamma dY C and dW = dY^T Xd of the prefill up-projection: T=4096, K=2560, "
+                               "N_out=6912, 2:4; 2*T*K*N_out flops per call (pruned positions of C included)",
+                       "l2": f"dY rotated over {R} copies (> 3x L2)"},
+            "calls": {"grad_x": {"us_per_call": round(dx_us, 3), "TFLOP/s": round(tf_x, 2)},
+                      "grad_w": {"us_per_call": round(dw_us, 3), "TFLOP/s": round(tf_w, 2),
+                                 "note": "two bf16 MMAs per step (the scaled dY split into hi and lo parts)"}},
+            "roofline": {"bound": "tensor", "achieved": round(dom_tf, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(dom_tf / peak, 4), "traffic": None, "kernel": dom,
+                         "launch_us": round(dom_us, 3),
+                         "peak_source": f"{peaks['source']} bf16_tflops (MEASURED_PEAKS.json)"}}
+
+
 def run_ffn3b(args, dev, stream, peaks, i8_peak_src, with_cpu):
     """Per pattern: sbn_quantize_weights of gate and down (the per-step dynamic
     mask, timed separately); per (pattern, projection, T): quantize_acts and
@@ -1055,6 +1112,8 @@ def run_ours(args, rank, world, local_rank):
             try:
                 if wl == "ffn3b":
                     extras[wl] = run_ffn3b(args, dev, stream, peaks, i8, with_cpu=not args.no_cpu_baseline)
+                elif wl == "backward":
+                    extras[wl] = run_backward(args, dev, stream, peaks)
                 else:
                     e = run_workload(wl, args, rank, world, dev, stream, peaks, i8, headline=False)
                     if not args.no_cpu_baseline:

@@ -25,6 +25,7 @@
 #include "expand_dense.cuh"
 #include "bl_tc_sp.cuh"
 #include "bl_tc2.cuh"
+#include "bwd_tc.cuh"
 #include "entropy.cuh"
 #include "entropy_pack.cuh"
 #include "bwd.cuh"
@@ -824,9 +825,65 @@ sbn_status launch_bwd_dx(const uint16_t* dy, int t, int k, int n_out, const uint
   return launch_status();
 }
 
+// dX on the tensor cores: dY [T, N_out] by TMA (N_out a multiple of 8, so
+// its rows start on 16-byte boundaries), C expanded by the producer warps.
+template <int MM, int CB, bool DENSE>
+sbn_status launch_bwd_dx_tc(const uint16_t* dy, int t, int k, int n_out, const uint8_t* codes,
+                            const uint8_t* meta, int cstride, int mstride, const float* gamma, uint16_t* dx,
+                            int sms, cudaStream_t st) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  auto kern = bwd_dx_tc_kernel<MM, CB, DENSE>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBxSmemBytes) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return SBN_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return SBN_ERR_CUDA;
+  CUtensorMap tm;
+  cuuint64_t gdim[2] = {(cuuint64_t)n_out, (cuuint64_t)t};
+  cuuint64_t gstride[1] = {(cuuint64_t)n_out * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBxBK, (cuuint32_t)kBxBM};
+  cuuint32_t estride[2] = {1, 1};
+  if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(dy), gdim, gstride, box, estride,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return SBN_ERR_CUDA;
+  BxParams p;
+  p.codes = codes; p.meta = meta; p.gamma = gamma; p.dx = dx;
+  p.T = t; p.K = k; p.N = n_out; p.cstride = cstride; p.mstride = mstride;
+  const int tiles = ((t + kBxBM - 1) / kBxBM) * ((k + kBxBN - 1) / kBxBN);
+  kern<<<std::min(tiles, sms), kTcThreads, kBxSmemBytes, st>>>(tm, p);
+  return launch_status();
+}
+
 sbn_status dispatch_bwd_dx(const uint16_t* dy, int t, int k, int n_out, int n, int m, const uint8_t* codes,
-                           const uint8_t* meta, const float* gamma, uint16_t* dx, cudaStream_t st) {
+                           const uint8_t* meta, const float* gamma, uint16_t* dx, int sms, cudaStream_t st) {
   const int cs = (int)sbn_codes_row_bytes(k, n, m), ms = (int)sbn_meta_row_bytes(k, n, m);
+  if ((n_out % 8) == 0) {
+    if (n == m) return launch_bwd_dx_tc<8, 4, true>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+    switch (m * 8 + 4 * n / m) {
+      case 4 * 8 + 1: return launch_bwd_dx_tc<4, 1, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 4 * 8 + 2: return launch_bwd_dx_tc<4, 2, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 4 * 8 + 3: return launch_bwd_dx_tc<4, 3, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 8 * 8 + 1: return launch_bwd_dx_tc<8, 1, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 8 * 8 + 2: return launch_bwd_dx_tc<8, 2, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 8 * 8 + 3: return launch_bwd_dx_tc<8, 3, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 16 * 8 + 1: return launch_bwd_dx_tc<16, 1, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 16 * 8 + 2: return launch_bwd_dx_tc<16, 2, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+      case 16 * 8 + 3: return launch_bwd_dx_tc<16, 3, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, sms, st);
+    }
+    return SBN_ERR_PATTERN;
+  }
+  // N_out not a multiple of 8: the CUDA-core kernel
   if (n == m) return launch_bwd_dx<8, 4, true>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
   switch (m * 8 + 4 * n / m) {
     case 4 * 8 + 1: return launch_bwd_dx<4, 1, false>(dy, t, k, n_out, codes, meta, cs, ms, gamma, dx, st);
@@ -1057,7 +1114,7 @@ sbn_status sbn_bitlinear_grad_x(const void* dy_bf16, int32_t t, int32_t k, int32
   sbn_status st = check_device(&dev, &sms);
   if (st != SBN_OK) return st;
   return dispatch_bwd_dx(reinterpret_cast<const uint16_t*>(dy_bf16), t, k, n_out, n, m, codes, meta, gamma,
-                         reinterpret_cast<uint16_t*>(dx_bf16), reinterpret_cast<cudaStream_t>(stream));
+                         reinterpret_cast<uint16_t*>(dx_bf16), sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_bitlinear_grad_w(const void* dy_bf16, const int8_t* xq, const float* x_scale, int32_t t,
@@ -1071,6 +1128,25 @@ sbn_status sbn_bitlinear_grad_w(const void* dy_bf16, const int8_t* xq, const flo
   int dev = 0, sms = 0;
   sbn_status st = check_device(&dev, &sms);
   if (st != SBN_OK) return st;
+  if ((n_out % 8) == 0 && t >= 32) {
+    // tensor cores: the scaled dY split into two bf16 parts (2^-18 relative),
+    // which needs at least 32 tokens to stay within the fp32 kernel's bound
+    static bool attr_set[kMaxDevices] = {};
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(bwd_dw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwSmemBytes) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        return SBN_ERR_CUDA;
+      }
+      attr_set[dev] = true;
+    }
+    BwParams p;
+    p.dy = reinterpret_cast<const uint16_t*>(dy_bf16); p.xq = xq; p.xs = x_scale;
+    p.dw = reinterpret_cast<uint16_t*>(dw_bf16); p.T = t; p.K = k; p.N = n_out;
+    const int tiles = ((n_out + kBwBM - 1) / kBwBM) * ((k + kBwBN - 1) / kBwBN);
+    bwd_dw_tc_kernel<<<std::min(tiles, sms), kTcThreads, kBwSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    return launch_status();
+  }
   const dim3 grid(k / kBwTile, (n_out + kBwTile - 1) / kBwTile);
   bwd_dw_kernel<<<grid, kBwThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint16_t*>(dy_bf16), xq, x_scale, t, k, n_out, reinterpret_cast<uint16_t*>(dw_bf16));

@@ -565,6 +565,21 @@ def test_backward_grads(nm, shape):
     _grad_check(w, x, dy, *nm)
 
 
+# N_out a multiple of 8: dX runs on the tensor cores (dY by TMA); token tiles
+# of 128 and position tiles of 256 with ragged tails, feature stages of 64
+BWD_TC_SHAPES = [(130, 384, 136), (300, 640, 72), (17, 256, 520), (257, 256, 8), (64, 1152, 264)]
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (6, 8), (8, 16), (8, 8), (1, 4)])
+@pytest.mark.parametrize("shape", BWD_TC_SHAPES)
+def test_backward_dx_tensor_core_tiles(nm, shape):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=27, tag=f"bwtc{nm}{shape}")
+    x = synth.activations(t, k, seed=27, tag=f"bwtc{nm}{shape}", outlier_channels=2)
+    dy = synth.activations(t, n_out, seed=28, tag=f"dytc{nm}{shape}")
+    _grad_check(w, x, dy, *nm)
+
+
 def test_backward_grads_decode_layer():
     # the decode layer's weights (6912 x 2560, 6:8) with 300 tokens
     w = synth.decode_weights()
