@@ -470,6 +470,20 @@ sbn_status sbn_probe_i8_sparse_mma(int32_t iters, int32_t* pairs, void* stream);
 sbn_status sbn_selftest_wait_timeout(int32_t which, int64_t limit_ns, void* stream);
 
 /*
+ * sbn_set_programmatic_launch -- library-wide launch setting (no counterpart
+ * in the method). Enabled (the default), the kernels of sbn_quantize_acts,
+ * of the contraction for T > 16 (expansion and tensor-core kernels) and of
+ * the decode GEMV are launched with CUDA's programmatic stream
+ * serialization: such a kernel may be scheduled while the previous kernel
+ * on the stream is finishing, and it waits on the device for that kernel to
+ * complete before it reads or writes global memory. Outputs are identical
+ * either way; only the gaps between kernels change. enable = 0 launches
+ * them with plain stream order. Returns the previous setting (1 or 0).
+ * Launches already enqueued keep the setting they were made with.
+ */
+int32_t sbn_set_programmatic_launch(int32_t enable);
+
+/*
  * sbn_get_device_error -- synchronizes `stream`, then reads and clears the
  * device error word of the current device. Returns SBN_OK, SBN_ERR_TIMEOUT
  * (a bounded device wait gave up; the affected outputs are unspecified) or

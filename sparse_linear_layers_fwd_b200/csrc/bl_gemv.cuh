@@ -98,12 +98,6 @@ struct GvParams {
   GvLayout L;             // shared-memory layout (the host's gv_layout)
 };
 
-// Programmatic dependent launch: wait for the grids this one depends on (a
-// no-op when the launch carries no such dependency), and let the next grid
-// on the stream start its launch.
-SBN_DEVFN void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
-SBN_DEVFN void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
-
 // Elementwise max(|a|, |b|) of two bf16 pairs (the sign of each result is
 // the xor of the operands' signs; callers clear it).
 SBN_DEVFN uint32_t gv_absmax2(uint32_t a, uint32_t b) {

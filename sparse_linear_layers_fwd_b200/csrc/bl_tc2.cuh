@@ -18,7 +18,11 @@
 //                 own rows);
 //   dense:        dense MMA on the expanded int8 weights, BN = 256. Per CTA
 //                 and stage two 128 x 128-byte weight blocks and two
-//                 128-row activation blocks.
+//                 128-row activation blocks;
+//   dense NARROW: the same with BN = 128 (two 64-row activation blocks per
+//                 CTA and stage, four stages), for layers whose 256-token
+//                 tiles would leave CTA pairs idle: twice the tiles, each
+//                 with half the MMA work per stage.
 // A stage spans 256 positions because each stage costs the MMA thread one
 // mbarrier wait and one commit, time in which it issues no MMA; at 128
 // positions per stage that was as long as the stage's sparse MMAs. A K that
@@ -65,9 +69,10 @@ constexpr int kT2Threads = 384;         // warps 0-11
 constexpr int kT2Epi = 256;             // warps 4-11
 constexpr uint32_t kT2TmemCols = 512;
 
-template <bool SPARSE>
+template <bool SPARSE, bool NARROW = false>
 struct T2Cfg {
-  static constexpr int BN = SPARSE ? 224 : 256;          // tokens per pair tile (MMA N)
+  static_assert(!(SPARSE && NARROW), "the narrow tile is a dense-MMA configuration");
+  static constexpr int BN = SPARSE ? 224 : NARROW ? 128 : 256;   // tokens per pair tile (MMA N)
   static constexpr int HALF = BN / 2;                    // activation rows per CTA
   static constexpr int ABYTES = SPARSE ? 128 * 128 : 2 * 128 * 128;
   static constexpr int BSUB = HALF * 128;                // activations of one 128-position block
@@ -75,7 +80,7 @@ struct T2Cfg {
   static constexpr int ESUB = 128 * 16;                  // metadata of one 128-position block
   static constexpr int EBYTES = SPARSE ? 2 * ESUB : 0;
   static constexpr int STAGE = ABYTES + BBYTES + EBYTES;
-  static constexpr int STAGES = SPARSE ? 4 : 3;
+  static constexpr int STAGES = (SPARSE || NARROW) ? 4 : 3;
   static constexpr int YBUF = (kT2Epi / 32) * 4096;      // two 32 x 32 bf16 tiles per epilogue warp
   static constexpr int MMAS = SPARSE ? 2 : 4;            // MMAs per 128-position block
   static constexpr uint32_t ECOL = 2 * BN;               // metadata ring after the accumulators
@@ -161,21 +166,21 @@ SBN_DEVFN void tmem_ld_wait(uint32_t (&r)[32]) {
                : "memory");
 }
 
-template <bool SPARSE>
+template <bool SPARSE, uint32_t IDESC>
 SBN_DEVFN void tc_mma_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t tmem_e, uint32_t accumulate) {
   if constexpr (SPARSE) {
     asm volatile(
         "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
         "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], %1, %2, [%6], %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n}\n" ::"r"(
             tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(T2Cfg<true>::IDESC), "r"(accumulate), "r"(0u), "r"(tmem_e)
+        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate), "r"(0u), "r"(tmem_e)
         : "memory");
   } else {
     asm volatile(
         "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
         "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n}\n" ::"r"(
             tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(T2Cfg<false>::IDESC), "r"(accumulate), "r"(0u)
+        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate), "r"(0u)
         : "memory");
   }
 }
@@ -189,12 +194,12 @@ SBN_DEVFN void tc_cp_meta_pair(uint32_t taddr, uint64_t sdesc) {
 // 128 bytes; tmap_y: the bf16 output, boxes of 32 tokens x 32 rows, used when
 // y_tma != 0 (every output row starts on a 16-byte boundary). Launched in
 // clusters of two CTAs; gridDim.x even.
-template <bool SPARSE, bool ACC>
+template <bool SPARSE, bool ACC, bool NARROW>
 __global__ void __launch_bounds__(kT2Threads, 1)
 bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
               const __grid_constant__ CUtensorMap tmap_e, const __grid_constant__ CUtensorMap tmap_y,
               const TcParams p, const int y_tma) {
-  using C = T2Cfg<SPARSE>;
+  using C = T2Cfg<SPARSE, NARROW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ybuf = smem + (size_t)C::STAGES * C::STAGE;
@@ -237,6 +242,10 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   cluster_sync_all();   // the leader's barriers are initialized before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  // the set-up above overlaps the previous grid on the stream; every role
+  // below reads or writes global memory
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ---- TMA producer (both CTAs): every box of a stage is loaded, the
@@ -309,7 +318,7 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             for (int k = 0; k < C::MMAS; ++k) {
               // B advances 64 bytes per sparse MMA (64 positions), 32 per
               // dense one; A 32 bytes either way; metadata two columns
-              tc_mma_pair<SPARSE>(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)((SPARSE ? 4 : 2) * k),
+              tc_mma_pair<SPARSE, C::IDESC>(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)((SPARSE ? 4 : 2) * k),
                                   e_tmem + 4u * (uint32_t)j + 2u * (uint32_t)k,
                                   (ks > 0 || j > 0 || k > 0) ? 1u : 0u);
             }

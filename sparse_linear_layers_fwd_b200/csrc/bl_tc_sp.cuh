@@ -347,6 +347,8 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
 __global__ void __launch_bounds__(512)
 expand_sparse24_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, int n_out, int n_pad,
                        int k, int cstride, int mstride, int8_t* __restrict__ wsp, uint8_t* __restrict__ esp) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int gpr = k >> 7;   // groups of 8 units per row
   const long long total = (long long)n_pad * gpr;
   for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;

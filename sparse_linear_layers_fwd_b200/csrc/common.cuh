@@ -24,6 +24,17 @@ SBN_DEVFN unsigned long long global_ns() {
   return t;
 }
 
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream-serialization attribute may start while the previous grid on the
+// stream is still running: griddep_wait() blocks until that grid has
+// completed and its writes are visible (a no-op for a launch without the
+// attribute), so every such kernel calls it before its first access to
+// global memory. griddep_launch_dependents() lets the next grid on the
+// stream be scheduled once every CTA of this one has called it or exited;
+// that grid's own griddep_wait() still waits for this grid to complete.
+SBN_DEVFN void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+SBN_DEVFN void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // Packed-format geometry. A "unit" is 16 consecutive positions along K; for
 // every supported pattern a unit's kept codes fill a whole number of bytes
 // (4*n/m) and its keep bits fill two bytes.

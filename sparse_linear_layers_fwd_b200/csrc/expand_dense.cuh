@@ -26,6 +26,8 @@ expand_dense_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
   __shared__ uint32_t s_sel[256];
   if (!DENSE) fill_selector_table(s_sel);
   __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
   const int upr = k >> 4;
   const long long total = (long long)n_out * upr;
   for (long long g = (long long)blockIdx.x * kXdThreads + threadIdx.x; g < total;

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kPkThreads, 1) i8_sparse_peak_kernel(int iters
     tc_cp_meta_pair(e, meta_block_desc(smem_u32(smem + kA + kB)));
     for (int i = 0; i < iters; ++i) {
       // 32-byte steps of A and 64-byte steps of B inside the swizzled rows
-      tc_mma_pair<true>(tmem, adesc + (uint64_t)(2 * (i & 3)), bdesc + (uint64_t)(4 * (i & 1)),
+      tc_mma_pair<true, T2Cfg<true>::IDESC>(tmem, adesc + (uint64_t)(2 * (i & 3)), bdesc + (uint64_t)(4 * (i & 1)),
                         e + 2u * (uint32_t)(i & 1), i > 0 ? 1u : 0u);
     }
     tc_commit_pair(bar);   // arrives in both CTAs once every MMA has completed

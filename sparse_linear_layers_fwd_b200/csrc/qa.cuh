@@ -80,6 +80,8 @@ SBN_DEVFN float block_absmax_scale(uint32_t amax) {
 template <int MAXC>
 __global__ void __launch_bounds__(kQaThreads)
 qa_kernel(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+  griddep_wait();
+  griddep_launch_dependents();
   const size_t row = blockIdx.x;
   const uint4* xr = x + row * kc;
   uint4 v[MAXC];
@@ -108,6 +110,8 @@ constexpr int kQawThreads = 128;   // small CTAs: 7 per SM at K = 2560
 template <int MAXC>
 __global__ void __launch_bounds__(kQawThreads)
 qa_warp_kernel(const uint4* __restrict__ x, int t, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int row = blockIdx.x * (kQawThreads / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= t) return;   // whole warps only
@@ -135,6 +139,8 @@ qa_warp_kernel(const uint4* __restrict__ x, int t, int kc, uint2* __restrict__ x
 // Rows too long for registers: two passes over the row (the second from L2).
 __global__ void __launch_bounds__(kQaThreads)
 qa_kernel_long(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+  griddep_wait();
+  griddep_launch_dependents();
   const size_t row = blockIdx.x;
   const uint4* xr = x + row * kc;
   uint32_t amax = 0u;

@@ -8,9 +8,11 @@
 #include "sbn.h"
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstdint>
 #include <cstring>
+#include <utility>
 
 #include "common.cuh"
 #include "qa.cuh"
@@ -76,6 +78,46 @@ sbn_status check_device(int* dev_out, int* sms_out) {
 
 sbn_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? SBN_OK : SBN_ERR_CUDA;
+}
+
+// Programmatic dependent launch of the kernels that call griddep_wait()
+// before touching global memory: each may be scheduled while the previous
+// grid on the stream is finishing, so its launch and set-up (barriers,
+// TMEM, selector tables) overlap that grid's tail. Switched by
+// sbn_set_programmatic_launch; on by default.
+std::atomic<int> g_pdl{1};
+
+// cudaLaunchKernelEx with the programmatic attribute (when switched on) and,
+// for cluster > 1, clusters of `cluster` CTAs along x.
+template <typename... KArgs, typename... Args>
+sbn_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     unsigned cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (g_pdl.load(std::memory_order_relaxed)) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  return SBN_OK;
 }
 
 sbn_status validate_weights_shape(int32_t n_out, int32_t k, int32_t n, int32_t m) {
@@ -230,21 +272,7 @@ sbn_status launch_gemv(const GvParams& p, int grid, size_t smem, cudaStream_t st
     }
     attr_set[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kGvThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
-    cudaGetLastError();
-    return SBN_ERR_CUDA;
-  }
-  return SBN_OK;
+  return launch_ex(kern, dim3((unsigned)grid), dim3(kGvThreads), smem, st, 1, p);
 }
 
 template <int NT, bool ACC, bool XBF>
@@ -409,8 +437,8 @@ sbn_status launch_expand(const uint8_t* codes, const uint8_t* meta, int n_out, i
   const long long units = (long long)n_out * (k / 16);
   const long long want = (units + kXdThreads - 1) / kXdThreads;
   const int grid = (int)std::max(1LL, std::min(want, (long long)sms * 4));
-  expand_dense_kernel<MM, CB, DENSE><<<grid, kXdThreads, 0, st>>>(codes, meta, n_out, k, cstride, mstride, wd);
-  return launch_status();
+  return launch_ex(expand_dense_kernel<MM, CB, DENSE>, dim3(grid), dim3(kXdThreads), 0, st, 1, codes, meta, n_out,
+                   k, cstride, mstride, wd);
 }
 
 sbn_status dispatch_expand(const uint8_t* codes, const uint8_t* meta, int n_out, int k, int n, int m,
@@ -528,7 +556,7 @@ sbn_status launch_tc_sp(const CUtensorMap& tm, const TcParams& p, int sms, cudaS
 
 // CTA pairs of the pair kernel that can be resident at once on this device
 // (clusters of two need both SMs in one GPC); 0 if none.
-template <bool SPARSE, bool ACC>
+template <bool SPARSE, bool ACC, bool NARROW = false>
 int tc2_max_pairs() {
   static int cached[kMaxDevices];   // 0 unknown, else pairs + 1
   int dev = 0;
@@ -537,8 +565,8 @@ int tc2_max_pairs() {
     return 0;
   }
   if (cached[dev] == 0) {
-    using C = T2Cfg<SPARSE>;
-    auto kern = bl_tc2_kernel<SPARSE, ACC>;
+    using C = T2Cfg<SPARSE, NARROW>;
+    auto kern = bl_tc2_kernel<SPARSE, ACC, NARROW>;
     int pairs = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
@@ -574,32 +602,30 @@ bool make_out_tensor_map(CUtensorMap* ty, const uint16_t* y, int t, int n_out) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool SPARSE, bool ACC>
+template <bool SPARSE, bool ACC, bool NARROW = false>
 sbn_status launch_tc2(const CUtensorMap& tm, const CUtensorMap& tw, const CUtensorMap& te, const TcParams& p,
                       int max_pairs, cudaStream_t st) {
-  using C = T2Cfg<SPARSE>;
+  using C = T2Cfg<SPARSE, NARROW>;
   // tile stores of the output where every row starts on a 16-byte boundary
   const bool al = !ACC && p.y && (p.N % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
   CUtensorMap ty = tm;   // unused unless y_tma
   const int y_tma = (al && make_out_tensor_map(&ty, p.y, p.T, p.N)) ? 1 : 0;
   const int tiles = ((p.N + 255) / 256) * ((p.T + C::BN - 1) / C::BN);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * std::min(tiles, max_pairs));
-  cfg.blockDim = dim3(kT2Threads);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, bl_tc2_kernel<SPARSE, ACC>, tm, tw, te, ty, p, y_tma) != cudaSuccess) {
-    cudaGetLastError();
-    return SBN_ERR_CUDA;
-  }
-  return launch_status();
+  return launch_ex(bl_tc2_kernel<SPARSE, ACC, NARROW>, dim3(2 * std::min(tiles, max_pairs)), dim3(kT2Threads), C::SMEM,
+                   st, 2, tm, tw, te, ty, p, y_tma);
+}
+
+// Whether the dense pair kernel should take 128-token tiles: rounds of tiles
+// over the resident pairs, a narrow tile (half the MMA work, the same
+// per-stage cost in the MMA thread) counted as 0.6 of a 256-token one. The
+// narrow tiles win where the wide ones leave pairs idle (few tiles, or a
+// short last round).
+bool tc2_narrow_pays(int t, int n_out, int wide_pairs, int narrow_pairs) {
+  if (narrow_pairs <= 0) return false;
+  const long long rp = (n_out + 255) / 256;
+  const long long wide = rp * ((t + 255) / 256), narrow = rp * ((t + 127) / 128);
+  const long long rw = (wide + wide_pairs - 1) / wide_pairs, rn = (narrow + narrow_pairs - 1) / narrow_pairs;
+  return 6 * rn < 10 * rw;
 }
 
 // 2:4 weights on the sparse tensor-core MMA: expanded once into the
@@ -619,8 +645,9 @@ sbn_status run_bitlinear_sp(const int8_t* xq, const TcParams& p, void* ws, int s
   uint8_t* esp = reinterpret_cast<uint8_t*>(ws) + sp_values_bytes(p.K, p.N);
   const long long groups = (long long)n_pad * (p.K / 128);
   const int grid = (int)std::max(1LL, std::min((groups + 511) / 512, (long long)sms * 4));
-  expand_sparse24_kernel<<<grid, 512, 0, st>>>(p.codes, p.meta, p.N, n_pad, p.K, p.cstride, p.mstride, wsp, esp);
-  if ((s2 = launch_status()) != SBN_OK) return s2;
+  if ((s2 = launch_ex(expand_sparse24_kernel, dim3(grid), dim3(512), 0, st, 1, p.codes, p.meta, p.N, n_pad, p.K,
+                      p.cstride, p.mstride, wsp, esp)) != SBN_OK)
+    return s2;
   CUtensorMap tw, te;
   if ((s2 = make_sp_weight_maps(&tw, &te, wsp, esp, p.N, n_pad, p.K)) != SBN_OK) return s2;
   if ((s2 = make_act_tensor_map(&tm, xq, p.T, p.K, T2Cfg<true>::HALF)) != SBN_OK) return s2;
@@ -674,6 +701,11 @@ sbn_status run_bitlinear(const int8_t* xq, const float* xs, int32_t t, int32_t k
     if (s2 != SBN_OK) return s2;
     CUtensorMap tw;
     if ((s2 = make_weight_tensor_map(&tw, wd, n_out, k)) != SBN_OK) return s2;
+    const int npairs = tc2_max_pairs<false, ACC_OUT, true>();
+    if (tc2_narrow_pays(t, n_out, pairs, npairs)) {
+      if ((s2 = make_act_tensor_map(&tm, xq, t, k, T2Cfg<false, true>::HALF)) != SBN_OK) return s2;
+      return launch_tc2<false, ACC_OUT, true>(tm, tw, tw, p, npairs, st);
+    }
     if ((s2 = make_act_tensor_map(&tm, xq, t, k, T2Cfg<false>::HALF)) != SBN_OK) return s2;
     return launch_tc2<false, ACC_OUT>(tm, tw, tw, p, pairs, st);
   }
@@ -735,25 +767,16 @@ sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, fl
   const uint4* x = reinterpret_cast<const uint4*>(x_bf16);
   uint2* q = reinterpret_cast<uint2*>(xq);
   const int wblocks = (t + kQawThreads / 32 - 1) / (kQawThreads / 32);
-  if (kc <= 32 * 4) {
-    qa_warp_kernel<4><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
-    return launch_status();
-  }
-  if (kc <= 32 * 8) {
-    qa_warp_kernel<8><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
-    return launch_status();
-  }
-  if (kc <= 32 * 10) {   // K <= 2560
-    qa_warp_kernel<10><<<wblocks, kQawThreads, 0, s>>>(x, t, kc, q, x_scale);
-    return launch_status();
-  }
+  const dim3 wg(wblocks), wb(kQawThreads), rg(t), rb(kQaThreads);
+  if (kc <= 32 * 4) return launch_ex(qa_warp_kernel<4>, wg, wb, 0, s, 1, x, t, kc, q, x_scale);
+  if (kc <= 32 * 8) return launch_ex(qa_warp_kernel<8>, wg, wb, 0, s, 1, x, t, kc, q, x_scale);
+  if (kc <= 32 * 10) return launch_ex(qa_warp_kernel<10>, wg, wb, 0, s, 1, x, t, kc, q, x_scale);   // K <= 2560
   const int need = (kc + kQaThreads - 1) / kQaThreads;   // >= 3 here
-  if (need <= 4) qa_kernel<4><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 8) qa_kernel<8><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 12) qa_kernel<12><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else if (need <= 16) qa_kernel<16><<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  else qa_kernel_long<<<t, kQaThreads, 0, s>>>(x, kc, q, x_scale);
-  return launch_status();
+  if (need <= 4) return launch_ex(qa_kernel<4>, rg, rb, 0, s, 1, x, kc, q, x_scale);
+  if (need <= 8) return launch_ex(qa_kernel<8>, rg, rb, 0, s, 1, x, kc, q, x_scale);
+  if (need <= 12) return launch_ex(qa_kernel<12>, rg, rb, 0, s, 1, x, kc, q, x_scale);
+  if (need <= 16) return launch_ex(qa_kernel<16>, rg, rb, 0, s, 1, x, kc, q, x_scale);
+  return launch_ex(qa_kernel_long, rg, rb, 0, s, 1, x, kc, q, x_scale);
 }
 
 // Grid, CTA range and shared memory of the entropy decode; false when the
@@ -1425,6 +1448,10 @@ sbn_status sbn_selftest_wait_timeout(int32_t which, int64_t limit_ns, void* stre
   if (st != SBN_OK) return st;
   wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(which, (unsigned long long)limit_ns);
   return launch_status();
+}
+
+int32_t sbn_set_programmatic_launch(int32_t enable) {
+  return sbn::g_pdl.exchange(enable ? 1 : 0);
 }
 
 sbn_status sbn_get_device_error(void* stream) {

@@ -71,6 +71,7 @@ PROTOTYPES = {
     "sbn_probe_i8_mma": (ctypes.c_int, [_c_i32, ctypes.POINTER(ctypes.c_int32), _c_p]),
     "sbn_probe_i8_sparse_mma": (ctypes.c_int, [_c_i32, ctypes.POINTER(ctypes.c_int32), _c_p]),
     "sbn_selftest_wait_timeout": (ctypes.c_int, [_c_i32, ctypes.c_int64, _c_p]),
+    "sbn_set_programmatic_launch": (_c_i32, [_c_i32]),
     "sbn_get_device_error": (ctypes.c_int, [_c_p]),
 }
 
@@ -427,6 +428,12 @@ def bitlinear_grad_w(dy: torch.Tensor, xq: torch.Tensor, s: torch.Tensor,
     st = lib().sbn_bitlinear_grad_w(_ptr(dy), _ptr(xq), _ptr(s), t, k, n_out, _ptr(out), _stream_ptr(stream))
     _check(st, "sbn_bitlinear_grad_w")
     return out
+
+
+def set_programmatic_launch(enable: bool) -> bool:
+    """sbn_set_programmatic_launch: switch programmatic dependent launch of
+    the library's kernels on or off; returns the previous setting."""
+    return bool(lib().sbn_set_programmatic_launch(1 if enable else 0))
 
 
 def get_device_error(stream=None) -> int:

@@ -72,6 +72,25 @@ def test_sparse24_tensor_core_tiles(shape, ws):
     full_parity(w, x, 2, 4, workspace=ws)
 
 
+# Dense patterns on CTA pairs: 128-token tiles where 256-token ones would
+# leave pairs idle, 256-token tiles otherwise (the host picks by the number
+# of tile rounds); ragged token, row and K tails for both.
+DENSE_PAIR_CASES = [
+    ((1000, 384, 4000), (6, 8)),    # wide tiles: 64 of them fill one round
+    ((300, 640, 520), (4, 8)),      # narrow tiles
+    ((129, 1152, 257), (8, 16)),    # narrow tiles, one token past a tile
+    ((2048, 896, 128), (6, 8)),     # narrow, a single 256-row pair tile half empty
+]
+
+
+@pytest.mark.parametrize("shape,nm", DENSE_PAIR_CASES, ids=[f"{c[0]}_{c[1][0]}of{c[1][1]}" for c in DENSE_PAIR_CASES])
+def test_dense_pair_tiles(shape, nm):
+    t, k, n_out = shape
+    w = synth.latent_weights(n_out, k, seed=6, tag=f"dp{shape}")
+    x = synth.activations(t, k, seed=6, tag=f"dp{shape}", outlier_channels=2)
+    full_parity(w, x, *nm)
+
+
 @pytest.mark.parametrize("ws", [None, False], ids=["workspace", "in_kernel"])
 def test_sparse24_every_group_mask(ws):
     """Rows whose 2:4 groups run through all six kept-position pairs (each
