@@ -95,6 +95,9 @@ struct T2Cfg {
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
+SBN_DEVFN void tma_prefetch_map(const CUtensorMap* tmap) {
+  asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
 SBN_DEVFN uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
@@ -231,6 +234,14 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
+  if (warp == 0 && lane == 0) {
+    // the tensor maps are kernel parameters: fetching them now takes their
+    // first use off the first TMA's path
+    tma_prefetch_map(&tmap_x);
+    tma_prefetch_map(&tmap_w);
+    if (SPARSE) tma_prefetch_map(&tmap_e);
+    if (y_tma) tma_prefetch_map(&tmap_y);
+  }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(s_tmem)),
                  "r"(kT2TmemCols)
@@ -245,7 +256,7 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
   // the set-up above overlaps the previous grid on the stream; every role
   // below reads or writes global memory
   griddep_wait();
-  griddep_launch_dependents();
+  if (pair >= n_tiles) griddep_launch_dependents();
 
   if (warp == 0) {
     // ---- TMA producer (both CTAs): every box of a stage is loaded, the
@@ -380,6 +391,7 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       if (lane == 0) got = mbar_wait(&acc_full[b], (jt >> 1) & 1u) ? 1 : 0;
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) break;
+      if (tile + npairs >= n_tiles) griddep_launch_dependents();   // the last tile's MMAs are done
       tc_fence_after();
       // chunk cc + 1 is read from TMEM while chunk cc is converted and stored
       uint32_t ra[32], rb[32];

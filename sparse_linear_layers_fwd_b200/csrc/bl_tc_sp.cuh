@@ -343,16 +343,28 @@ bl_tc_sp_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
 // rounded up to 256; pad rows get the metadata of positions (0, 1), so every
 // row the MMA reads is valid. One thread takes 8 consecutive units of a row
 // (K is a multiple of 128): 16-byte loads of their codes and keep masks,
-// 16-byte stores of 64 value bytes and 16 metadata bytes; grid-stride.
-__global__ void __launch_bounds__(512)
+// 16-byte stores of 64 value bytes and 16 metadata bytes; a warp takes 32
+// consecutive groups, the chunks dealt out over all CTAs. One CTA of 1024
+// threads per SM (the host requests more than half of an SM's shared memory,
+// unused, to keep a second one off): launched behind the previous
+// contraction, CTAs are placed as its CTAs retire, and several on the SMs
+// freed first would leave the others idle. (The contraction that follows
+// could not share the SM anyway: registers.)
+constexpr int kSpXThreads = 1024;
+constexpr int kSpXExclusiveSmem = 120 * 1024;
+__global__ void __launch_bounds__(kSpXThreads)
 expand_sparse24_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, int n_out, int n_pad,
                        int k, int cstride, int mstride, int8_t* __restrict__ wsp, uint8_t* __restrict__ esp) {
   griddep_wait();
   griddep_launch_dependents();
   const int gpr = k >> 7;   // groups of 8 units per row
   const long long total = (long long)n_pad * gpr;
-  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
-       g += (long long)gridDim.x * blockDim.x) {
+  // chunks of 32 consecutive groups, one per warp, dealt out CTA-first
+  const long long nchunk = (total + 31) / 32;
+  for (long long c = (long long)(threadIdx.x >> 5) * gridDim.x + blockIdx.x; c < nchunk;
+       c += (long long)gridDim.x * (blockDim.x >> 5)) {
+    const long long g = c * 32 + (threadIdx.x & 31);
+    if (g >= total) continue;
     const int row = (int)(g / gpr);
     const int gu = (int)(g - (long long)row * gpr);
     uint4 e = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);

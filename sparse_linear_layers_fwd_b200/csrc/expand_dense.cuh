@@ -7,9 +7,11 @@
 // each weight tile again for every token tile.
 //
 // One thread expands one unit (16 positions of one row) into one 16-byte
-// store; a grid-stride loop over all units, consecutive threads on
-// consecutive units (coalesced reads of codes and keep bits, coalesced
-// 16-byte writes).
+// store; a warp takes 32 consecutive units (coalesced reads of codes and keep
+// bits, coalesced 16-byte writes), the warps' chunks dealt out over all CTAs
+// so that each CTA has a share even when the layer is small. CTAs of 512
+// threads leave room on an SM for the contraction that follows (launched
+// early, it sets up next to them).
 #pragma once
 
 #include "common.cuh"
@@ -30,8 +32,13 @@ expand_dense_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
   griddep_launch_dependents();
   const int upr = k >> 4;
   const long long total = (long long)n_out * upr;
-  for (long long g = (long long)blockIdx.x * kXdThreads + threadIdx.x; g < total;
-       g += (long long)gridDim.x * kXdThreads) {
+  // chunks of 32 consecutive units, one per warp, dealt out CTA-first so that
+  // every CTA (every SM) has work even when the layer is small
+  const long long nchunk = (total + 31) / 32;
+  for (long long c = (long long)(threadIdx.x >> 5) * gridDim.x + blockIdx.x; c < nchunk;
+       c += (long long)gridDim.x * (kXdThreads / 32)) {
+    const long long g = c * 32 + (threadIdx.x & 31);
+    if (g >= total) continue;
     const int row = (int)(g / upr);
     const int u = (int)(g - (long long)row * upr);
     const uint8_t* cp = codes + (size_t)row * cstride + (size_t)u * CB;

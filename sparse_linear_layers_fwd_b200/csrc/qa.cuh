@@ -10,6 +10,10 @@
 // is read from HBM exactly once: max |x| (integer max of the 15 magnitude
 // bits), one IEEE division for the multiplier 127/s, then
 // q = clamp(rint(x * mult), -127, 127).
+// The grid is a full wave (as many CTAs as can be resident on every SM) and
+// the rows are dealt out CTA-first: launched behind another kernel, CTAs are
+// placed as that kernel's CTAs retire, and a full wave still ends up evenly
+// spread, so every SM gets the same number of rows.
 #pragma once
 
 #include "common.cuh"
@@ -79,77 +83,82 @@ SBN_DEVFN float block_absmax_scale(uint32_t amax) {
 // MAXC > 0: the row stays in registers. kc = K / 8 chunks of 16 bytes.
 template <int MAXC>
 __global__ void __launch_bounds__(kQaThreads)
-qa_kernel(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+qa_kernel(const uint4* __restrict__ x, int t, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
   griddep_wait();
   griddep_launch_dependents();
-  const size_t row = blockIdx.x;
-  const uint4* xr = x + row * kc;
-  uint4 v[MAXC];
-  uint32_t amax = 0u;
+  for (size_t row = blockIdx.x; row < (size_t)t; row += gridDim.x) {
+    const uint4* xr = x + row * kc;
+    uint4 v[MAXC];
+    uint32_t amax = 0u;
 #pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int idx = threadIdx.x + c * kQaThreads;
-    v[c] = (idx < kc) ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
-    amax = max(amax, mag_max8(v[c]));
-  }
-  const float s = block_absmax_scale(amax);
-  const float mult = __fdiv_rn(127.0f, s);
-  if (threadIdx.x == 0) scale[row] = s;
-  uint2* qr = xq + row * kc;
+    for (int c = 0; c < MAXC; ++c) {
+      const int idx = threadIdx.x + c * kQaThreads;
+      v[c] = (idx < kc) ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
+      amax = max(amax, mag_max8(v[c]));
+    }
+    const float s = block_absmax_scale(amax);
+    const float mult = __fdiv_rn(127.0f, s);
+    if (threadIdx.x == 0) scale[row] = s;
+    uint2* qr = xq + row * kc;
 #pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int idx = threadIdx.x + c * kQaThreads;
-    if (idx < kc) qr[idx] = quant8(v[c], mult);
+    for (int c = 0; c < MAXC; ++c) {
+      const int idx = threadIdx.x + c * kQaThreads;
+      if (idx < kc) qr[idx] = quant8(v[c], mult);
+    }
+    __syncthreads();   // the reduction's shared words are reused by the next row
   }
 }
 
 // One warp per token row (rows of kc <= 32 * MAXC chunks, K <= 2560): the
 // row in registers, all its loads in flight at once, the maximum reduced in
-// the warp (no block barrier), and one wave of CTAs for thousands of rows.
+// the warp (no block barrier); rows dealt out to warp w of CTA b in the order
+// (w, b), so a full wave covers thousands of rows with each SM's share even.
 constexpr int kQawThreads = 128;   // small CTAs: 7 per SM at K = 2560
 template <int MAXC>
 __global__ void __launch_bounds__(kQawThreads)
 qa_warp_kernel(const uint4* __restrict__ x, int t, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
   griddep_wait();
   griddep_launch_dependents();
-  const int row = blockIdx.x * (kQawThreads / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= t) return;   // whole warps only
-  const uint4* xr = x + (size_t)row * kc;
-  uint4 v[MAXC];
-  uint32_t amax = 0u;
+  for (int row = (threadIdx.x >> 5) * gridDim.x + blockIdx.x; row < t; row += (kQawThreads / 32) * gridDim.x) {
+    const uint4* xr = x + (size_t)row * kc;
+    uint4 v[MAXC];
+    uint32_t amax = 0u;
 #pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int idx = lane + 32 * c;
-    v[c] = (idx < kc) ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
-    amax = max(amax, mag_max8(v[c]));
-  }
-  amax = __reduce_max_sync(0xffffffffu, amax);
-  const float s = fmaxf(__uint_as_float(amax << 16), 1e-5f);
-  const float mult = __fdiv_rn(127.0f, s);
-  if (lane == 0) scale[row] = s;
-  uint2* qr = xq + (size_t)row * kc;
+    for (int c = 0; c < MAXC; ++c) {
+      const int idx = lane + 32 * c;
+      v[c] = (idx < kc) ? __ldg(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
+      amax = max(amax, mag_max8(v[c]));
+    }
+    amax = __reduce_max_sync(0xffffffffu, amax);
+    const float s = fmaxf(__uint_as_float(amax << 16), 1e-5f);
+    const float mult = __fdiv_rn(127.0f, s);
+    if (lane == 0) scale[row] = s;
+    uint2* qr = xq + (size_t)row * kc;
 #pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int idx = lane + 32 * c;
-    if (idx < kc) qr[idx] = quant8(v[c], mult);
+    for (int c = 0; c < MAXC; ++c) {
+      const int idx = lane + 32 * c;
+      if (idx < kc) qr[idx] = quant8(v[c], mult);
+    }
   }
 }
 
 // Rows too long for registers: two passes over the row (the second from L2).
 __global__ void __launch_bounds__(kQaThreads)
-qa_kernel_long(const uint4* __restrict__ x, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
+qa_kernel_long(const uint4* __restrict__ x, int t, int kc, uint2* __restrict__ xq, float* __restrict__ scale) {
   griddep_wait();
   griddep_launch_dependents();
-  const size_t row = blockIdx.x;
-  const uint4* xr = x + row * kc;
-  uint32_t amax = 0u;
-  for (int idx = threadIdx.x; idx < kc; idx += kQaThreads) amax = max(amax, mag_max8(__ldg(xr + idx)));
-  const float s = block_absmax_scale(amax);
-  const float mult = __fdiv_rn(127.0f, s);
-  if (threadIdx.x == 0) scale[row] = s;
-  uint2* qr = xq + row * kc;
-  for (int idx = threadIdx.x; idx < kc; idx += kQaThreads) qr[idx] = quant8(__ldg(xr + idx), mult);
+  for (size_t row = blockIdx.x; row < (size_t)t; row += gridDim.x) {
+    const uint4* xr = x + row * kc;
+    uint32_t amax = 0u;
+    for (int idx = threadIdx.x; idx < kc; idx += kQaThreads) amax = max(amax, mag_max8(__ldg(xr + idx)));
+    const float s = block_absmax_scale(amax);
+    const float mult = __fdiv_rn(127.0f, s);
+    if (threadIdx.x == 0) scale[row] = s;
+    uint2* qr = xq + row * kc;
+    for (int idx = threadIdx.x; idx < kc; idx += kQaThreads) qr[idx] = quant8(__ldg(xr + idx), mult);
+    __syncthreads();   // the reduction's shared words are reused by the next row
+  }
 }
 
 }  // namespace sbn

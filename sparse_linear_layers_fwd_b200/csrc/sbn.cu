@@ -87,6 +87,25 @@ sbn_status launch_status() {
 // sbn_set_programmatic_launch; on by default.
 std::atomic<int> g_pdl{1};
 
+// The dynamic shared-memory limit of a kernel, raised once per device (flags:
+// one per device, owned by the caller's instantiation).
+template <typename K>
+bool set_smem_attr_once(K kern, size_t bytes, bool* flags) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return false;
+  }
+  if (!flags[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    flags[dev] = true;
+  }
+  return true;
+}
+
 // cudaLaunchKernelEx with the programmatic attribute (when switched on) and,
 // for cluster > 1, clusters of `cluster` CTAs along x.
 template <typename... KArgs, typename... Args>
@@ -434,11 +453,10 @@ sbn_status dispatch_tc(const CUtensorMap& tm, const TcParams& p, int n, int m, i
 template <int MM, int CB, bool DENSE>
 sbn_status launch_expand(const uint8_t* codes, const uint8_t* meta, int n_out, int k, int cstride,
                          int mstride, int8_t* wd, int sms, cudaStream_t st) {
-  const long long units = (long long)n_out * (k / 16);
-  const long long want = (units + kXdThreads - 1) / kXdThreads;
-  const int grid = (int)std::max(1LL, std::min(want, (long long)sms * 4));
-  return launch_ex(expand_dense_kernel<MM, CB, DENSE>, dim3(grid), dim3(kXdThreads), 0, st, 1, codes, meta, n_out,
-                   k, cstride, mstride, wd);
+  const long long chunks = ((long long)n_out * (k / 16) + 31) / 32;
+  const int grid = (int)std::max(1LL, std::min(chunks, (long long)sms * 4));
+  return launch_ex(expand_dense_kernel<MM, CB, DENSE>, dim3(grid), dim3(kXdThreads), 0, st, 1, codes, meta, n_out, k,
+                   cstride, mstride, wd);
 }
 
 sbn_status dispatch_expand(const uint8_t* codes, const uint8_t* meta, int n_out, int k, int n, int m,
@@ -643,10 +661,12 @@ sbn_status run_bitlinear_sp(const int8_t* xq, const TcParams& p, void* ws, int s
   const int n_pad = sp_rows_padded(p.N);
   int8_t* wsp = reinterpret_cast<int8_t*>(ws);
   uint8_t* esp = reinterpret_cast<uint8_t*>(ws) + sp_values_bytes(p.K, p.N);
+  static bool attr_set[kMaxDevices] = {};
+  if (!set_smem_attr_once(expand_sparse24_kernel, kSpXExclusiveSmem, attr_set)) return SBN_ERR_CUDA;
   const long long groups = (long long)n_pad * (p.K / 128);
-  const int grid = (int)std::max(1LL, std::min((groups + 511) / 512, (long long)sms * 4));
-  if ((s2 = launch_ex(expand_sparse24_kernel, dim3(grid), dim3(512), 0, st, 1, p.codes, p.meta, p.N, n_pad, p.K,
-                      p.cstride, p.mstride, wsp, esp)) != SBN_OK)
+  const int grid = (int)std::max(1LL, std::min((groups + 31) / 32, (long long)sms));
+  if ((s2 = launch_ex(expand_sparse24_kernel, dim3(grid), dim3(kSpXThreads), kSpXExclusiveSmem, st, 1, p.codes,
+                      p.meta, p.N, n_pad, p.K, p.cstride, p.mstride, wsp, esp)) != SBN_OK)
     return s2;
   CUtensorMap tw, te;
   if ((s2 = make_sp_weight_maps(&tw, &te, wsp, esp, p.N, n_pad, p.K)) != SBN_OK) return s2;
@@ -759,24 +779,51 @@ size_t bitlinear_x_ws_bytes(int32_t t, int32_t k, int32_t n_out) {
   return round_up16((size_t)t * k) + round_up16((size_t)t * 4) + bitlinear_ws_bytes(t, k, n_out);
 }
 
+// CTAs of `kern` (threads per CTA, no dynamic shared memory) resident per SM,
+// cached per device in `cache` (one slot per device, owned by the caller's
+// instantiation); 1 if the query fails.
+template <typename K>
+int resident_ctas(K kern, int threads, int* cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 1;
+  }
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, 0) != cudaSuccess || n < 1) n = 1;
+    cudaGetLastError();
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// A quantize_acts kernel over a full wave of CTAs (at most one per token row);
+// the residency cache is per kernel (the template argument).
+template <auto KERN>
+sbn_status launch_qa(int threads, int t, int sms, cudaStream_t s, const uint4* x, int kc, uint2* q, float* x_scale) {
+  static int cache[kMaxDevices];
+  const long long wave = (long long)resident_ctas(KERN, threads, cache) * sms;
+  const int grid = (int)std::max(1LL, std::min(wave, (long long)t));
+  return launch_ex(KERN, dim3(grid), dim3(threads), 0, s, 1, x, t, kc, q, x_scale);
+}
+
 // One warp per token row up to K = 2560, else one CTA per row (qa.cuh); rows
 // up to 16 * 128 * 8 positions stay in registers.
-sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, float* x_scale,
+sbn_status launch_quantize_acts(const void* x_bf16, int t, int k, int8_t* xq, float* x_scale, int sms,
                                 cudaStream_t s) {
   const int kc = k / 8;
   const uint4* x = reinterpret_cast<const uint4*>(x_bf16);
   uint2* q = reinterpret_cast<uint2*>(xq);
-  const int wblocks = (t + kQawThreads / 32 - 1) / (kQawThreads / 32);
-  const dim3 wg(wblocks), wb(kQawThreads), rg(t), rb(kQaThreads);
-  if (kc <= 32 * 4) return launch_ex(qa_warp_kernel<4>, wg, wb, 0, s, 1, x, t, kc, q, x_scale);
-  if (kc <= 32 * 8) return launch_ex(qa_warp_kernel<8>, wg, wb, 0, s, 1, x, t, kc, q, x_scale);
-  if (kc <= 32 * 10) return launch_ex(qa_warp_kernel<10>, wg, wb, 0, s, 1, x, t, kc, q, x_scale);   // K <= 2560
+  if (kc <= 32 * 4) return launch_qa<qa_warp_kernel<4>>(kQawThreads, t, sms, s, x, kc, q, x_scale);
+  if (kc <= 32 * 8) return launch_qa<qa_warp_kernel<8>>(kQawThreads, t, sms, s, x, kc, q, x_scale);
+  if (kc <= 32 * 10) return launch_qa<qa_warp_kernel<10>>(kQawThreads, t, sms, s, x, kc, q, x_scale);
   const int need = (kc + kQaThreads - 1) / kQaThreads;   // >= 3 here
-  if (need <= 4) return launch_ex(qa_kernel<4>, rg, rb, 0, s, 1, x, kc, q, x_scale);
-  if (need <= 8) return launch_ex(qa_kernel<8>, rg, rb, 0, s, 1, x, kc, q, x_scale);
-  if (need <= 12) return launch_ex(qa_kernel<12>, rg, rb, 0, s, 1, x, kc, q, x_scale);
-  if (need <= 16) return launch_ex(qa_kernel<16>, rg, rb, 0, s, 1, x, kc, q, x_scale);
-  return launch_ex(qa_kernel_long, rg, rb, 0, s, 1, x, kc, q, x_scale);
+  if (need <= 4) return launch_qa<qa_kernel<4>>(kQaThreads, t, sms, s, x, kc, q, x_scale);
+  if (need <= 8) return launch_qa<qa_kernel<8>>(kQaThreads, t, sms, s, x, kc, q, x_scale);
+  if (need <= 12) return launch_qa<qa_kernel<12>>(kQaThreads, t, sms, s, x, kc, q, x_scale);
+  if (need <= 16) return launch_qa<qa_kernel<16>>(kQaThreads, t, sms, s, x, kc, q, x_scale);
+  return launch_qa<qa_kernel_long>(kQaThreads, t, sms, s, x, kc, q, x_scale);
 }
 
 // Grid, CTA range and shared memory of the entropy decode; false when the
@@ -1040,7 +1087,7 @@ sbn_status sbn_quantize_acts(const void* x_bf16, int32_t t, int32_t k, int8_t* x
   int dev = 0, sms = 0;
   sbn_status st = check_device(&dev, &sms);
   if (st != SBN_OK) return st;
-  return launch_quantize_acts(x_bf16, t, k, xq, x_scale, reinterpret_cast<cudaStream_t>(stream));
+  return launch_quantize_acts(x_bf16, t, k, xq, x_scale, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_mask_flips(const uint8_t* meta_a, const uint8_t* meta_b, int32_t n_out, int32_t k,
@@ -1210,7 +1257,7 @@ sbn_status sbn_bitlinear_entropy_x(const void* x_bf16, int32_t t, int32_t k, int
   uint8_t* w8 = reinterpret_cast<uint8_t*>(workspace);
   int8_t* q8 = xq ? xq : reinterpret_cast<int8_t*>(w8);
   float* sc = x_scale ? x_scale : reinterpret_cast<float*>(w8 + round_up16((size_t)t * k));
-  if ((st = launch_quantize_acts(x_bf16, t, k, q8, sc, cs)) != SBN_OK) return st;
+  if ((st = launch_quantize_acts(x_bf16, t, k, q8, sc, sms, cs)) != SBN_OK) return st;
   return launch_bitlinear_entropy<false, false>(q8, sc, nullptr, nullptr, nullptr, t, k, n_out, n, m, ent,
                                                 gamma, y, nullptr, grid, per_cta, smem, cs);
 }
@@ -1261,7 +1308,7 @@ sbn_status sbn_bitlinear_x(const void* x_bf16, int32_t t, int32_t k, int32_t n_o
   int8_t* q8 = xq ? xq : reinterpret_cast<int8_t*>(w8);
   float* sc = x_scale ? x_scale : reinterpret_cast<float*>(w8 + round_up16((size_t)t * k));
   void* rest = w8 + round_up16((size_t)t * k) + round_up16((size_t)t * 4);
-  if ((st = launch_quantize_acts(x_bf16, t, k, q8, sc, cs)) != SBN_OK) return st;
+  if ((st = launch_quantize_acts(x_bf16, t, k, q8, sc, sms, cs)) != SBN_OK) return st;
   return run_bitlinear<false>(q8, sc, t, k, n_out, n, m, codes, meta, gamma,
                               reinterpret_cast<uint16_t*>(y_bf16), nullptr,
                               bitlinear_ws_bytes(t, k, n_out) ? rest : nullptr, sms, cs);

@@ -216,6 +216,21 @@ def test_activation_rounding_ties_quantize_acts():
         assert np.array_equal(xs.cpu().numpy(), sc) and np.array_equal(xq.cpu().numpy(), q)
 
 
+@pytest.mark.parametrize("t,k", [(20000, 128), (9000, 896), (8000, 1536), (6000, 2560), (5000, 3072), (3000, 6912),
+                                 (2000, 12288), (700, 17408)])
+def test_quantize_acts_rows_beyond_one_wave(t, k):
+    """More rows than one wave of CTAs holds: each warp (K <= 2560) or CTA
+    (longer rows) takes several rows in turn."""
+    from sparse_linear_layers_fwd_b200 import sbn
+    import torch
+    x = synth.activations(t, k, seed=3, tag=f"qawave{t}_{k}", outlier_channels=1)
+    q, sc = oracle.quantize_acts(x)
+    xq, xs = sbn.quantize_acts(to_dev_bf16(x))
+    torch.cuda.synchronize()
+    assert np.array_equal(xs.cpu().numpy(), sc), "scales differ"
+    assert np.array_equal(xq.cpu().numpy(), q), "INT8 activations differ"
+
+
 @pytest.mark.parametrize("t,k", [(16, 2560), (9, 640), (1, 1152), (16, 384)])
 def test_activation_rounding_ties_fused(t, k):
     # the fused decode path, 16 (or t) tie scales per call, all of them in turn
