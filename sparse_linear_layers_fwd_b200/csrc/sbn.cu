@@ -633,11 +633,11 @@ sbn_status launch_tc2(const CUtensorMap& tm, const CUtensorMap& tw, const CUtens
                    st, 2, tm, tw, te, ty, p, y_tma);
 }
 
-// Whether the dense pair kernel should take 128-token tiles: rounds of tiles
+// Whether the dense pair kernel should take 128-token tiles: waves of tiles
 // over the resident pairs, a narrow tile (half the MMA work, the same
 // per-stage cost in the MMA thread) counted as 0.6 of a 256-token one. The
 // narrow tiles win where the wide ones leave pairs idle (few tiles, or a
-// short last round).
+// short last wave).
 bool tc2_narrow_pays(int t, int n_out, int wide_pairs, int narrow_pairs) {
   if (narrow_pairs <= 0) return false;
   const long long rp = (n_out + 255) / 256;
