@@ -13,9 +13,9 @@
 //   SPARSE (2:4): sparse MMA, BN = 224. Per CTA and 256-position stage: the
 //                 kept values (128 rows x 128 bytes, 128-byte swizzle), two
 //                 128-position blocks of 112 activation rows (128-byte
-//                 swizzle) and two 128 x 16-byte metadata blocks, which
-//                 tcgen05.cp.cta_group::2 moves into a TMEM ring (each CTA's
-//                 own rows);
+//                 swizzle) and two 128 x 16-byte metadata blocks, which one
+//                 tcgen05.cp.cta_group::2 per stage moves into a TMEM ring
+//                 (each CTA's own rows);
 //   dense:        dense MMA on the expanded int8 weights, BN = 256. Per CTA
 //                 and stage two 128 x 128-byte weight blocks and two
 //                 128-row activation blocks;
@@ -187,6 +187,22 @@ SBN_DEVFN void tc_mma_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint
         : "memory");
   }
 }
+// Both metadata blocks of a stage in one copy: 128 rows x 32 bytes, the two
+// 16-byte halves (block 0 and block 1, 2 KB apart) landing in columns 0-3
+// and 4-7 of the ring slot. No swizzle: core matrices of 8 rows x 16 bytes,
+// the next one along a row 2 KB further (leading offset), the next 8 rows
+// 128 bytes further (stride offset).
+SBN_DEVFN uint64_t meta_stage_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(2048 >> 4) << 16;
+  d |= (uint64_t)(128 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+SBN_DEVFN void tc_cp_meta_stage_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;\n" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 SBN_DEVFN void tc_cp_meta_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;\n" ::"r"(taddr), "l"(sdesc) : "memory");
 }
@@ -301,7 +317,8 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
       const uint32_t a0 = smem_u32(smem);
       const uint64_t adesc0 = sw128_kmajor_desc(a0);
       const uint64_t bdesc0 = sw128_kmajor_desc(a0 + C::ABYTES);
-      const uint64_t edesc0 = meta_block_desc(a0 + C::ABYTES + C::BBYTES);
+      const uint64_t edesc0 = meta_stage_desc(a0 + C::ABYTES + C::BBYTES);
+      static_assert(!SPARSE || C::ESUB == 2048, "the stage copy takes the two metadata blocks 2 KB apart");
       int it = 0, jt = 0;
       bool ok = true;
       for (int tile = pair; tile < n_tiles && ok; tile += npairs, ++jt) {
@@ -316,6 +333,8 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
           if (!mbar_test(&full[s], ph) && !mbar_wait(&full[s], ph)) { ok = false; break; }
           const uint32_t e_tmem = tmem + C::ECOL + 8u * (uint32_t)s;
           const int nsub = (2 * ks + 1 < nkb) ? 2 : 1;
+          // both blocks' metadata (a half stage's second block is zeros)
+          if (SPARSE) tc_cp_meta_stage_pair(e_tmem, edesc0 + (uint64_t)(s * (C::STAGE / 16)));
           for (int j = 0; j < nsub; ++j) {
             // A: sparse, one 128-byte swizzled row of kept values per 256
             // positions (block j at +64 bytes, MMA k at +32 bytes); dense,
@@ -324,7 +343,6 @@ bl_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant_
             const uint64_t so = (uint64_t)(s * (C::STAGE / 16));
             const uint64_t adesc = adesc0 + so + (uint64_t)(SPARSE ? 4 * j : j * (128 * 128 / 16));
             const uint64_t bdesc = bdesc0 + so + (uint64_t)(j * (C::BSUB / 16));
-            if (SPARSE) tc_cp_meta_pair(e_tmem + 4u * (uint32_t)j, edesc0 + so + (uint64_t)(j * (C::ESUB / 16)));
 #pragma unroll
             for (int k = 0; k < C::MMAS; ++k) {
               // B advances 64 bytes per sparse MMA (64 positions), 32 per
