@@ -472,11 +472,11 @@ sbn_status sbn_selftest_wait_timeout(int32_t which, int64_t limit_ns, void* stre
 /*
  * sbn_set_programmatic_launch -- library-wide launch setting (no counterpart
  * in the method). Enabled (the default), the kernels of sbn_quantize_acts,
- * of the contraction for T > 16 (expansion and tensor-core kernels) and of
- * the decode GEMV are launched with CUDA's programmatic stream
- * serialization: such a kernel may be scheduled while the previous kernel
- * on the stream is finishing, and it waits on the device for that kernel to
- * complete before it reads or writes global memory. Outputs are identical
+ * of the contraction for T > 16 with a workspace (the weight expansion and
+ * the CTA-pair kernel) and of the decode GEMV are launched with CUDA's
+ * programmatic stream serialization: such a kernel may be scheduled while
+ * the previous kernel on the stream is finishing, and it waits on the device
+ * for that kernel to complete before it reads or writes global memory. Outputs are identical
  * either way; only the gaps between kernels change. enable = 0 launches
  * them with plain stream order. Returns the previous setting (1 or 0).
  * Launches already enqueued keep the setting they were made with.
